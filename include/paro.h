@@ -1,0 +1,163 @@
+/*
+ * paro.h -- C ABI of the ParoQuant runtime hot path on NVIDIA B200 (sm_100a).
+ *
+ * The path (page "ParoQuant: pairwise rotations that survive deployment"):
+ *   section "A rotation small enough to execute": each stage rotates disjoint
+ *   channel pairs (i, j) by a Givens angle,
+ *       x_i' = cos(t) x_i + sin(t) x_j,   x_j' = -sin(t) x_i + cos(t) x_j,
+ *   K stages are composed and a channel-wise scale follows them; the weight
+ *   transform is folded in and quantised at build time, and the activation
+ *   transform x~ = diag(1/s) R_K ... R_1 x runs right before the INT4 linear;
+ *   section "My reduced-calibration experiment": INT4 weights, group size 128;
+ *   section "From fake quantization to a real TensorRT engine": one rotation
+ *   operator and one group-wise INT4 GEMM operator per linear layer, built
+ *   from weights that were transformed and packed beforehand.
+ *
+ * Conventions shared by every call:
+ *   - Pointers named d_* are DEVICE pointers owned by the caller; the library
+ *     never frees or retains them.  h_* pointers are host pointers.
+ *   - bf16 and fp16 buffers are passed as uint16_t bit patterns.
+ *   - Matrices are dense row-major with no padding.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  Asynchronous device faults surface at the
+ *     caller's next synchronisation.
+ *   - Arguments are validated on the host before anything is enqueued; an
+ *     invalid call enqueues nothing and returns PARO_ERR_INVALID_ARG (bad
+ *     value, null or misaligned pointer) or PARO_ERR_UNSUPPORTED (a valid
+ *     value outside what the kernels implement).  A failed launch returns
+ *     PARO_ERR_CUDA.  paro_last_error() describes the last failure of the
+ *     calling thread.
+ *   - Pair tables: uint16_t pairs[K][d/2][2]; stage k = 0 (R_1) is applied
+ *     first; each stage must be a set of disjoint pairs covering channels
+ *     0..d-1 (a perfect matching).  Kernels check that every index is < d; an
+ *     out-of-range index is skipped and reported through
+ *     paro_get_device_status().  Repeated channels inside a stage are not
+ *     detected and give unspecified (but in-bounds) results.
+ *   - cos_t[K][d/2], sin_t[K][d/2] (fp32) hold cos and sin of each pair's
+ *     angle; scale[d] (fp32, > 0) is the channel scale s, NULL meaning s = 1.
+ *   - Packed weights (layout version 1): qweight uint32 [d_out][d_in/8], the
+ *     4-bit code of input column 8w+e in bits [4e, 4e+4) of word w;
+ *     scales, zeros fp16 [d_out][d_in/128]; the zero point is an integer
+ *     0..15 stored in fp16; the weight is w^ = (q - zero) * scale.
+ *   - Supported sizes: d (= d_in for the rotation) even, 2 <= d <= 49152;
+ *     d_in % 128 == 0 and group_size == 128 for the INT4 calls; d_out % 16 == 0;
+ *     0 <= K <= 16; M >= 0 (M == 0 enqueues nothing and returns PARO_OK).
+ *   - No exception crosses this boundary.  Calls are thread-safe; the only
+ *     library state is one device status word per GPU.
+ */
+#ifndef PARO_H
+#define PARO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define PARO_API __attribute__((visibility("default")))
+#else
+#define PARO_API
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* paro_stream_t; /* the same handle as cudaStream_t */
+
+typedef enum {
+  PARO_OK = 0,
+  PARO_ERR_INVALID_ARG = 1,
+  PARO_ERR_UNSUPPORTED = 2,
+  PARO_ERR_CUDA = 3,
+  PARO_ERR_TIMEOUT = 4
+} paro_status;
+
+/* Layout version of the packed weights described above. */
+PARO_API int paro_weight_layout_version(void);
+
+/* Static English name of a status code. */
+PARO_API const char* paro_status_string(paro_status s);
+
+/* Message of the last failed call on the calling thread ("" if none). */
+PARO_API const char* paro_last_error(void);
+
+/*
+ * Build-time transform and packing ("transform and pack INT4 weights", page
+ * "ParoQuant: pairwise rotations that survive deployment", section "From fake
+ * quantization to a real TensorRT engine"; fold from section "A rotation small
+ * enough to execute").
+ *
+ * For every output row n: w~_n = diag(s) R_K ... R_1 w_n (fp32 arithmetic),
+ * so that W~ x~ = W x; then per group of 128 input columns, in fp32 IEEE
+ * arithmetic with round-half-to-even:
+ *   mn = min(0, min v), mx = max(0, max v), scale = fp16((mx - mn) / 15);
+ *   scale == 0 -> scale = 1, zero = 0; else zero = clamp(rint(-mn / scale), 0, 15);
+ *   q = clamp(rint(v / scale) + zero, 0, 15).
+ * d_W:        fp32 [d_out][d_in], read only.
+ * K, d_pairs, d_cos, d_sin, d_scale: the layer's transform (K == 0 and
+ *             d_scale == NULL pack W itself: the plain INT4 linear).
+ * d_workspace: fp32 [d_out][d_in] scratch for the folded weights; may be NULL
+ *             when K == 0 and d_scale == NULL.  Must not alias d_W.
+ * d_qweight, d_scales, d_zeros: outputs in layout version 1.
+ */
+PARO_API paro_status paro_pack_weights(const float* d_W, int d_out, int d_in, int group_size, int K,
+                              const uint16_t* d_pairs, const float* d_cos, const float* d_sin,
+                              const float* d_scale, float* d_workspace, uint32_t* d_qweight,
+                              uint16_t* d_scales, uint16_t* d_zeros, paro_stream_t stream);
+
+/*
+ * Activation-side transform x~ = diag(1/s) R_K ... R_1 x, per token row (page
+ * "ParoQuant: pairwise rotations that survive deployment", section "A
+ * rotation small enough to execute").  fp32 arithmetic, bf16 in and out
+ * (round to nearest even).
+ * d_x:     bf16 [M][d].    d_x_rot: bf16 [M][d]; may equal d_x (in place).
+ */
+PARO_API paro_status paro_rotate(const uint16_t* d_x, uint16_t* d_x_rot, int M, int d, int K,
+                        const uint16_t* d_pairs, const float* d_cos, const float* d_sin,
+                        const float* d_scale, paro_stream_t stream);
+
+/*
+ * Group-wise INT4 weight-only linear y = x W^T with w^ = (q - zero) * scale
+ * (page "ParoQuant: pairwise rotations that survive deployment", section
+ * "From fake quantization to a real TensorRT engine": the group-wise INT4 GEMM
+ * operator).  fp32 accumulation, bf16 output (round to nearest even).
+ * d_x: bf16 [M][d_in] (already transformed); d_y: bf16 [M][d_out]; d_y must not
+ * overlap any input.
+ */
+PARO_API paro_status paro_w4_linear(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                           const uint16_t* d_zeros, uint16_t* d_y, int M, int d_in, int d_out,
+                           int group_size, paro_stream_t stream);
+
+/* Bytes of device workspace paro_rotate_w4_linear needs for M tokens of width d_in. */
+PARO_API size_t paro_workspace_bytes(int M, int d_in);
+
+/*
+ * The runtime path of one linear layer: the activation transform run right
+ * before the packed INT4 linear (page "ParoQuant: pairwise rotations that
+ * survive deployment", section "A rotation small enough to execute", last
+ * paragraph).  y = (diag(1/s) R_K ... R_1 x) W~^T.  The transformed
+ * activations never leave the GPU as bf16: they are handed to the linear in
+ * fp16 through d_workspace (paro_workspace_bytes(M, d_in) bytes, 256-byte
+ * aligned, caller-owned, contents undefined between calls; two calls that run
+ * at the same time need two workspaces).
+ * d_x: bf16 [M][d_in]; d_y: bf16 [M][d_out], not overlapping any input.
+ */
+PARO_API paro_status paro_rotate_w4_linear(const uint16_t* d_x, int K, const uint16_t* d_pairs,
+                                  const float* d_cos, const float* d_sin, const float* d_scale,
+                                  const uint32_t* d_qweight, const uint16_t* d_scales,
+                                  const uint16_t* d_zeros, uint16_t* d_y, int M, int d_in, int d_out,
+                                  int group_size, void* d_workspace, size_t workspace_bytes,
+                                  paro_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of
+ * the current GPU: PARO_OK, PARO_ERR_INVALID_ARG (a kernel met a pair index
+ * >= d and skipped it) or PARO_ERR_TIMEOUT (a bounded wait gave up).
+ */
+PARO_API paro_status paro_get_device_status(paro_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARO_H */

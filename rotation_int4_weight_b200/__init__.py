@@ -1,0 +1,172 @@
+"""Python binding of libparo, the C ABI of the ParoQuant runtime hot path on B200.
+
+Argument marshalling only: every function forwards device pointers, sizes and
+the current CUDA stream to the entry point of the same name in libparo.so
+(declared in include/paro.h) and raises ParoError on a non-OK status.  Output
+tensors are allocated here with torch when the caller passes none; no step of
+the computation runs in Python.  Importing this module fails loudly when the
+library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "ParoError", "LIB_PATH", "lib", "paro_weight_layout_version", "paro_workspace_bytes",
+    "paro_pack_weights", "paro_rotate", "paro_w4_linear", "paro_rotate_w4_linear",
+    "paro_get_device_status", "EXPORTED",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libparo.so")
+
+# name -> (restype, argtypes) of every entry point of include/paro.h
+_P, _I, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+EXPORTED = {
+    "paro_weight_layout_version": (_I, []),
+    "paro_status_string": (ctypes.c_char_p, [_I]),
+    "paro_last_error": (ctypes.c_char_p, []),
+    "paro_pack_weights": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "paro_rotate": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "paro_w4_linear": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "paro_workspace_bytes": (_S, [_I, _I]),
+    "paro_rotate_w4_linear": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
+    "paro_get_device_status": (_I, [_P]),
+}
+
+
+class ParoError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__(message)
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m rotation_int4_weight_b200._build` "
+            "(there is no fallback implementation)")
+    handle = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in EXPORTED.items():
+        fn = getattr(handle, name)
+        fn.restype = res
+        fn.argtypes = args
+    return handle
+
+
+lib = _load()
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        name = lib.paro_status_string(status).decode()
+        msg = lib.paro_last_error().decode()
+        raise ParoError(status, f"{what}: {name}: {msg}")
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _u16(t: torch.Tensor) -> torch.Tensor:
+    """bf16/fp16/int16/uint16 tensors all pass as 16-bit patterns."""
+    if t.element_size() != 2:
+        raise ValueError(f"expected a 16-bit tensor, got {t.dtype}")
+    return t
+
+
+def paro_weight_layout_version() -> int:
+    return int(lib.paro_weight_layout_version())
+
+
+def paro_workspace_bytes(M: int, d_in: int) -> int:
+    return int(lib.paro_workspace_bytes(M, d_in))
+
+
+def _K(pairs):
+    return 0 if pairs is None else int(pairs.shape[0])
+
+
+def paro_pack_weights(W: torch.Tensor, pairs=None, cos_t=None, sin_t=None, scale=None, *,
+                      group_size: int = 128, workspace=None, qweight=None, scales=None, zeros=None,
+                      stream=None):
+    """Fold the layer's transform into fp32 W [d_out, d_in] and pack it (layout version 1).
+
+    Returns (qweight int32 [d_out, d_in/8], scales fp16 [d_out, G], zeros fp16 [d_out, G]).
+    """
+    d_out, d_in = W.shape
+    dev = W.device
+    K = _K(pairs)
+    if qweight is None:
+        qweight = torch.empty(d_out, d_in // 8, dtype=torch.int32, device=dev)
+    if scales is None:
+        scales = torch.empty(d_out, max(d_in // 128, 1), dtype=torch.float16, device=dev)
+    if zeros is None:
+        zeros = torch.empty_like(scales)
+    if workspace is None and (K > 0 or scale is not None):
+        workspace = torch.empty(d_out, d_in, dtype=torch.float32, device=dev)
+    st = lib.paro_pack_weights(_ptr(W), d_out, d_in, group_size, K, _ptr(pairs), _ptr(cos_t), _ptr(sin_t),
+                               _ptr(scale), _ptr(workspace), _ptr(qweight), _ptr(_u16(scales)),
+                               _ptr(_u16(zeros)), _stream(stream))
+    _check(st, "paro_pack_weights")
+    return qweight, scales, zeros
+
+
+def paro_rotate(x: torch.Tensor, pairs=None, cos_t=None, sin_t=None, scale=None, *, out=None, stream=None):
+    """x~ = diag(1/s) R_K ... R_1 x for bf16 x [M, d]; returns bf16 [M, d] (out may be x)."""
+    M, d = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    st = lib.paro_rotate(_ptr(_u16(x)), _ptr(_u16(out)), M, d, _K(pairs), _ptr(pairs), _ptr(cos_t), _ptr(sin_t),
+                         _ptr(scale), _stream(stream))
+    _check(st, "paro_rotate")
+    return out
+
+
+def paro_w4_linear(x: torch.Tensor, qweight, scales, zeros, *, out=None, group_size: int = 128, stream=None):
+    """y = x W^^T for bf16 x [M, d_in] and packed INT4 weights; returns bf16 [M, d_out]."""
+    M, d_in = x.shape
+    d_out = qweight.shape[0]
+    if out is None:
+        out = torch.empty(M, d_out, dtype=torch.bfloat16, device=x.device)
+    st = lib.paro_w4_linear(_ptr(_u16(x)), _ptr(qweight), _ptr(_u16(scales)), _ptr(_u16(zeros)), _ptr(_u16(out)),
+                            M, d_in, d_out, group_size, _stream(stream))
+    _check(st, "paro_w4_linear")
+    return out
+
+
+def paro_rotate_w4_linear(x: torch.Tensor, pairs, cos_t, sin_t, scale, qweight, scales, zeros, *, out=None,
+                          workspace=None, group_size: int = 128, stream=None):
+    """The runtime path of one linear: transform x, then the packed INT4 linear; bf16 [M, d_out]."""
+    M, d_in = x.shape
+    d_out = qweight.shape[0]
+    if out is None:
+        out = torch.empty(M, d_out, dtype=torch.bfloat16, device=x.device)
+    need = paro_workspace_bytes(M, d_in)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    st = lib.paro_rotate_w4_linear(_ptr(_u16(x)), _K(pairs), _ptr(pairs), _ptr(cos_t), _ptr(sin_t), _ptr(scale),
+                                   _ptr(qweight), _ptr(_u16(scales)), _ptr(_u16(zeros)), _ptr(_u16(out)),
+                                   M, d_in, d_out, group_size, _ptr(workspace), workspace.numel(),
+                                   _stream(stream))
+    _check(st, "paro_rotate_w4_linear")
+    return out
+
+
+def paro_get_device_status(stream=None) -> int:
+    """Synchronise the stream and return/clear the device status word (0 = OK)."""
+    return int(lib.paro_get_device_status(_stream(stream)))

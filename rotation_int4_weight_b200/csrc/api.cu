@@ -1,0 +1,251 @@
+// Host side of the C ABI declared in include/paro.h: argument validation,
+// dispatch to the kernels, the per-device status word and error strings.
+// Every check runs before anything is enqueued, so an invalid call leaves the
+// stream untouched.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "paro_internal.cuh"
+
+namespace {
+
+__device__ int g_paro_status;  // first error met by a kernel on this device (0 = none)
+
+thread_local char t_last_error[512];
+
+paro_status fail(paro_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+paro_status ok() {
+  t_last_error[0] = '\0';
+  return PARO_OK;
+}
+
+paro_status from_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ok();
+  return fail(PARO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+std::atomic<int*> g_status_addr[kMaxDevices];
+
+// Device address of the status word on the current device (looked up once per device).
+int* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  int* p = g_status_addr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_paro_status) != cudaSuccess) return nullptr;
+    p = static_cast<int*>(a);
+    g_status_addr[dev].store(p, std::memory_order_release);
+  }
+  return p;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return na && nb && x < y + nb && y < x + na;
+}
+
+paro_status check_tables(int K, int d, const uint16_t* pairs, const float* c, const float* s,
+                         const float* scale) {
+  if (K < 0) return fail(PARO_ERR_INVALID_ARG, "K = %d is negative", K);
+  if (K > paro::kMaxStages) return fail(PARO_ERR_UNSUPPORTED, "K = %d exceeds %d stages", K, paro::kMaxStages);
+  if (K > 0) {
+    if (!pairs || !c || !s) return fail(PARO_ERR_INVALID_ARG, "K > 0 needs pair, cos and sin tables");
+    if (!aligned(pairs, 4) || !aligned(c, 4) || !aligned(s, 4))
+      return fail(PARO_ERR_INVALID_ARG, "pair/cos/sin tables must be 4-byte aligned");
+  }
+  if (scale && !aligned(scale, 4)) return fail(PARO_ERR_INVALID_ARG, "scale must be 4-byte aligned");
+  (void)d;
+  return PARO_OK;
+}
+
+paro_status check_width(int d) {
+  if (d < 2 || (d & 1)) return fail(PARO_ERR_INVALID_ARG, "d = %d must be even and >= 2", d);
+  if (d > paro::kMaxDim) return fail(PARO_ERR_UNSUPPORTED, "d = %d exceeds %d", d, paro::kMaxDim);
+  return PARO_OK;
+}
+
+paro_status check_linear_shape(int M, int d_in, int d_out, int group_size) {
+  if (M < 0) return fail(PARO_ERR_INVALID_ARG, "M = %d is negative", M);
+  if (group_size <= 0) return fail(PARO_ERR_INVALID_ARG, "group_size = %d", group_size);
+  if (group_size != paro::kGroup) return fail(PARO_ERR_UNSUPPORTED, "group_size = %d (only 128)", group_size);
+  if (d_in <= 0 || d_in % paro::kGroup)
+    return fail(PARO_ERR_INVALID_ARG, "d_in = %d must be a positive multiple of 128", d_in);
+  if (d_out <= 0 || d_out % 16)
+    return fail(d_out <= 0 ? PARO_ERR_INVALID_ARG : PARO_ERR_UNSUPPORTED,
+                "d_out = %d must be a positive multiple of 16", d_out);
+  return PARO_OK;
+}
+
+paro_status check_weights(const uint32_t* qweight, const uint16_t* scales, const uint16_t* zeros) {
+  if (!qweight || !scales || !zeros) return fail(PARO_ERR_INVALID_ARG, "null weight pointer");
+  if (!aligned(qweight, 16)) return fail(PARO_ERR_INVALID_ARG, "qweight must be 16-byte aligned");
+  if (!aligned(scales, 2) || !aligned(zeros, 2))
+    return fail(PARO_ERR_INVALID_ARG, "scales/zeros must be 2-byte aligned");
+  return PARO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int paro_weight_layout_version(void) { return 1; }
+
+const char* paro_status_string(paro_status s) {
+  switch (s) {
+    case PARO_OK: return "PARO_OK";
+    case PARO_ERR_INVALID_ARG: return "PARO_ERR_INVALID_ARG";
+    case PARO_ERR_UNSUPPORTED: return "PARO_ERR_UNSUPPORTED";
+    case PARO_ERR_CUDA: return "PARO_ERR_CUDA";
+    case PARO_ERR_TIMEOUT: return "PARO_ERR_TIMEOUT";
+  }
+  return "PARO_ERR_UNKNOWN";
+}
+
+const char* paro_last_error(void) { return t_last_error; }
+
+paro_status paro_pack_weights(const float* d_W, int d_out, int d_in, int group_size, int K,
+                              const uint16_t* d_pairs, const float* d_cos, const float* d_sin,
+                              const float* d_scale, float* d_workspace, uint32_t* d_qweight,
+                              uint16_t* d_scales, uint16_t* d_zeros, paro_stream_t stream) {
+  paro_status st;
+  if (d_out <= 0) return fail(PARO_ERR_INVALID_ARG, "d_out = %d must be positive", d_out);
+  if (group_size <= 0) return fail(PARO_ERR_INVALID_ARG, "group_size = %d", group_size);
+  if (group_size != paro::kGroup) return fail(PARO_ERR_UNSUPPORTED, "group_size = %d (only 128)", group_size);
+  if (d_in <= 0 || d_in % paro::kGroup)
+    return fail(PARO_ERR_INVALID_ARG, "d_in = %d must be a positive multiple of 128", d_in);
+  if ((st = check_tables(K, d_in, d_pairs, d_cos, d_sin, d_scale)) != PARO_OK) return st;
+  if (!d_W || !aligned(d_W, 16)) return fail(PARO_ERR_INVALID_ARG, "W must be non-null and 16-byte aligned");
+  if ((st = check_weights(d_qweight, d_scales, d_zeros)) != PARO_OK) return st;
+  const bool transform = K > 0 || d_scale != nullptr;
+  const size_t wbytes = (size_t)d_out * d_in * sizeof(float);
+  if (transform) {
+    if ((st = check_width(d_in)) != PARO_OK) return st;
+    if (!d_workspace || !aligned(d_workspace, 16))
+      return fail(PARO_ERR_INVALID_ARG, "a transform needs a 16-byte aligned fp32 [d_out][d_in] workspace");
+    if (overlap(d_workspace, wbytes, d_W, wbytes)) return fail(PARO_ERR_INVALID_ARG, "workspace overlaps W");
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const float* src = d_W;
+  if (transform) {
+    int* status = status_ptr();
+    if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
+    cudaError_t e = paro::launch_fold_weights(d_W, d_workspace, d_out, d_in, K, d_pairs, d_cos, d_sin,
+                                              d_scale, status, s);
+    if (e != cudaSuccess) return from_cuda(e, "fold launch");
+    src = d_workspace;
+  }
+  cudaError_t e = paro::launch_quantize_pack(src, d_out, d_in, d_qweight, reinterpret_cast<__half*>(d_scales),
+                                             reinterpret_cast<__half*>(d_zeros), s);
+  return from_cuda(e, "quantize/pack launch");
+}
+
+paro_status paro_rotate(const uint16_t* d_x, uint16_t* d_x_rot, int M, int d, int K,
+                        const uint16_t* d_pairs, const float* d_cos, const float* d_sin,
+                        const float* d_scale, paro_stream_t stream) {
+  paro_status st;
+  if (M < 0) return fail(PARO_ERR_INVALID_ARG, "M = %d is negative", M);
+  if ((st = check_width(d)) != PARO_OK) return st;
+  if ((st = check_tables(K, d, d_pairs, d_cos, d_sin, d_scale)) != PARO_OK) return st;
+  if (M == 0) return ok();
+  if (!d_x || !d_x_rot) return fail(PARO_ERR_INVALID_ARG, "null activation pointer");
+  if (!aligned(d_x, 16) || !aligned(d_x_rot, 16)) return fail(PARO_ERR_INVALID_ARG, "x and x_rot must be 16-byte aligned");
+  const size_t xb = (size_t)M * d * 2;
+  if (d_x != d_x_rot && overlap(d_x, xb, d_x_rot, xb))
+    return fail(PARO_ERR_INVALID_ARG, "x_rot partially overlaps x (only exact in-place is allowed)");
+  int* status = status_ptr();
+  if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
+  cudaError_t e = paro::launch_rotate_act(d_x, d_x_rot, 0, M, d, K, d_pairs, d_cos, d_sin, d_scale, status,
+                                          reinterpret_cast<cudaStream_t>(stream), false);
+  return from_cuda(e, "rotate launch");
+}
+
+paro_status paro_w4_linear(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                           const uint16_t* d_zeros, uint16_t* d_y, int M, int d_in, int d_out,
+                           int group_size, paro_stream_t stream) {
+  paro_status st;
+  if ((st = check_linear_shape(M, d_in, d_out, group_size)) != PARO_OK) return st;
+  if (M == 0) return ok();
+  if ((st = check_weights(d_qweight, d_scales, d_zeros)) != PARO_OK) return st;
+  if (!d_x || !d_y) return fail(PARO_ERR_INVALID_ARG, "null activation pointer");
+  if (!aligned(d_x, 16) || !aligned(d_y, 16)) return fail(PARO_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
+  const size_t yb = (size_t)M * d_out * 2;
+  if (overlap(d_y, yb, d_x, (size_t)M * d_in * 2) || overlap(d_y, yb, d_qweight, (size_t)d_out * d_in / 2) ||
+      overlap(d_y, yb, d_scales, (size_t)d_out * (d_in / 128) * 2) ||
+      overlap(d_y, yb, d_zeros, (size_t)d_out * (d_in / 128) * 2))
+    return fail(PARO_ERR_INVALID_ARG, "y overlaps an input");
+  cudaError_t e = paro::launch_w4_linear_mma(d_x, 0, d_qweight, reinterpret_cast<const __half*>(d_scales),
+                                             reinterpret_cast<const __half*>(d_zeros),
+                                             reinterpret_cast<__nv_bfloat16*>(d_y), M, d_in, d_out,
+                                             reinterpret_cast<cudaStream_t>(stream), false);
+  return from_cuda(e, "w4 linear launch");
+}
+
+size_t paro_workspace_bytes(int M, int d_in) {
+  if (M <= 0 || d_in <= 0) return 0;
+  const size_t b = (size_t)M * d_in * 2;  // fp16 transformed activations
+  return (b + 255) & ~(size_t)255;
+}
+
+paro_status paro_rotate_w4_linear(const uint16_t* d_x, int K, const uint16_t* d_pairs,
+                                  const float* d_cos, const float* d_sin, const float* d_scale,
+                                  const uint32_t* d_qweight, const uint16_t* d_scales,
+                                  const uint16_t* d_zeros, uint16_t* d_y, int M, int d_in, int d_out,
+                                  int group_size, void* d_workspace, size_t workspace_bytes,
+                                  paro_stream_t stream) {
+  paro_status st;
+  if ((st = check_linear_shape(M, d_in, d_out, group_size)) != PARO_OK) return st;
+  if ((st = check_width(d_in)) != PARO_OK) return st;
+  if ((st = check_tables(K, d_in, d_pairs, d_cos, d_sin, d_scale)) != PARO_OK) return st;
+  if (M == 0) return ok();
+  if ((st = check_weights(d_qweight, d_scales, d_zeros)) != PARO_OK) return st;
+  if (!d_x || !d_y) return fail(PARO_ERR_INVALID_ARG, "null activation pointer");
+  if (!aligned(d_x, 16) || !aligned(d_y, 16)) return fail(PARO_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
+  const size_t need = paro_workspace_bytes(M, d_in);
+  if (!d_workspace || workspace_bytes < need || !aligned(d_workspace, 256))
+    return fail(PARO_ERR_INVALID_ARG, "workspace must be 256-byte aligned and hold %zu bytes", need);
+  const size_t yb = (size_t)M * d_out * 2;
+  if (overlap(d_y, yb, d_x, (size_t)M * d_in * 2) || overlap(d_y, yb, d_workspace, need) ||
+      overlap(d_workspace, need, d_x, (size_t)M * d_in * 2) ||
+      overlap(d_y, yb, d_qweight, (size_t)d_out * d_in / 2))
+    return fail(PARO_ERR_INVALID_ARG, "y, x and workspace must not overlap");
+  int* status = status_ptr();
+  if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = paro::launch_rotate_act(d_x, d_workspace, 1, M, d_in, K, d_pairs, d_cos, d_sin, d_scale,
+                                          status, s, true);
+  if (e != cudaSuccess) return from_cuda(e, "rotate launch");
+  e = paro::launch_w4_linear_mma(d_workspace, 1, d_qweight, reinterpret_cast<const __half*>(d_scales),
+                                 reinterpret_cast<const __half*>(d_zeros), reinterpret_cast<__nv_bfloat16*>(d_y),
+                                 M, d_in, d_out, s, true);
+  return from_cuda(e, "w4 linear launch");
+}
+
+paro_status paro_get_device_status(paro_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return from_cuda(e, "stream synchronize");
+  int* p = status_ptr();
+  if (!p) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
+  int v = 0;
+  e = cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return from_cuda(e, "status read");
+  const int zero = 0;
+  e = cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return from_cuda(e, "status clear");
+  if (v == 0) return ok();
+  return fail(static_cast<paro_status>(v), "device reported %s", paro_status_string(static_cast<paro_status>(v)));
+}
+
+}  // extern "C"

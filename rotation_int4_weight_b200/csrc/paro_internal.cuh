@@ -1,0 +1,47 @@
+// Internal declarations shared by the CUDA translation units of libparo.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/paro.h"
+
+namespace paro {
+
+// Values written into the per-device status word (first error wins).
+constexpr int kStatusBadIndex = PARO_ERR_INVALID_ARG;
+constexpr int kStatusTimeout = PARO_ERR_TIMEOUT;
+
+constexpr int kGroup = 128;      // quantisation group along d_in
+constexpr int kMaxStages = 16;   // K
+constexpr int kMaxDim = 49152;   // rotation width (one fp32 row in shared memory)
+
+__device__ __forceinline__ void report_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// ---- launchers implemented in the kernel translation units --------------------
+// All return a cudaError_t from the launch (cudaSuccess when nothing failed).
+
+// Activation transform, bf16 -> bf16 (mode 0) or bf16 -> fp16 (mode 1).
+cudaError_t launch_rotate_act(const uint16_t* x, void* out, int out_is_f16, int M, int d, int K,
+                              const uint16_t* pairs, const float* cos_t, const float* sin_t,
+                              const float* scale, int* status, cudaStream_t stream, bool pdl_trigger);
+
+// Weight fold, fp32 -> fp32: rows of W go through the same stages, then * s.
+cudaError_t launch_fold_weights(const float* W, float* out, int rows, int d, int K,
+                                const uint16_t* pairs, const float* cos_t, const float* sin_t,
+                                const float* scale, int* status, cudaStream_t stream);
+
+// Group quantisation + nibble packing of fp32 rows.
+cudaError_t launch_quantize_pack(const float* Wt, int d_out, int d_in, uint32_t* qweight,
+                                 __half* scales, __half* zeros, cudaStream_t stream);
+
+// INT4 linear, M small or large, x in bf16 (x_is_f16 = 0) or fp16 (1).
+cudaError_t launch_w4_linear_mma(const void* x, int x_is_f16, const uint32_t* qweight,
+                                 const __half* scales, const __half* zeros, __nv_bfloat16* y,
+                                 int M, int d_in, int d_out, cudaStream_t stream, bool pdl_wait);
+
+}  // namespace paro

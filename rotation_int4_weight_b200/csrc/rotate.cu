@@ -1,0 +1,202 @@
+// Givens-stage transform kernels: the activation-side transform
+//   x~ = diag(1/s) R_K ... R_1 x                       (runtime, per token row)
+// and the build-time weight fold
+//   w~ = diag(s)   R_K ... R_1 w                       (per output row of W)
+// Page "ParoQuant: pairwise rotations that survive deployment", section "A
+// rotation small enough to execute": a stage rotates disjoint channel pairs
+// (i, j) with x_i' = c x_i + s x_j, x_j' = -s x_i + c x_j, so every pair of a
+// stage can be updated in parallel without write conflicts.
+//
+// One CTA owns R whole rows.  It stages them in shared memory as fp32 in a
+// channel-major layout xs[channel][R] (the R rows of one channel are adjacent,
+// so a pair update moves R values with one vector load/store per channel),
+// applies all K stages there with a barrier between stages, and writes the
+// result once.  HBM sees one read and one write of the rows; the pair and
+// cos/sin tables stream from L2.
+#include "paro_internal.cuh"
+
+namespace paro {
+namespace {
+
+enum Mode { kActBf16 = 0, kActF16 = 1, kFoldF32 = 2 };
+
+template <int R>
+__device__ __forceinline__ void ld_vec(const float* p, float (&v)[R]) {
+  if constexpr (R == 1) {
+    v[0] = *p;
+  } else if constexpr (R == 2) {
+    float2 t = *reinterpret_cast<const float2*>(p);
+    v[0] = t.x; v[1] = t.y;
+  } else {
+    float4 t = *reinterpret_cast<const float4*>(p);
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  }
+}
+
+template <int R>
+__device__ __forceinline__ void st_vec(float* p, const float (&v)[R]) {
+  if constexpr (R == 1) {
+    *p = v[0];
+  } else if constexpr (R == 2) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  } else {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+template <int R, int MODE>
+__global__ void __launch_bounds__(512)
+givens_rows_kernel(const void* __restrict__ in, void* __restrict__ out, int M, int d, int K,
+                   const uint32_t* __restrict__ pairs, const float* __restrict__ cos_t,
+                   const float* __restrict__ sin_t, const float* __restrict__ scale, int* status,
+                   int pdl_trigger) {
+  extern __shared__ __align__(16) float xs[];  // [d][R]
+  if (pdl_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  const int row0 = blockIdx.x * R;
+  const int nrows = min(R, M - row0);
+  const int tid = threadIdx.x, nth = blockDim.x;
+
+  // ---- load: rows -> xs[c][r] ------------------------------------------------
+  // Each thread takes two adjacent channels of every row (4-byte bf16 pairs or
+  // 8-byte fp32 pairs: a warp reads 128 or 256 contiguous bytes per row) and
+  // writes the 2 x R values with vector stores to consecutive channel slots.
+  const int npairs_ch = d >> 1;
+  for (int cp = tid; cp < npairs_ch; cp += nth) {
+    float v0[R], v1[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (r < nrows) {
+        const size_t off = (size_t)(row0 + r) * d + 2 * cp;
+        if constexpr (MODE == kFoldF32) {
+          const float2 f = *reinterpret_cast<const float2*>(static_cast<const float*>(in) + off);
+          v0[r] = f.x; v1[r] = f.y;
+        } else {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
+              static_cast<const __nv_bfloat16*>(in) + off));
+          v0[r] = f.x; v1[r] = f.y;
+        }
+      } else {
+        v0[r] = 0.f; v1[r] = 0.f;
+      }
+    }
+    st_vec<R>(xs + (size_t)(2 * cp) * R, v0);
+    st_vec<R>(xs + (size_t)(2 * cp + 1) * R, v1);
+  }
+  __syncthreads();
+
+  // ---- K stages of disjoint pair rotations -------------------------------------
+  const int half = d >> 1;
+  for (int k = 0; k < K; ++k) {
+    const uint32_t* pk = pairs + (size_t)k * half;
+    const float* ck = cos_t + (size_t)k * half;
+    const float* sk = sin_t + (size_t)k * half;
+    for (int t = tid; t < half; t += nth) {
+      const uint32_t pr = __ldg(pk + t);
+      const int i = pr & 0xFFFF, j = pr >> 16;
+      const float c = __ldg(ck + t), s = __ldg(sk + t);
+      if (i >= d || j >= d) {
+        report_status(status, kStatusBadIndex);
+        continue;
+      }
+      float a[R], b[R];
+      ld_vec<R>(xs + (size_t)i * R, a);
+      ld_vec<R>(xs + (size_t)j * R, b);
+      float na[R], nb[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        na[r] = fmaf(c, a[r], s * b[r]);
+        nb[r] = fmaf(-s, a[r], c * b[r]);
+      }
+      st_vec<R>(xs + (size_t)i * R, na);
+      st_vec<R>(xs + (size_t)j * R, nb);
+    }
+    __syncthreads();
+  }
+
+  // ---- channel scale and store -------------------------------------------------
+  for (int cp = tid; cp < npairs_ch; cp += nth) {
+    const int c = 2 * cp;
+    float f0 = 1.0f, f1 = 1.0f;
+    if (scale) {
+      const float s0 = __ldg(scale + c), s1 = __ldg(scale + c + 1);
+      if constexpr (MODE == kFoldF32) { f0 = s0; f1 = s1; }
+      else { f0 = 1.0f / s0; f1 = 1.0f / s1; }
+    }
+    float v0[R], v1[R];
+    ld_vec<R>(xs + (size_t)c * R, v0);
+    ld_vec<R>(xs + (size_t)(c + 1) * R, v1);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (r < nrows) {
+        const size_t off = (size_t)(row0 + r) * d + c;
+        const float a = v0[r] * f0, b = v1[r] * f1;
+        if constexpr (MODE == kFoldF32) {
+          *reinterpret_cast<float2*>(static_cast<float*>(out) + off) = make_float2(a, b);
+        } else if constexpr (MODE == kActBf16) {
+          *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(out) + off) = __floats2bfloat162_rn(a, b);
+        } else {
+          *reinterpret_cast<__half2*>(static_cast<__half*>(out) + off) = __floats2half2_rn(a, b);
+        }
+      }
+    }
+  }
+}
+
+int pick_rows_per_cta(int M, int d) {
+  int R = 1;
+  if (d <= 6144) R = 4;
+  else if (d <= 12288) R = 2;
+  while (R > 1 && R > M) R >>= 1;
+  return R;
+}
+
+template <int MODE>
+cudaError_t launch_givens(const void* in, void* out, int M, int d, int K, const uint16_t* pairs,
+                          const float* cos_t, const float* sin_t, const float* scale, int* status,
+                          cudaStream_t stream, bool pdl_trigger) {
+  const int R = pick_rows_per_cta(M, d);
+  const int threads = d >= 2048 ? 512 : 256;
+  const size_t smem = (size_t)R * d * sizeof(float);
+  const dim3 grid((M + R - 1) / R);
+  const uint32_t* p32 = reinterpret_cast<const uint32_t*>(pairs);
+  const int trig = pdl_trigger ? 1 : 0;
+  cudaError_t e = cudaSuccess;
+  switch (R) {
+    case 4:
+      e = cudaFuncSetAttribute(givens_rows_kernel<4, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess)
+        givens_rows_kernel<4, MODE><<<grid, threads, smem, stream>>>(in, out, M, d, K, p32, cos_t, sin_t, scale, status, trig);
+      break;
+    case 2:
+      e = cudaFuncSetAttribute(givens_rows_kernel<2, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess)
+        givens_rows_kernel<2, MODE><<<grid, threads, smem, stream>>>(in, out, M, d, K, p32, cos_t, sin_t, scale, status, trig);
+      break;
+    default:
+      e = cudaFuncSetAttribute(givens_rows_kernel<1, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess)
+        givens_rows_kernel<1, MODE><<<grid, threads, smem, stream>>>(in, out, M, d, K, p32, cos_t, sin_t, scale, status, trig);
+      break;
+  }
+  if (e != cudaSuccess) return e;
+  return cudaPeekAtLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_rotate_act(const uint16_t* x, void* out, int out_is_f16, int M, int d, int K,
+                              const uint16_t* pairs, const float* cos_t, const float* sin_t,
+                              const float* scale, int* status, cudaStream_t stream, bool pdl_trigger) {
+  if (out_is_f16)
+    return launch_givens<kActF16>(x, out, M, d, K, pairs, cos_t, sin_t, scale, status, stream, pdl_trigger);
+  return launch_givens<kActBf16>(x, out, M, d, K, pairs, cos_t, sin_t, scale, status, stream, pdl_trigger);
+}
+
+cudaError_t launch_fold_weights(const float* W, float* out, int rows, int d, int K,
+                                const uint16_t* pairs, const float* cos_t, const float* sin_t,
+                                const float* scale, int* status, cudaStream_t stream) {
+  return launch_givens<kFoldF32>(W, out, rows, d, K, pairs, cos_t, sin_t, scale, status, stream, false);
+}
+
+}  // namespace paro

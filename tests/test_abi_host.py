@@ -1,0 +1,139 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+entry point, and rejects invalid calls before touching the GPU.  No kernel is
+launched by these tests (no CUDA device is needed)."""
+import ctypes
+import os
+import re
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+import rotation_int4_weight_b200 as paro
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+OK, INVALID, UNSUPPORTED = 0, 1, 2
+
+A = ctypes.c_void_p(1 << 20)        # aligned fake device pointers, never dereferenced
+B = ctypes.c_void_p((1 << 20) + 4096 * 1024)
+C = ctypes.c_void_p((1 << 21) + 8192 * 1024)
+D = ctypes.c_void_p((1 << 22) + 8192 * 1024)
+E = ctypes.c_void_p((1 << 23) + 8192 * 1024)
+W = ctypes.c_void_p((1 << 24))
+MIS = ctypes.c_void_p((1 << 20) + 2)  # misaligned
+
+
+def declared_symbols():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", f)).read()
+            names |= set(re.findall(r"PARO_API\s+[\w\s\*]+?\b(paro_\w+)\s*\(", txt))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert {"paro_pack_weights", "paro_rotate", "paro_w4_linear", "paro_rotate_w4_linear"} <= names
+    out = subprocess.run(["nm", "-D", "--defined-only", paro.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (paro_\w+)", out))
+    assert names <= exported, f"declared but not exported: {names - exported}"
+    assert names <= set(paro.EXPORTED), f"declared but not bound: {names - set(paro.EXPORTED)}"
+    for n in names:
+        assert hasattr(paro.lib, n)
+
+
+def test_status_strings_and_version():
+    assert paro.paro_weight_layout_version() == 1
+    for code, name in [(0, "PARO_OK"), (1, "PARO_ERR_INVALID_ARG"), (2, "PARO_ERR_UNSUPPORTED"),
+                       (3, "PARO_ERR_CUDA"), (4, "PARO_ERR_TIMEOUT")]:
+        assert paro.lib.paro_status_string(code).decode() == name
+
+
+def test_workspace_bytes():
+    assert paro.paro_workspace_bytes(0, 512) == 0
+    assert paro.paro_workspace_bytes(1, 512) == 1024
+    assert paro.paro_workspace_bytes(3, 1536) == 9216
+    assert paro.paro_workspace_bytes(1, 128) % 256 == 0
+
+
+def rot(x=A, y=B, M=4, d=512, K=8, pairs=C, c=D, s=E, scale=W):
+    return paro.lib.paro_rotate(x, y, M, d, K, pairs, c, s, scale, None)
+
+
+def lin(x=A, q=B, sc=C, z=D, y=E, M=4, d_in=512, d_out=512, g=128):
+    return paro.lib.paro_w4_linear(x, q, sc, z, y, M, d_in, d_out, g, None)
+
+
+def fused(x=A, K=8, pairs=C, c=D, s=E, scale=W, q=B, sc=C, z=D, y=E, M=4, d_in=512, d_out=512, g=128,
+          ws=ctypes.c_void_p(1 << 26), wsb=1 << 20):
+    return paro.lib.paro_rotate_w4_linear(x, K, pairs, c, s, scale, q, sc, z, y, M, d_in, d_out, g, ws, wsb, None)
+
+
+def pack(Wp=W, d_out=512, d_in=512, g=128, K=8, pairs=C, c=D, s=E, scale=A, ws=ctypes.c_void_p(1 << 27),
+         q=B, sc=C, z=D):
+    return paro.lib.paro_pack_weights(Wp, d_out, d_in, g, K, pairs, c, s, scale, ws, q, sc, z, None)
+
+
+@pytest.mark.parametrize("kwargs,expect", [
+    (dict(d=7), INVALID), (dict(d=0), INVALID), (dict(d=49154), UNSUPPORTED), (dict(M=-1), INVALID),
+    (dict(K=-1), INVALID), (dict(K=17), UNSUPPORTED), (dict(pairs=None), INVALID), (dict(c=None), INVALID),
+    (dict(x=None), INVALID), (dict(y=None), INVALID), (dict(x=MIS), INVALID),
+    (dict(pairs=ctypes.c_void_p((1 << 20) + 2)), INVALID), (dict(scale=ctypes.c_void_p((1 << 24) + 2)), INVALID),
+    (dict(y=ctypes.c_void_p((1 << 20) + 16)), INVALID),  # partial overlap with x
+    (dict(M=0, x=None, y=None), OK),                       # empty batch: nothing enqueued
+])
+def test_rotate_validation(kwargs, expect):
+    assert rot(**kwargs) == expect
+    if expect != OK:
+        assert paro.lib.paro_last_error().decode()
+
+
+@pytest.mark.parametrize("kwargs,expect", [
+    (dict(d_in=500), INVALID), (dict(d_in=0), INVALID), (dict(d_out=8), UNSUPPORTED), (dict(d_out=0), INVALID),
+    (dict(g=64), UNSUPPORTED), (dict(g=0), INVALID), (dict(M=-2), INVALID), (dict(q=None), INVALID),
+    (dict(q=MIS), INVALID), (dict(x=MIS), INVALID), (dict(sc=ctypes.c_void_p((1 << 21) + 1)), INVALID),
+    (dict(y=A), INVALID),                                  # output aliases the input
+    (dict(M=0, x=None, y=None), OK),
+])
+def test_w4_linear_validation(kwargs, expect):
+    assert lin(**kwargs) == expect
+
+
+@pytest.mark.parametrize("kwargs,expect", [
+    (dict(ws=None), INVALID), (dict(wsb=100), INVALID), (dict(ws=ctypes.c_void_p((1 << 26) + 16)), INVALID),
+    (dict(K=20), UNSUPPORTED), (dict(d_in=50000 * 128 // 128 * 128 + 128 * 400), UNSUPPORTED),
+    (dict(d_out=24), UNSUPPORTED), (dict(pairs=None), INVALID), (dict(y=A), INVALID),
+    (dict(M=0, x=None, y=None), OK),
+])
+def test_fused_validation(kwargs, expect):
+    assert fused(**kwargs) == expect
+
+
+@pytest.mark.parametrize("kwargs,expect", [
+    (dict(Wp=None), INVALID), (dict(d_in=100), INVALID), (dict(g=256), UNSUPPORTED), (dict(d_out=0), INVALID),
+    (dict(ws=None), INVALID), (dict(ws=W), INVALID), (dict(K=-3), INVALID), (dict(q=None), INVALID),
+    (dict(d_in=65536), UNSUPPORTED),
+])
+def test_pack_validation(kwargs, expect):
+    assert pack(**kwargs) == expect
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    pkg = tmp_path / "rotation_int4_weight_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "rotation_int4_weight_b200", "__init__.py"), pkg / "__init__.py")
+    r = subprocess.run([sys.executable, "-c", "import rotation_int4_weight_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libparo.so is missing" in r.stderr
+
+
+def test_product_path_does_not_touch_the_oracle():
+    pkg = os.path.join(ROOT, "rotation_int4_weight_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in txt.replace("oracle-free", ""), f
+                assert "import synth" not in txt and "from synth" not in txt, f

@@ -1,0 +1,242 @@
+"""CUDA path against the fp64 oracle on the same seeded inputs (needs a B200).
+
+Bit-exact: packing, unpacking, pair indexing.  Within the criteria of
+tests/tolerances.py: the rotation and the linear.  Sizes span several tiles
+and ragged tails; the full-size layers are checked on sampled output rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import config_problems, linear_problem
+from tests.tolerances import assert_linear_close, assert_rotation_close, linear_errors, rotation_errors
+
+pytestmark = pytest.mark.gpu
+
+paro = pytest.importorskip("rotation_int4_weight_b200")
+DEV = "cuda"
+
+
+def dev_tables(p):
+    pairs = torch.from_numpy(p.pairs.view(np.int16)).to(DEV)
+    return (pairs, torch.from_numpy(p.cos_t).to(DEV), torch.from_numpy(p.sin_t).to(DEV),
+            torch.from_numpy(p.scale).to(DEV))
+
+
+def dev_x(x):
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(DEV).to(torch.bfloat16)
+
+
+def host(t):
+    if t.dtype == torch.bfloat16:
+        return t.float().cpu().numpy()
+    return t.cpu().numpy()
+
+
+def oracle_pack_from_fp32(wt32):
+    q, sc, z = oracle.quantize_groups(wt32)
+    return oracle.pack_nibbles(q), sc, z.astype(np.float16)
+
+
+def gpu_pack(W32, tables=None):
+    W = torch.from_numpy(np.ascontiguousarray(W32)).to(DEV)
+    if tables is None:
+        return paro.paro_pack_weights(W)
+    return paro.paro_pack_weights(W, *tables)
+
+
+def to_np_pack(qw, sc, z):
+    return (qw.cpu().numpy().view(np.uint32), sc.cpu().numpy(), z.cpu().numpy())
+
+
+# ---------------------------------------------------------------- packing
+@pytest.mark.parametrize("shape", [(512, 512), (48, 1536), (272, 8960 // 2)])
+def test_pack_is_bit_exact_on_the_same_fp32_weights(shape):
+    d_out, d_in = shape
+    p = linear_problem(21, d_in, d_in, d_out, 1)
+    wt32 = oracle.fold_weights(p.W, p.pairs, p.cos_t, p.sin_t, p.scale).astype(np.float32)
+    ref = oracle_pack_from_fp32(wt32)
+    got = to_np_pack(*gpu_pack(wt32))
+    assert np.array_equal(got[0], ref[0])
+    assert np.array_equal(got[1].view(np.uint16), ref[1].view(np.uint16))
+    assert np.array_equal(got[2].view(np.uint16), ref[2].view(np.uint16))
+
+
+def test_pack_degenerate_groups_bit_exact():
+    v = np.zeros((16, 512), dtype=np.float32)
+    v[1, :128] = 0.5
+    v[2, 130] = -1e-30
+    v[3, 256:384] = -0.5
+    v[4, :] = np.linspace(-3, 1, 512, dtype=np.float32)
+    v[5, ::2] = 1e-3
+    ref = oracle_pack_from_fp32(v)
+    got = to_np_pack(*gpu_pack(v))
+    assert np.array_equal(got[0], ref[0])
+    assert np.array_equal(got[1].view(np.uint16), ref[1].view(np.uint16))
+    assert np.array_equal(got[2].view(np.uint16), ref[2].view(np.uint16))
+
+
+def test_brute_force_unpack_of_gpu_pack():
+    """Every nibble, scale and zero of a GPU-packed layer unpacks to the oracle's codes."""
+    p = next(config_problems(0))
+    wt32 = oracle.fold_weights(p.W, p.pairs, p.cos_t, p.sin_t, p.scale).astype(np.float32)
+    qw, sc, z = to_np_pack(*gpu_pack(wt32))
+    q_ref, sc_ref, z_ref = oracle.quantize_groups(wt32)
+    by = qw.astype("<u4").view(np.uint8).reshape(qw.shape[0], -1)
+    codes = np.empty((qw.shape[0], by.shape[1] * 2), dtype=np.uint8)
+    codes[:, 0::2], codes[:, 1::2] = by & 0xF, by >> 4
+    assert np.array_equal(codes, q_ref)
+    assert np.array_equal(z.astype(np.float32).astype(np.uint8), z_ref)
+    assert np.array_equal(sc.view(np.uint16), sc_ref.view(np.uint16))
+
+
+@pytest.mark.parametrize("cfg,only", [(0, None), (1, ["k", "down"])])
+def test_pack_with_fold(cfg, only):
+    for p in config_problems(cfg, only=only):
+        tables = dev_tables(p)
+        W = torch.from_numpy(p.W).to(DEV)
+        ws = torch.empty(p.d_out, p.d_in, dtype=torch.float32, device=DEV)
+        qw, sc, z = paro.paro_pack_weights(W, *tables, workspace=ws)
+        fold_ref = oracle.fold_weights(p.W, p.pairs, p.cos_t, p.sin_t, p.scale)
+        fold_gpu = ws.cpu().numpy().astype(np.float64)
+        rel = np.linalg.norm(fold_gpu - fold_ref, axis=1) / np.linalg.norm(fold_ref, axis=1)
+        assert rel.max() <= 1e-5
+        # the GPU's fp32 fold packs bit-exactly like the oracle's quantiser
+        ref_from_gpu_fold = oracle_pack_from_fp32(ws.cpu().numpy())
+        got = to_np_pack(qw, sc, z)
+        assert np.array_equal(got[0], ref_from_gpu_fold[0])
+        # against the oracle's own fp64 fold only rare rounding ties may flip a code
+        q_ref = oracle.unpack_nibbles(oracle.pack_weights(p.W, p.pairs, p.cos_t, p.sin_t, p.scale)[0])
+        flips = np.count_nonzero(oracle.unpack_nibbles(got[0]) != q_ref)
+        assert flips <= max(2, q_ref.size // 100000)
+
+
+# ---------------------------------------------------------------- rotation
+@pytest.mark.parametrize("M,d", [(1, 512), (3, 512), (4, 512), (5, 1536), (17, 1536), (9, 8960), (2, 14336),
+                                 (7, 130), (33, 4096)])
+def test_rotate_parity(M, d):
+    p = linear_problem(31, M * 1000 + d, d, 16, M)
+    x = dev_x(p.x)
+    got = host(paro.paro_rotate(x, *dev_tables(p)))
+    ref = oracle.rotate(p.x, p.pairs, p.cos_t, p.sin_t, p.scale)
+    assert_rotation_close(got, ref)
+
+
+def test_rotate_signed_permutation_is_bit_exact():
+    """c = 0, s = 1 makes every stage an exact signed permutation: bit-exact pair indexing."""
+    p = linear_problem(32, 0, 4096, 16, 6)
+    c = np.zeros_like(p.cos_t)
+    s = np.ones_like(p.sin_t)
+    tables = (torch.from_numpy(p.pairs.view(np.int16)).to(DEV), torch.from_numpy(c).to(DEV),
+              torch.from_numpy(s).to(DEV), None)
+    got = host(paro.paro_rotate(dev_x(p.x), *tables))
+    ref = oracle.rotate(p.x, p.pairs, c, s, None)
+    assert np.array_equal(got, ref.astype(np.float32))
+
+
+def test_rotate_pair_order_within_stage_is_bit_irrelevant():
+    p = linear_problem(33, 0, 1536, 16, 8)
+    rng = np.random.default_rng(0)
+    perm = np.stack([rng.permutation(p.d_in // 2) for _ in range(p.K)])
+    pairs2 = np.stack([p.pairs[k][perm[k]] for k in range(p.K)])
+    c2 = np.stack([p.cos_t[k][perm[k]] for k in range(p.K)])
+    s2 = np.stack([p.sin_t[k][perm[k]] for k in range(p.K)])
+    x = dev_x(p.x)
+    a = paro.paro_rotate(x, *dev_tables(p))
+    b = paro.paro_rotate(x, torch.from_numpy(pairs2.view(np.int16)).to(DEV), torch.from_numpy(c2).to(DEV),
+                         torch.from_numpy(s2).to(DEV), torch.from_numpy(p.scale).to(DEV))
+    assert torch.equal(a, b)
+
+
+def test_rotate_in_place_and_k0():
+    p = linear_problem(34, 0, 1536, 16, 5)
+    x = dev_x(p.x)
+    ref = paro.paro_rotate(x, *dev_tables(p))
+    y = x.clone()
+    paro.paro_rotate(y, *dev_tables(p), out=y)
+    assert torch.equal(y, ref)
+    # K = 0, no scale: the identity
+    assert torch.equal(paro.paro_rotate(x), x)
+    # K = 0 with scale only
+    got = host(paro.paro_rotate(x, scale=torch.from_numpy(p.scale).to(DEV)))
+    assert_rotation_close(got, p.x / p.scale.astype(np.float64))
+
+
+def test_rotate_bad_pair_index_is_reported_not_faulted():
+    p = linear_problem(35, 0, 512, 16, 2)
+    bad = p.pairs.copy()
+    bad[3, 7, 1] = 600  # >= d
+    assert paro.paro_get_device_status() == 0
+    paro.paro_rotate(dev_x(p.x), torch.from_numpy(bad.view(np.int16)).to(DEV), *dev_tables(p)[1:])
+    assert paro.paro_get_device_status() == 1
+    assert paro.paro_get_device_status() == 0  # cleared
+
+
+# ---------------------------------------------------------------- linear
+def _packed(p, rotate=True):
+    if rotate:
+        return paro.paro_pack_weights(torch.from_numpy(p.W).to(DEV), *dev_tables(p))
+    return paro.paro_pack_weights(torch.from_numpy(p.W).to(DEV))
+
+
+@pytest.mark.parametrize("M,d_in,d_out", [(1, 512, 512), (3, 512, 512), (8, 1536, 256), (9, 1536, 272),
+                                          (16, 512, 1024), (17, 384, 96), (40, 1024, 64), (2, 8960, 1536)])
+def test_w4_linear_parity(M, d_in, d_out):
+    p = linear_problem(41, M * 7 + d_out, d_in, d_out, M)
+    qw, sc, z = _packed(p, rotate=False)
+    got = host(paro.paro_w4_linear(dev_x(p.x), qw, sc, z))
+    ref = oracle.w4_linear(p.x, *to_np_pack(qw, sc, z))
+    assert_linear_close(got, ref)
+
+
+@pytest.mark.parametrize("M,d_in,d_out", [(1, 512, 512), (4, 512, 512), (16, 1536, 256), (11, 4096, 1024),
+                                          (24, 1536, 1536)])
+def test_rotate_w4_linear_parity(M, d_in, d_out):
+    p = linear_problem(51, M * 13 + d_in, d_in, d_out, M)
+    qw, sc, z = _packed(p)
+    got = host(paro.paro_rotate_w4_linear(dev_x(p.x), *dev_tables(p), qw, sc, z))
+    ref = oracle.rotate_w4_linear(p.x, p.pairs, p.cos_t, p.sin_t, p.scale, *to_np_pack(qw, sc, z))
+    assert_linear_close(got, ref)
+    # and the unfused composition agrees with the same reference
+    xr = paro.paro_rotate(dev_x(p.x), *dev_tables(p))
+    got2 = host(paro.paro_w4_linear(xr, qw, sc, z))
+    assert_linear_close(got2, ref)
+
+
+def test_empty_batch_is_a_noop():
+    p = linear_problem(52, 0, 512, 512, 1)
+    qw, sc, z = _packed(p)
+    x = torch.empty(0, 512, dtype=torch.bfloat16, device=DEV)
+    assert paro.paro_w4_linear(x, qw, sc, z).shape == (0, 512)
+    assert paro.paro_rotate_w4_linear(x, *dev_tables(p), qw, sc, z).shape == (0, 512)
+    assert paro.paro_rotate(x, *dev_tables(p)).shape == (0, 512)
+
+
+# ---------------------------------------------------------------- full-size layers, sampled rows
+def _sampled_check(p, M_rows, n_cols=256, seed=0):
+    """Full-size fused call; compare sampled tokens x sampled output columns with the oracle."""
+    qw, sc, z = _packed(p)
+    y = host(paro.paro_rotate_w4_linear(dev_x(p.x), *dev_tables(p), qw, sc, z))
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(p.M, size=min(M_rows, p.M), replace=False))
+    cols = np.sort(rng.choice(p.d_out, size=min(n_cols, p.d_out), replace=False))
+    qwn, scn, zn = to_np_pack(qw, sc, z)
+    xt = oracle.rotate(p.x[rows], p.pairs, p.cos_t, p.sin_t, p.scale)
+    w_hat = oracle.dequantize(qwn[cols], scn[cols], zn[cols])
+    ref = oracle.linear(xt, w_hat)
+    got = y[rows][:, cols]
+    # the rms in the criterion is the full output row's, estimated from the sample
+    metric, literal = linear_errors(got, ref)
+    assert metric <= 1e-2, (p.name, metric, literal)
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_full_size_decode_layers(cfg):
+    for p in config_problems(cfg, M=1 if cfg == 1 else 16):
+        _sampled_check(p, 16)
+
+
+def test_full_size_prefill_layer_sampled():
+    p = next(config_problems(3, only=["k"]))
+    _sampled_check(p, 64, 128)
