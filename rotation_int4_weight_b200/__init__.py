@@ -46,7 +46,7 @@ class ParoError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m rotation_int4_weight_b200._build` "
+            f"{LIB_PATH} is missing: build it with `python rotation_int4_weight_b200/_build.py` "
             "(there is no fallback implementation)")
     handle = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in EXPORTED.items():

@@ -1,6 +1,7 @@
 """Builds libparo.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-Usage: python -m rotation_int4_weight_b200._build [--force] [-v]
+Usage: python rotation_int4_weight_b200/_build.py [--force] [-v]
+(run it as a file: importing the package would first load the library it builds)
 """
 from __future__ import annotations
 
