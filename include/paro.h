@@ -150,6 +150,27 @@ PARO_API paro_status paro_rotate_w4_linear(const uint16_t* d_x, int K, const uin
                                   paro_stream_t stream);
 
 /*
+ * The same computation as paro_rotate_w4_linear for callers that cannot
+ * allocate device memory (the paper has no counterpart: this is an interface
+ * convenience of this library).  Instead of a caller-provided workspace, the
+ * transformed activations go to a scratch array built into the library: every
+ * GPU that loads libparo holds 512 KiB for it until the process exits, and
+ * M * d_in may not exceed 262144 (PARO_ERR_UNSUPPORTED, nothing enqueued).
+ * The call allocates nothing.  Its first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  All calls on a device
+ * share the one array: calls that may overlap on the GPU (different streams,
+ * or other work between them that is not ordered) race on it and must be
+ * serialised by the caller.  Arguments, layouts and results are those of
+ * paro_rotate_w4_linear.
+ */
+PARO_API paro_status paro_rotate_w4_linear_noalloc(const uint16_t* d_x, int K, const uint16_t* d_pairs,
+                                  const float* d_cos, const float* d_sin, const float* d_scale,
+                                  const uint32_t* d_qweight, const uint16_t* d_scales,
+                                  const uint16_t* d_zeros, uint16_t* d_y, int M, int d_in, int d_out,
+                                  int group_size, paro_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of
  * the current GPU: PARO_OK, PARO_ERR_INVALID_ARG (a kernel met a pair index
  * >= d and skipped it) or PARO_ERR_TIMEOUT (a bounded wait gave up).

@@ -17,7 +17,7 @@ import torch
 __all__ = [
     "ParoError", "LIB_PATH", "lib", "paro_weight_layout_version", "paro_workspace_bytes",
     "paro_pack_weights", "paro_rotate", "paro_w4_linear", "paro_rotate_w4_linear",
-    "paro_get_device_status", "EXPORTED",
+    "paro_rotate_w4_linear_noalloc", "paro_get_device_status", "EXPORTED",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libparo.so")
@@ -33,6 +33,7 @@ EXPORTED = {
     "paro_w4_linear": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "paro_workspace_bytes": (_S, [_I, _I]),
     "paro_rotate_w4_linear": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
+    "paro_rotate_w4_linear_noalloc": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "paro_get_device_status": (_I, [_P]),
 }
 
@@ -164,6 +165,22 @@ def paro_rotate_w4_linear(x: torch.Tensor, pairs, cos_t, sin_t, scale, qweight, 
                                    M, d_in, d_out, group_size, _ptr(workspace), workspace.numel(),
                                    _stream(stream))
     _check(st, "paro_rotate_w4_linear")
+    return out
+
+
+def paro_rotate_w4_linear_noalloc(x: torch.Tensor, pairs, cos_t, sin_t, scale, qweight, scales, zeros, *,
+                                  out=None, group_size: int = 128, stream=None):
+    """paro_rotate_w4_linear without a workspace: the library's built-in scratch
+    array holds the transformed activations, so the call allocates nothing
+    (M * d_in <= 262144; calls that overlap on the GPU race on the array)."""
+    M, d_in = x.shape
+    d_out = qweight.shape[0]
+    if out is None:
+        out = torch.empty(M, d_out, dtype=torch.bfloat16, device=x.device)
+    st = lib.paro_rotate_w4_linear_noalloc(_ptr(_u16(x)), _K(pairs), _ptr(pairs), _ptr(cos_t), _ptr(sin_t),
+                                           _ptr(scale), _ptr(qweight), _ptr(_u16(scales)), _ptr(_u16(zeros)),
+                                           _ptr(_u16(out)), M, d_in, d_out, group_size, _stream(stream))
+    _check(st, "paro_rotate_w4_linear_noalloc")
     return out
 
 

@@ -99,6 +99,16 @@ paro_status check_weights(const uint32_t* qweight, const uint16_t* scales, const
 
 }  // namespace
 
+namespace paro {
+paro_status record_error(paro_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+}  // namespace paro
+
 extern "C" {
 
 int paro_weight_layout_version(void) { return 1; }

@@ -1,0 +1,76 @@
+// paro_rotate_w4_linear_noalloc: the fused rotate + INT4 linear for callers
+// that cannot allocate device memory.
+//
+// Who cannot allocate: code that runs where cudaMalloc/cudaFree are off
+// limits, e.g. a plugin hosted by an inference engine that owns every byte of
+// device memory and hands its plugins no workspace, a latency-critical path
+// that must not take the implicit device synchronisation cudaFree can cause,
+// or a program that reserves all of its memory at start-up and forbids any
+// allocation afterwards.  Those callers still own their inputs and outputs;
+// only the fused call's scratch (the transformed activations in fp16) is
+// provided here, by a fixed device array that the library carries.
+//
+// The array is a file-scope __device__ variable: every GPU that loads this
+// library holds kNoAllocMaxElems fp16 values (512 KiB) until the process
+// exits.  Host code cannot use the array's name as a device address (it is a
+// host-side stand-in), so the entry point looks the address up once per
+// device with cudaGetSymbolAddress, with that device current, and passes it
+// to the kernels as their workspace.
+#include <atomic>
+
+#include "paro_internal.cuh"
+
+namespace {
+
+// M * d_in of one call may not exceed this many fp16 elements (e.g. M = 16
+// tokens of width 16384, or one token of width 49152).
+constexpr size_t kNoAllocMaxElems = size_t(1) << 18;
+
+static __device__ __align__(256) __half g_noalloc_scratch[kNoAllocMaxElems];
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_scratch_addr[kMaxDevices];
+
+// Device address of the scratch array on the current device; looked up on the
+// first call made on each device.
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" paro_status paro_rotate_w4_linear_noalloc(const uint16_t* d_x, int K, const uint16_t* d_pairs,
+                                                     const float* d_cos, const float* d_sin, const float* d_scale,
+                                                     const uint32_t* d_qweight, const uint16_t* d_scales,
+                                                     const uint16_t* d_zeros, uint16_t* d_y, int M, int d_in,
+                                                     int d_out, int group_size, paro_stream_t stream) {
+  if (M > 0 && d_in > 0 && (size_t)M * (size_t)d_in > kNoAllocMaxElems) {
+    return paro::record_error(PARO_ERR_UNSUPPORTED,
+                              "paro_rotate_w4_linear_noalloc: M * d_in = %zu exceeds the built-in scratch of %zu "
+                              "fp16 values; use paro_rotate_w4_linear with a caller-provided workspace",
+                              (size_t)M * (size_t)d_in, kNoAllocMaxElems);
+  }
+  void* scratch = nullptr;
+  if (M > 0) {
+    cudaError_t e = scratch_address(&scratch);
+    if (e != cudaSuccess)
+      return paro::record_error(PARO_ERR_CUDA, "paro_rotate_w4_linear_noalloc: scratch address lookup: %s",
+                                cudaGetErrorString(e));
+  }
+  // Same validation and kernels as the workspace-taking call; nothing here
+  // needs to start at zero because the transform overwrites every scratch
+  // value it hands to the linear.
+  return paro_rotate_w4_linear(d_x, K, d_pairs, d_cos, d_sin, d_scale, d_qweight, d_scales, d_zeros, d_y, M,
+                               d_in, d_out, group_size, scratch, kNoAllocMaxElems * sizeof(__half), stream);
+}

@@ -22,6 +22,9 @@ __device__ __forceinline__ void report_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Stores a printf-style message for paro_last_error() and returns s.
+paro_status record_error(paro_status s, const char* fmt, ...);
+
 // ---- launchers implemented in the kernel translation units --------------------
 // All return a cudaError_t from the launch (cudaSuccess when nothing failed).
 
