@@ -358,6 +358,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--variants", default="fused,plain,unfused,rotate")
+    ap.add_argument("--profile", action="store_true",
+                    help="run only the listed variants (no end-to-end leg, no CPU baseline): a fixed, short "
+                         "launch sequence for ncu; its numbers are not bench values")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -398,13 +401,13 @@ def main():
         return sum(linear_bytes(l.d_in, l.d_out, M, unfused=(variant == "unfused")) for l in step_lins)
 
     variants = [v for v in args.variants.split(",") if v]
-    if "fused" not in variants:
+    if "fused" not in variants and not args.profile:
         variants.insert(0, "fused")
     results = {}
     clocks = None
     for v in variants:
         graphs = capture(torch, paro, units, v)
-        if v == "fused":
+        if v == "fused" and not args.profile:
             with ClockSampler(_smi_id(torch)) as cs:
                 ms = time_graphs(torch, graphs, args.steps, args.warmup, dist)
             clocks = cs.summary()
@@ -412,6 +415,12 @@ def main():
             ms = time_graphs(torch, graphs, args.steps, args.warmup, dist)
         results[v] = ms
         del graphs
+    if args.profile:
+        if rank == 0:
+            print(json.dumps({"profile_run": True, "variants_ms_per_step": results}), flush=True)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
     # end to end: per step the inputs come from pinned host memory and outputs go back
     graphs = capture(torch, paro, units, "fused_e2e")
     ms_e2e = time_graphs(torch, graphs, args.steps, args.warmup, dist)
