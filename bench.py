@@ -122,8 +122,45 @@ class Linear:
         self.y_host.copy_(self.y, non_blocking=True)
 
 
-# kernels launched per call of each variant
+# kernels launched per linear of each variant (batched: 2 per call of up to 7 linears)
 LAUNCHES = {"fused": 2, "unfused": 2, "plain": 1, "rotate": 1, "fused_e2e": 2}
+BATCH = 7  # linears per batched call (one decoder layer)
+
+
+class Unit:
+    """The linears of one step; runs them per linear or as batched calls."""
+
+    def __init__(self, lins, paro):
+        self.lins = lins
+        self.calls = []
+        for i in range(0, len(lins), BATCH):
+            grp = lins[i:i + BATCH]
+            descs = [paro.paro_linear(l.x, l.pairs, l.cos, l.sin, l.scale, l.qw, l.sc, l.z, l.y) for l in grp]
+            plain = [paro.paro_linear(l.x, None, None, None, None, l.qw0, l.sc0, l.z0, l.y) for l in grp]
+            need = paro.paro_batched_workspace_bytes(descs)
+            ws = __import__("torch").empty(max(need, 256), dtype=__import__("torch").uint8, device=lins[0].x.device)
+            self.calls.append((grp, descs, plain, ws))
+
+    def run(self, paro, variant):
+        if variant in ("batched", "batched_e2e", "batched_plain"):
+            for grp, descs, plain, ws in self.calls:
+                if variant == "batched_e2e":
+                    for l in grp:
+                        l.x.copy_(l.x_host, non_blocking=True)
+                paro.paro_rotate_w4_linear_batched(plain if variant == "batched_plain" else descs, workspace=ws)
+                if variant == "batched_e2e":
+                    for l in grp:
+                        l.y_host.copy_(l.y, non_blocking=True)
+        else:
+            for lin in self.lins:
+                getattr(lin, variant)(paro)
+
+    def launches(self, variant):
+        if variant == "batched_plain":
+            return len(self.calls)
+        if variant.startswith("batched"):
+            return 2 * len(self.calls)
+        return LAUNCHES[variant] * len(self.lins)
 
 
 def build_layers(config, M, n_layers, rank, dev):
@@ -147,24 +184,21 @@ def capture(torch, paro, units, variant):
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         for unit in units:           # warm the launch path outside capture
-            for lin in unit:
-                getattr(lin, variant)(paro)
+            unit.run(paro, variant)
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
     per_unit = []
     for unit in units:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            for lin in unit:
-                getattr(lin, variant)(paro)
+            unit.run(paro, variant)
         per_unit.append(g)
     cycle = None
     if len(units) > 1:
         cycle = torch.cuda.CUDAGraph()
         with torch.cuda.graph(cycle):
             for unit in units:
-                for lin in unit:
-                    getattr(lin, variant)(paro)
+                unit.run(paro, variant)
     return per_unit, cycle
 
 
@@ -357,7 +391,7 @@ def main():
     ap.add_argument("--M", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--variants", default="fused,plain,unfused,rotate")
+    ap.add_argument("--variants", default="batched,batched_plain,fused,plain,unfused,rotate")
     ap.add_argument("--profile", action="store_true",
                     help="run only the listed variants (no end-to-end leg, no CPU baseline): a fixed, short "
                          "launch sequence for ncu; its numbers are not bench values")
@@ -389,8 +423,8 @@ def main():
     name, shapes, M, n_layers, stack = workload(args.config, args.M)
     layers = build_layers(args.config, M, n_layers, rank, dev)
     torch.cuda.synchronize()
-    units = [sum(layers, [])] if stack else layers
-    step_lins = units[0]
+    units = [Unit(sum(layers, []), paro)] if stack else [Unit(l, paro) for l in layers]
+    step_lins = units[0].lins
     flops_step = sum(2 * M * l.d_in * l.d_out for l in step_lins)
 
     def bytes_of(variant):
@@ -401,13 +435,13 @@ def main():
         return sum(linear_bytes(l.d_in, l.d_out, M, unfused=(variant == "unfused")) for l in step_lins)
 
     variants = [v for v in args.variants.split(",") if v]
-    if "fused" not in variants and not args.profile:
-        variants.insert(0, "fused")
+    if "batched" not in variants and not args.profile:
+        variants.insert(0, "batched")
     results = {}
     clocks = None
     for v in variants:
         graphs = capture(torch, paro, units, v)
-        if v == "fused" and not args.profile:
+        if v == "batched" and not args.profile:
             with ClockSampler(_smi_id(torch)) as cs:
                 ms = time_graphs(torch, graphs, args.steps, args.warmup, dist)
             clocks = cs.summary()
@@ -422,19 +456,21 @@ def main():
             dist.destroy_process_group()
         return
     # end to end: per step the inputs come from pinned host memory and outputs go back
-    graphs = capture(torch, paro, units, "fused_e2e")
+    graphs = capture(torch, paro, units, "batched_e2e")
     ms_e2e = time_graphs(torch, graphs, args.steps, args.warmup, dist)
     del graphs
     h2d = sum(l.x.numel() * 2 for l in step_lins)
     d2h = sum(l.y.numel() * 2 for l in step_lins)
 
-    ms = results["fused"]
+    ms = results["batched"]
     step_bytes = bytes_of("fused")
     value = step_bytes * world / (ms * 1e-3) / 1e9
     e2e_value = (step_bytes + h2d + d2h) * world / (ms_e2e * 1e-3) / 1e9
     plain_ms = results.get("plain")
-    # dominant kernel: the INT4 linear, timed alone (plain weights: no transform)
-    w4_gbs = bytes_of("plain") / (plain_ms * 1e-3) / 1e9 if plain_ms else None
+    # dominant kernel: the INT4 linear, timed alone (plain weights, no transform:
+    # one launch per batched call when that variant ran, else one per linear)
+    w4_ms = results.get("batched_plain", plain_ms)
+    w4_gbs = bytes_of("plain") / (w4_ms * 1e-3) / 1e9 if w4_ms else None
     rot_gbs = bytes_of("rotate") / (results["rotate"] * 1e-3) / 1e9 if "rotate" in results else None
     prefill = M >= 512
 
@@ -445,8 +481,8 @@ def main():
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {
-            "workload": f"{name}: fused rotate + INT4 linear, M={M}, K={K_STAGES}, group={GROUP}, "
-                        f"asymmetric INT4, bf16 activations",
+            "workload": f"{name}: fused rotate + INT4 linear (one batched C-ABI call per {BATCH} linears), "
+                        f"M={M}, K={K_STAGES}, group={GROUP}, asymmetric INT4, bf16 activations",
             "linears_per_step": len(step_lins), "distinct_units_cycled": len(units),
             "l2": ("inputs larger than L2: each step streams a different layer's weights "
                    f"({len(units)} units, {sum(bytes_of('fused') for _ in units) / 1e9:.2f} GB)") if len(units) > 1
@@ -456,26 +492,31 @@ def main():
         "roofline": {
             "bound": "hbm", "achieved": round(w4_gbs, 1) if w4_gbs else None, "peak": hbm, "unit": "GB/s",
             "frac": round(w4_gbs / hbm, 4) if w4_gbs else None, "traffic": None,
-            "kernel": "w4_mma_kernel (INT4 linear), algorithmic bytes / device time",
+            "kernel": "w4_gemv_kernel (INT4 linear; one launch per batched call of a step's linears), "
+                      "algorithmic bytes / device time",
             "peak_kind": f"{peak_kind} HBM copy bandwidth",
         },
         "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e, 6)},
-        "gpu_launches": LAUNCHES["fused"] * len(step_lins) * args.steps,
+        "gpu_launches": units[0].launches("batched") * args.steps,
         "clocks": clocks,
         "variants_ms_per_step": {k: round(v, 6) for k, v in results.items()},
-        "rotation_overhead_pct": round(100 * (ms - plain_ms) / plain_ms, 2) if plain_ms else None,
+        "rotation_overhead_pct": (round(100 * (ms - results["batched_plain"]) / results["batched_plain"], 2)
+                                  if "batched_plain" in results else None),
+        "rotation_overhead_vs_per_linear_plain_pct": round(100 * (ms - plain_ms) / plain_ms, 2) if plain_ms else None,
         "rotation_overhead_unfused_pct": (round(100 * (results["unfused"] - plain_ms) / plain_ms, 2)
                                           if plain_ms and "unfused" in results else None),
+        "rotation_overhead_per_linear_fused_pct": (round(100 * (results["fused"] - plain_ms) / plain_ms, 2)
+                                                   if plain_ms and "fused" in results else None),
         "rotate_kernel_gbs": round(rot_gbs, 1) if rot_gbs else None,
         "tokens_per_s": round(M * world / (ms * 1e-3), 1),
         "tflops": round(flops_step * world / (ms * 1e-3) / 1e12, 3),
         "hbm_frac_of_measured": round(value / hbm, 4),
     }
     if prefill:
-        out["roofline"] = {"bound": "tensor", "achieved": round(flops_step / (plain_ms * 1e-3) / 1e12, 2),
+        out["roofline"] = {"bound": "tensor", "achieved": round(flops_step / (w4_ms * 1e-3) / 1e12, 2),
                            "peak": bf16, "unit": "TFLOP/s",
-                           "frac": round(flops_step / (plain_ms * 1e-3) / 1e12 / bf16, 4), "traffic": None,
+                           "frac": round(flops_step / (w4_ms * 1e-3) / 1e12 / bf16, 4), "traffic": None,
                            "kernel": "INT4 linear, 2*M*d_in*d_out / device time",
                            "peak_kind": f"{peak_kind} bf16 dense (f16 operands: same nominal rate)"}
     if rank == 0 and not args.no_cpu:

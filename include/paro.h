@@ -150,6 +150,48 @@ PARO_API paro_status paro_rotate_w4_linear(const uint16_t* d_x, int K, const uin
                                   paro_stream_t stream);
 
 /*
+ * One linear layer of a batch for paro_rotate_w4_linear_batched: the same
+ * arguments as paro_rotate_w4_linear, gathered in a host-side struct.
+ */
+typedef struct {
+  const uint16_t* d_x;        /* bf16 [M][d_in] */
+  uint16_t* d_y;              /* bf16 [M][d_out], overlapping no input of the batch */
+  int M, d_in, d_out, K;
+  const uint16_t* d_pairs;    /* [K][d_in/2][2] */
+  const float* d_cos;         /* [K][d_in/2] */
+  const float* d_sin;         /* [K][d_in/2] */
+  const float* d_scale;       /* [d_in] or NULL */
+  const uint32_t* d_qweight;  /* [d_out][d_in/8], layout version 1 */
+  const uint16_t* d_scales;   /* fp16 [d_out][d_in/128] */
+  const uint16_t* d_zeros;    /* fp16 [d_out][d_in/128] */
+} paro_linear;
+
+/* Largest number of linears one paro_rotate_w4_linear_batched call takes. */
+#define PARO_MAX_BATCH 8
+
+/* Workspace bytes paro_rotate_w4_linear_batched needs for these linears. */
+PARO_API size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int count);
+
+/*
+ * Runs paro_rotate_w4_linear for up to PARO_MAX_BATCH independent linears with
+ * two kernel launches in all (one transform launch, one INT4-linear launch),
+ * e.g. the seven linears of one decoder layer; each linear has its own
+ * transform ("one rotation operator plus one group-wise INT4 GEMM operator for
+ * each layer", page "ParoQuant: pairwise rotations that survive deployment",
+ * section "From fake quantization to a real TensorRT engine").  h_layers is a
+ * HOST array read during the call; d_workspace holds
+ * paro_batched_workspace_bytes(h_layers, count) bytes (256-byte aligned,
+ * caller-owned, undefined between calls).  Results equal count separate calls
+ * of paro_rotate_w4_linear.  Every linear is validated before anything is
+ * enqueued; the message of paro_last_error() names the failing index.  When no
+ * linear has a transform (K == 0 and d_scale == NULL for all), only the INT4
+ * linear launch runs, on the bf16 inputs, and d_workspace may be NULL.
+ */
+PARO_API paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count, int group_size,
+                                                  void* d_workspace, size_t workspace_bytes,
+                                                  paro_stream_t stream);
+
+/*
  * The same computation as paro_rotate_w4_linear for callers that cannot
  * allocate device memory (the paper has no counterpart: this is an interface
  * convenience of this library).  Instead of a caller-provided workspace, the

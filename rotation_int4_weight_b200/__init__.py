@@ -17,7 +17,8 @@ import torch
 __all__ = [
     "ParoError", "LIB_PATH", "lib", "paro_weight_layout_version", "paro_workspace_bytes",
     "paro_pack_weights", "paro_rotate", "paro_w4_linear", "paro_rotate_w4_linear",
-    "paro_rotate_w4_linear_noalloc", "paro_get_device_status", "EXPORTED",
+    "paro_rotate_w4_linear_noalloc", "paro_get_device_status", "EXPORTED", "ParoLinear", "paro_linear",
+    "paro_batched_workspace_bytes", "paro_rotate_w4_linear_batched",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libparo.so")
@@ -34,8 +35,17 @@ EXPORTED = {
     "paro_workspace_bytes": (_S, [_I, _I]),
     "paro_rotate_w4_linear": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
     "paro_rotate_w4_linear_noalloc": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "paro_batched_workspace_bytes": (_S, [_P, _I]),
+    "paro_rotate_w4_linear_batched": (_I, [_P, _I, _I, _P, _S, _P]),
     "paro_get_device_status": (_I, [_P]),
 }
+
+
+class ParoLinear(ctypes.Structure):
+    """Host-side description of one linear (the C struct paro_linear)."""
+    _fields_ = [("d_x", _P), ("d_y", _P), ("M", _I), ("d_in", _I), ("d_out", _I), ("K", _I),
+                ("d_pairs", _P), ("d_cos", _P), ("d_sin", _P), ("d_scale", _P),
+                ("d_qweight", _P), ("d_scales", _P), ("d_zeros", _P)]
 
 
 class ParoError(RuntimeError):
@@ -182,6 +192,31 @@ def paro_rotate_w4_linear_noalloc(x: torch.Tensor, pairs, cos_t, sin_t, scale, q
                                            _ptr(_u16(out)), M, d_in, d_out, group_size, _stream(stream))
     _check(st, "paro_rotate_w4_linear_noalloc")
     return out
+
+
+def paro_linear(x, pairs, cos_t, sin_t, scale, qweight, scales, zeros, out) -> ParoLinear:
+    """Describe one linear for paro_rotate_w4_linear_batched (tensors stay owned by the caller)."""
+    def p(t):
+        return None if t is None else _ptr(t).value
+    return ParoLinear(p(_u16(x)), p(_u16(out)), x.shape[0], x.shape[1], qweight.shape[0], _K(pairs), p(pairs),
+                      p(cos_t), p(sin_t), p(scale), p(qweight), p(_u16(scales)), p(_u16(zeros)))
+
+
+def paro_batched_workspace_bytes(layers) -> int:
+    arr = (ParoLinear * len(layers))(*layers)
+    return int(lib.paro_batched_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), len(layers)))
+
+
+def paro_rotate_w4_linear_batched(layers, *, workspace=None, group_size: int = 128, stream=None):
+    """Run a list of ParoLinear descriptions (at most 8) with two kernel launches."""
+    arr = (ParoLinear * len(layers))(*layers)
+    need = int(lib.paro_batched_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), len(layers)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+    st = lib.paro_rotate_w4_linear_batched(ctypes.cast(arr, ctypes.c_void_p), len(layers), group_size,
+                                           _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "paro_rotate_w4_linear_batched")
+    return workspace
 
 
 def paro_get_device_status(stream=None) -> int:

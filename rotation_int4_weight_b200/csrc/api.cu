@@ -8,6 +8,8 @@
 #include <cstring>
 
 #include "paro_internal.cuh"
+#include "w4_gemv.cuh"
+#include "rotate_decode.cuh"
 
 namespace {
 
@@ -97,6 +99,62 @@ paro_status check_weights(const uint32_t* qweight, const uint16_t* scales, const
   return PARO_OK;
 }
 
+// The INT4 linear on x (bf16, or fp16 when x_f16).  With pdl_wait the kernel is
+// launched as a programmatic dependent of the previous kernel in the stream and
+// waits for it before reading x (the weights may be read earlier, so only a
+// previous kernel that does not write them may trigger early).
+cudaError_t launch_linear(const uint16_t* x, bool x_f16, const uint32_t* qweight, const uint16_t* scales,
+                          const uint16_t* zeros, uint16_t* y, int M, int d_in, int d_out, cudaStream_t s,
+                          bool pdl_wait) {
+  paro::GemvProblem p = {};
+  p.x = x;
+  p.qw = qweight;
+  p.sc = reinterpret_cast<const __half*>(scales);
+  p.z = reinterpret_cast<const __half*>(zeros);
+  p.y = reinterpret_cast<__nv_bfloat16*>(y);
+  p.M = M;
+  p.d_in = d_in;
+  p.d_out = d_out;
+  paro::GemvBatch b;
+  int nt = 1;
+  cudaError_t e = paro::plan_gemv_batch(&p, 1, x_f16, &b, &nt);
+  if (e != cudaSuccess) return e;
+  return paro::launch_gemv_batch(b, nt, s, pdl_wait);
+}
+
+// Prefixes the current error message with the index of the failing layer.
+paro_status prefix_error(paro_status st, int layer) {
+  char msg[sizeof(t_last_error)];
+  snprintf(msg, sizeof(msg), "%s", t_last_error);
+  return fail(st, "layer %d: %s", layer, msg);
+}
+
+// Activation transform of one linear: the table-prefetching decode kernel for
+// few rows, the row-block kernel otherwise.
+cudaError_t launch_transform(const uint16_t* x, void* out, bool f16_out, int M, int d, int K,
+                             const uint16_t* pairs, const float* c, const float* s, const float* scale,
+                             int* status, cudaStream_t stream, bool pdl_trigger) {
+  if (M <= 64 && (K == 0 || paro::rot_decode_supported(d, pairs, c, s))) {
+    paro::RotProblem p = {};
+    p.x = x;
+    p.out = out;
+    p.M = M;
+    p.d = d;
+    p.K = K;
+    p.pairs = reinterpret_cast<const uint32_t*>(pairs);
+    p.cos_t = c;
+    p.sin_t = s;
+    p.scale = scale;
+    paro::RotBatch b;
+    int R = 1;
+    cudaError_t e = paro::plan_rot_batch(&p, 1, &b, &R);
+    if (e != cudaSuccess) return e;
+    return paro::launch_rot_batch(b, R, f16_out, status, stream, pdl_trigger);
+  }
+  return paro::launch_rotate_act(x, out, f16_out ? 1 : 0, M, d, K, pairs, c, s, scale, status, stream,
+                                 pdl_trigger);
+}
+
 }  // namespace
 
 namespace paro {
@@ -177,8 +235,8 @@ paro_status paro_rotate(const uint16_t* d_x, uint16_t* d_x_rot, int M, int d, in
     return fail(PARO_ERR_INVALID_ARG, "x_rot partially overlaps x (only exact in-place is allowed)");
   int* status = status_ptr();
   if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
-  cudaError_t e = paro::launch_rotate_act(d_x, d_x_rot, 0, M, d, K, d_pairs, d_cos, d_sin, d_scale, status,
-                                          reinterpret_cast<cudaStream_t>(stream), false);
+  cudaError_t e = launch_transform(d_x, d_x_rot, false, M, d, K, d_pairs, d_cos, d_sin, d_scale, status,
+                                   reinterpret_cast<cudaStream_t>(stream), false);
   return from_cuda(e, "rotate launch");
 }
 
@@ -196,10 +254,8 @@ paro_status paro_w4_linear(const uint16_t* d_x, const uint32_t* d_qweight, const
       overlap(d_y, yb, d_scales, (size_t)d_out * (d_in / 128) * 2) ||
       overlap(d_y, yb, d_zeros, (size_t)d_out * (d_in / 128) * 2))
     return fail(PARO_ERR_INVALID_ARG, "y overlaps an input");
-  cudaError_t e = paro::launch_w4_linear_mma(d_x, 0, d_qweight, reinterpret_cast<const __half*>(d_scales),
-                                             reinterpret_cast<const __half*>(d_zeros),
-                                             reinterpret_cast<__nv_bfloat16*>(d_y), M, d_in, d_out,
-                                             reinterpret_cast<cudaStream_t>(stream), false);
+  cudaError_t e = launch_linear(d_x, false, d_qweight, d_scales, d_zeros, d_y, M, d_in, d_out,
+                                reinterpret_cast<cudaStream_t>(stream), false);
   return from_cuda(e, "w4 linear launch");
 }
 
@@ -234,13 +290,120 @@ paro_status paro_rotate_w4_linear(const uint16_t* d_x, int K, const uint16_t* d_
   int* status = status_ptr();
   if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = paro::launch_rotate_act(d_x, d_workspace, 1, M, d_in, K, d_pairs, d_cos, d_sin, d_scale,
-                                          status, s, true);
+  cudaError_t e = launch_transform(d_x, d_workspace, true, M, d_in, K, d_pairs, d_cos, d_sin, d_scale, status, s,
+                                   true);
   if (e != cudaSuccess) return from_cuda(e, "rotate launch");
-  e = paro::launch_w4_linear_mma(d_workspace, 1, d_qweight, reinterpret_cast<const __half*>(d_scales),
-                                 reinterpret_cast<const __half*>(d_zeros), reinterpret_cast<__nv_bfloat16*>(d_y),
-                                 M, d_in, d_out, s, true);
+  e = launch_linear(static_cast<const uint16_t*>(d_workspace), true, d_qweight, d_scales, d_zeros, d_y, M, d_in,
+                    d_out, s, true);
   return from_cuda(e, "w4 linear launch");
+}
+
+size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int count) {
+  if (!h_layers || count <= 0) return 0;
+  size_t b = 0;
+  for (int i = 0; i < count; ++i) b += paro_workspace_bytes(h_layers[i].M, h_layers[i].d_in);
+  return b;
+}
+
+paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count, int group_size,
+                                          void* d_workspace, size_t workspace_bytes, paro_stream_t stream) {
+  if (count == 0) return ok();
+  if (!h_layers || count < 0) return fail(PARO_ERR_INVALID_ARG, "null layer array or negative count");
+  if (count > PARO_MAX_BATCH) return fail(PARO_ERR_UNSUPPORTED, "count = %d exceeds %d", count, PARO_MAX_BATCH);
+  const size_t need = paro_batched_workspace_bytes(h_layers, count);
+  paro::RotProblem rp[PARO_MAX_BATCH];
+  paro::GemvProblem gp[PARO_MAX_BATCH];
+  int n = 0;
+  size_t off = 0;
+  bool decode_ok = true, any_transform = false;
+  for (int i = 0; i < count; ++i) {
+    const paro_linear& L = h_layers[i];
+    paro_status st;
+    if ((st = check_linear_shape(L.M, L.d_in, L.d_out, group_size)) != PARO_OK ||
+        (st = check_width(L.d_in)) != PARO_OK ||
+        (st = check_tables(L.K, L.d_in, L.d_pairs, L.d_cos, L.d_sin, L.d_scale)) != PARO_OK)
+      return prefix_error(st, i);
+    if (L.M == 0) continue;
+    if ((st = check_weights(L.d_qweight, L.d_scales, L.d_zeros)) != PARO_OK)
+      return prefix_error(st, i);
+    if (!L.d_x || !L.d_y || !aligned(L.d_x, 16) || !aligned(L.d_y, 16))
+      return fail(PARO_ERR_INVALID_ARG, "layer %d: x and y must be non-null and 16-byte aligned", i);
+    const size_t yb = (size_t)L.M * L.d_out * 2;
+    for (int j = 0; j < count; ++j) {
+      const paro_linear& O = h_layers[j];
+      if (O.M == 0) continue;
+      if (overlap(L.d_y, yb, O.d_x, (size_t)O.M * O.d_in * 2) ||
+          overlap(L.d_y, yb, O.d_qweight, (size_t)O.d_out * O.d_in / 2) ||
+          (j != i && overlap(L.d_y, yb, O.d_y, (size_t)O.M * O.d_out * 2)))
+        return fail(PARO_ERR_INVALID_ARG, "layer %d: y overlaps an input or output of layer %d", i, j);
+    }
+    if (L.M > 64 || (L.K > 0 && !paro::rot_decode_supported(L.d_in, L.d_pairs, L.d_cos, L.d_sin)))
+      decode_ok = false;
+    if (L.K > 0 || L.d_scale) any_transform = true;
+    uint16_t* xt = reinterpret_cast<uint16_t*>(static_cast<char*>(d_workspace) + off);
+    off += paro_workspace_bytes(L.M, L.d_in);
+    rp[n] = paro::RotProblem{};
+    rp[n].x = L.d_x;
+    rp[n].out = xt;
+    rp[n].M = L.M;
+    rp[n].d = L.d_in;
+    rp[n].K = L.K;
+    rp[n].pairs = reinterpret_cast<const uint32_t*>(L.d_pairs);
+    rp[n].cos_t = L.d_cos;
+    rp[n].sin_t = L.d_sin;
+    rp[n].scale = L.d_scale;
+    gp[n] = paro::GemvProblem{};
+    gp[n].x = xt;
+    gp[n].qw = L.d_qweight;
+    gp[n].sc = reinterpret_cast<const __half*>(L.d_scales);
+    gp[n].z = reinterpret_cast<const __half*>(L.d_zeros);
+    gp[n].y = reinterpret_cast<__nv_bfloat16*>(L.d_y);
+    gp[n].M = L.M;
+    gp[n].d_in = L.d_in;
+    gp[n].d_out = L.d_out;
+    ++n;
+  }
+  if (n == 0) return ok();
+  if (any_transform && (!d_workspace || workspace_bytes < need || !aligned(d_workspace, 256)))
+    return fail(PARO_ERR_INVALID_ARG, "workspace must be 256-byte aligned and hold %zu bytes", need);
+  for (int i = 0; i < count && any_transform; ++i) {
+    const paro_linear& L = h_layers[i];
+    if (L.M == 0) continue;
+    if (overlap(d_workspace, need, L.d_x, (size_t)L.M * L.d_in * 2) ||
+        overlap(d_workspace, need, L.d_y, (size_t)L.M * L.d_out * 2))
+      return fail(PARO_ERR_INVALID_ARG, "layer %d: workspace overlaps x or y", i);
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (!any_transform) {
+    // no layer has a transform: the INT4 linear reads the bf16 inputs directly
+    for (int i = 0; i < n; ++i) gp[i].x = rp[i].x;
+    paro::GemvBatch gb;
+    int nt = 1;
+    e = paro::plan_gemv_batch(gp, n, false, &gb, &nt);
+    if (e == cudaSuccess) e = paro::launch_gemv_batch(gb, nt, s, false);
+    return from_cuda(e, "batched w4 linear launch");
+  }
+  int* status = status_ptr();
+  if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
+  if (decode_ok) {
+    paro::RotBatch rb;
+    int R = 1;
+    e = paro::plan_rot_batch(rp, n, &rb, &R);
+    if (e == cudaSuccess) e = paro::launch_rot_batch(rb, R, true, status, s, true);
+  } else {
+    e = cudaSuccess;
+    for (int i = 0; i < n && e == cudaSuccess; ++i)
+      e = launch_transform(rp[i].x, rp[i].out, true, rp[i].M, rp[i].d, rp[i].K,
+                           reinterpret_cast<const uint16_t*>(rp[i].pairs), rp[i].cos_t, rp[i].sin_t, rp[i].scale,
+                           status, s, i == n - 1);
+  }
+  if (e != cudaSuccess) return from_cuda(e, "batched transform launch");
+  paro::GemvBatch gb;
+  int nt = 1;
+  e = paro::plan_gemv_batch(gp, n, true, &gb, &nt);
+  if (e == cudaSuccess) e = paro::launch_gemv_batch(gb, nt, s, true);
+  return from_cuda(e, "batched w4 linear launch");
 }
 
 paro_status paro_get_device_status(paro_stream_t stream) {

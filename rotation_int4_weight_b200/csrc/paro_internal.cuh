@@ -42,9 +42,4 @@ cudaError_t launch_fold_weights(const float* W, float* out, int rows, int d, int
 cudaError_t launch_quantize_pack(const float* Wt, int d_out, int d_in, uint32_t* qweight,
                                  __half* scales, __half* zeros, cudaStream_t stream);
 
-// INT4 linear, M small or large, x in bf16 (x_is_f16 = 0) or fp16 (1).
-cudaError_t launch_w4_linear_mma(const void* x, int x_is_f16, const uint32_t* qweight,
-                                 const __half* scales, const __half* zeros, __nv_bfloat16* y,
-                                 int M, int d_in, int d_out, cudaStream_t stream, bool pdl_wait);
-
 }  // namespace paro

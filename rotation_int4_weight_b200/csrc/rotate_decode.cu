@@ -1,0 +1,301 @@
+// Activation-side transform for few tokens (decode), several linears per launch:
+//   x~ = diag(1/s) R_K ... R_1 x
+// (page "ParoQuant: pairwise rotations that survive deployment", section "A
+// rotation small enough to execute": disjoint channel pairs per stage, each
+// rotated by x_i' = c x_i + s x_j, x_j' = -s x_i + c x_j; channel scale last).
+//
+// With one or a few token rows the work per stage is tiny and the time goes
+// into fetching the stage tables (12 bytes per pair and stage), so the tables
+// are requested up front: one thread of every CTA issues bulk (TMA) copies of
+// as many whole stages (pairs, cos, sin) as fit in shared memory before the
+// rows are touched, each stage completing on its own mbarrier, and refills a
+// slot as soon as its stage is done.  Bulk copies keep a single SM's stream of
+// table bytes deep without one request per 16 bytes.  Waits are bounded: a
+// stage that never lands is reported as PARO_ERR_TIMEOUT.  The rows themselves live in
+// shared memory as fp32 (channel-major, R rows per channel) after one bulk copy
+// of the rows and the scales, and each stage is one pass over its disjoint
+// pairs followed by one barrier.
+#include "paro_internal.cuh"
+#include "rotate_decode.cuh"
+
+namespace paro {
+namespace {
+
+constexpr int kRotThreads = 1024;
+constexpr int kMaxRing = 8;
+constexpr size_t kRotSmemBudget = 227 * 1024 - 256;
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Waits for phase `parity` of an mbarrier; gives up after about a second of
+// SM clock (then returns false and the caller reports PARO_ERR_TIMEOUT).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_test(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_test(bar, parity))
+    if (clock64() - t0 > (1LL << 31)) return false;
+  return true;
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+template <int R>
+__device__ __forceinline__ void ld_rows(const float* p, float (&v)[R]) {
+  if constexpr (R == 1) {
+    v[0] = *p;
+  } else if constexpr (R == 2) {
+    const float2 t = *reinterpret_cast<const float2*>(p);
+    v[0] = t.x; v[1] = t.y;
+  } else {
+    const float4 t = *reinterpret_cast<const float4*>(p);
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  }
+}
+template <int R>
+__device__ __forceinline__ void st_rows(float* p, const float (&v)[R]) {
+  if constexpr (R == 1) {
+    *p = v[0];
+  } else if constexpr (R == 2) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  } else {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+template <int R, bool F16OUT>
+__global__ void __launch_bounds__(kRotThreads)
+rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_trigger) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ __align__(8) uint64_t bars[kMaxRing + 1];
+  if (pdl_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  int pi = 0;
+#pragma unroll 1
+  while (pi + 1 < batch.count && (int)blockIdx.x >= batch.p[pi + 1].cta_begin) ++pi;
+  const RotProblem& P = batch.p[pi];
+  const int d = P.d, K = P.K, half = d >> 1, ring = P.ring;
+  const int row0 = ((int)blockIdx.x - P.cta_begin) * R;
+  const int nrows = min(R, P.M - row0);
+  const int tid = threadIdx.x;
+
+  // shared memory: xs [d][R] fp32 | x staging [R][d] bf16 | factors [d] fp32 | ring [ring][6d]
+  float* xs = reinterpret_cast<float*>(smem);
+  __nv_bfloat16* xst = reinterpret_cast<__nv_bfloat16*>(xs + (size_t)d * R);
+  float* fac = reinterpret_cast<float*>(xst + (size_t)d * R);
+  unsigned char* tab = reinterpret_cast<unsigned char*>(fac + d);
+  const size_t stage_bytes = (size_t)6 * d;  // pairs | cos | sin
+  const uint32_t s_tab = static_cast<uint32_t>(__cvta_generic_to_shared(tab));
+  const uint32_t s_bar = static_cast<uint32_t>(__cvta_generic_to_shared(bars));
+  const uint32_t bar_in = s_bar + 8u * kMaxRing;  // rows and scale
+  const bool scale_bulk = P.scale && (reinterpret_cast<uintptr_t>(P.scale) & 15) == 0;
+
+  // one thread requests whole stages with bulk copies (three per stage); the
+  // stage's mbarrier completes when all 6d bytes have landed
+  auto issue_stage = [&](int k) {
+    if (k < K) {
+      const int slot = k % ring;
+      const uint32_t base = s_tab + (uint32_t)(slot * stage_bytes), bar = s_bar + 8u * slot;
+      mbar_expect_tx(bar, (uint32_t)stage_bytes);
+      bulk_g2s(base, P.pairs + (size_t)k * half, 2u * d, bar);
+      bulk_g2s(base + 2u * d, P.cos_t + (size_t)k * half, 2u * d, bar);
+      bulk_g2s(base + 4u * d, P.sin_t + (size_t)k * half, 2u * d, bar);
+    }
+  };
+  if (tid == 0) {
+    for (int k = 0; k <= kMaxRing; ++k) mbar_init(s_bar + 8u * k, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    const uint32_t in_bytes = (uint32_t)(nrows * 2 * d) + (scale_bulk ? 4u * d : 0u);
+    mbar_expect_tx(bar_in, in_bytes);
+    bulk_g2s(static_cast<uint32_t>(__cvta_generic_to_shared(xst)), P.x + (size_t)row0 * d, (uint32_t)(nrows * 2 * d),
+             bar_in);
+    if (scale_bulk) bulk_g2s(static_cast<uint32_t>(__cvta_generic_to_shared(fac)), P.scale, 4u * d, bar_in);
+    for (int k = 0; k < ring; ++k) issue_stage(k);
+  }
+  __syncthreads();  // barriers initialised before anyone waits on them
+
+  bool ok = mbar_wait_bounded(bar_in, 0);
+  // rows -> xs as fp32 (channel-major), factors 1/s
+  for (int cp = tid; cp < half && ok; cp += kRotThreads) {
+    float v0[R], v1[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (r < nrows) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xst + (size_t)r * d + 2 * cp));
+        v0[r] = f.x; v1[r] = f.y;
+      } else {
+        v0[r] = 0.f; v1[r] = 0.f;
+      }
+    }
+    st_rows<R>(xs + (size_t)(2 * cp) * R, v0);
+    st_rows<R>(xs + (size_t)(2 * cp + 1) * R, v1);
+    float s0 = 1.f, s1 = 1.f;
+    if (P.scale) {
+      if (scale_bulk) { s0 = fac[2 * cp]; s1 = fac[2 * cp + 1]; }
+      else { s0 = __ldg(P.scale + 2 * cp); s1 = __ldg(P.scale + 2 * cp + 1); }
+    }
+    fac[2 * cp] = 1.0f / s0;
+    fac[2 * cp + 1] = 1.0f / s1;
+  }
+  if (__syncthreads_or(!ok)) {
+    // the rows never arrived: report, let the stage copies in flight land (bounded), leave
+    report_status(status, kStatusTimeout);
+    if (tid == 0)
+      for (int q = 0; q < K && q < ring; ++q) mbar_wait_bounded(s_bar + 8u * q, 0);
+    __syncthreads();
+    return;
+  }
+
+  // K stages.  The pairs of a stage are disjoint, so the loads of a batch of
+  // pairs may all be issued before any of its stores.
+  constexpr int U = R == 4 ? 2 : 4;
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) {
+    const bool arrived = mbar_wait_bounded(s_bar + 8u * (k % ring), (uint32_t)((k / ring) & 1));
+    if (arrived) {
+      const unsigned char* st = tab + (size_t)(k % ring) * stage_bytes;
+      const uint32_t* pk = reinterpret_cast<const uint32_t*>(st);
+      const float* ck = reinterpret_cast<const float*>(st + 2 * d);
+      const float* sk = reinterpret_cast<const float*>(st + 4 * d);
+      for (int t0 = tid; t0 < half; t0 += U * kRotThreads) {
+        int ii[U], jj[U];
+        float c[U], sn[U], a[U][R], b[U][R];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int t = t0 + u * kRotThreads;
+          ii[u] = -1;
+          if (t < half) {
+            const uint32_t pr = pk[t];
+            const int i = pr & 0xFFFF, j = pr >> 16;
+            if (i < d && j < d) { ii[u] = i; jj[u] = j; c[u] = ck[t]; sn[u] = sk[t]; }
+            else report_status(status, kStatusBadIndex);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (ii[u] >= 0) {
+            ld_rows<R>(xs + (size_t)ii[u] * R, a[u]);
+            ld_rows<R>(xs + (size_t)jj[u] * R, b[u]);
+          }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (ii[u] >= 0) {
+            float na[R], nb[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              na[r] = fmaf(c[u], a[u][r], sn[u] * b[u][r]);
+              nb[r] = fmaf(-sn[u], a[u][r], c[u] * b[u][r]);
+            }
+            st_rows<R>(xs + (size_t)ii[u] * R, na);
+            st_rows<R>(xs + (size_t)jj[u] * R, nb);
+          }
+      }
+    }
+    if (__syncthreads_or(!arrived)) {
+      // a stage never arrived: report, let this CTA's copies in flight land
+      // (each wait bounded again), then leave
+      report_status(status, kStatusTimeout);
+      if (tid == 0)
+        for (int q = k; q < K && q < k + ring; ++q)
+          mbar_wait_bounded(s_bar + 8u * (q % ring), (uint32_t)((q / ring) & 1));
+      __syncthreads();
+      return;
+    }
+    if (tid == 0) issue_stage(k + ring);  // refill the slot this stage used
+  }
+
+  // channel scale and store
+  for (int cp = tid; cp < half; cp += kRotThreads) {
+    const int c = 2 * cp;
+    float v0[R], v1[R];
+    ld_rows<R>(xs + (size_t)c * R, v0);
+    ld_rows<R>(xs + (size_t)(c + 1) * R, v1);
+    const float f0 = fac[c], f1 = fac[c + 1];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (r < nrows) {
+        const size_t off = (size_t)(row0 + r) * d + c;
+        if constexpr (F16OUT)
+          *reinterpret_cast<__half2*>(static_cast<__half*>(P.out) + off) = __floats2half2_rn(v0[r] * f0, v1[r] * f1);
+        else
+          *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(P.out) + off) =
+              __floats2bfloat162_rn(v0[r] * f0, v1[r] * f1);
+      }
+    }
+  }
+}
+
+size_t rot_smem(int d, int R, int ring) {
+  return (size_t)d * R * 4 + (size_t)d * R * 2 + (size_t)d * 4 + (size_t)ring * 6 * d;
+}
+
+}  // namespace
+
+bool rot_decode_supported(int d, const void* pairs, const void* c, const void* s) {
+  auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  return (d % 8) == 0 && rot_smem(d, 1, 1) <= kRotSmemBudget && al(pairs) && al(c) && al(s);
+}
+
+cudaError_t plan_rot_batch(const RotProblem* probs, int count, RotBatch* out, int* R_out) {
+  if (count < 1 || count > kMaxBatch) return cudaErrorInvalidValue;
+  int maxM = 0;
+  for (int i = 0; i < count; ++i) maxM = probs[i].M > maxM ? probs[i].M : maxM;
+  int R = maxM >= 4 ? 4 : (maxM >= 2 ? 2 : 1);
+  // the widest problem must still hold its rows, factors and one stage
+  for (int i = 0; i < count; ++i)
+    while (R > 1 && rot_smem(probs[i].d, R, 1) > kRotSmemBudget) R >>= 1;
+  *out = RotBatch{};
+  int ctas = 0;
+  for (int i = 0; i < count; ++i) {
+    RotProblem p = probs[i];
+    int ring = p.K < 1 ? 1 : p.K;
+    if (ring > 8) ring = 8;
+    while (ring > 1 && rot_smem(p.d, R, ring) > kRotSmemBudget) --ring;
+    p.ring = ring;
+    p.cta_begin = ctas;
+    ctas += (p.M + R - 1) / R;
+    out->p[i] = p;
+  }
+  out->count = count;
+  out->total_ctas = ctas;
+  *R_out = R;
+  return cudaSuccess;
+}
+
+cudaError_t launch_rot_batch(const RotBatch& b, int R, bool f16_out, int* status, cudaStream_t stream,
+                             bool pdl_trigger) {
+  size_t smem = 0;
+  for (int i = 0; i < b.count; ++i) {
+    const size_t s = rot_smem(b.p[i].d, R, b.p[i].ring);
+    smem = s > smem ? s : smem;
+  }
+  const int trig = pdl_trigger ? 1 : 0;
+  cudaError_t e;
+#define PARO_ROT_LAUNCH(r, f16)                                                                     \
+  {                                                                                                 \
+    auto k = rot_decode_kernel<r, f16>;                                                             \
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);            \
+    if (e != cudaSuccess) return e;                                                                 \
+    k<<<b.total_ctas, kRotThreads, smem, stream>>>(b, status, trig);                                \
+    return cudaPeekAtLastError();                                                                   \
+  }
+  if (f16_out) {
+    if (R == 4) PARO_ROT_LAUNCH(4, true) else if (R == 2) PARO_ROT_LAUNCH(2, true) else PARO_ROT_LAUNCH(1, true)
+  } else {
+    if (R == 4) PARO_ROT_LAUNCH(4, false) else if (R == 2) PARO_ROT_LAUNCH(2, false) else PARO_ROT_LAUNCH(1, false)
+  }
+#undef PARO_ROT_LAUNCH
+}
+
+}  // namespace paro

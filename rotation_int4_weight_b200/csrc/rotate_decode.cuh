@@ -1,0 +1,37 @@
+// Problem descriptors of the few-token (decode) transform kernel (rotate_decode.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "w4_gemv.cuh"  // kMaxBatch
+
+namespace paro {
+
+struct RotProblem {
+  const uint16_t* x;      // bf16 [M][d]
+  void* out;              // bf16 or fp16 [M][d] (one type per launch)
+  int M, d, K;
+  const uint32_t* pairs;  // [K][d/2], (i | j << 16)
+  const float* cos_t;     // [K][d/2]
+  const float* sin_t;     // [K][d/2]
+  const float* scale;     // [d] or null
+  // filled by plan_rot_batch
+  int ring;               // stages of tables held in shared memory at once
+  int cta_begin;          // first CTA of this problem
+};
+
+struct RotBatch {
+  RotProblem p[kMaxBatch];
+  int count;
+  int total_ctas;
+};
+
+// True when the decode kernel can run this width with these table pointers
+// (d % 8 == 0 and 16-byte aligned tables, since stages are copied in 16-byte pieces).
+bool rot_decode_supported(int d, const void* pairs, const void* cos_t, const void* sin_t);
+cudaError_t plan_rot_batch(const RotProblem* probs, int count, RotBatch* out, int* R_out);
+cudaError_t launch_rot_batch(const RotBatch& b, int R, bool f16_out, int* status, cudaStream_t stream,
+                             bool pdl_trigger);
+
+}  // namespace paro

@@ -137,3 +137,22 @@ def test_product_path_does_not_touch_the_oracle():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in txt.replace("oracle-free", ""), f
                 assert "import synth" not in txt and "from synth" not in txt, f
+
+
+def test_batched_validation_on_host():
+    L = paro.ParoLinear
+    good = dict(d_x=1 << 20, d_y=1 << 22, M=1, d_in=512, d_out=512, K=8, d_pairs=1 << 24, d_cos=1 << 25,
+                d_sin=1 << 26, d_scale=None, d_qweight=1 << 27, d_scales=1 << 28, d_zeros=1 << 29)
+    arr = (L * 2)(L(**good), L(**dict(good, d_out=500, d_y=(1 << 22) + 4096)))
+    ptr = ctypes.cast(arr, ctypes.c_void_p)
+    assert paro.lib.paro_rotate_w4_linear_batched(ptr, 2, 128, ctypes.c_void_p(1 << 30), 1 << 20, None) == UNSUPPORTED
+    assert "layer 1" in paro.lib.paro_last_error().decode()
+    arr = (L * 1)(L(**dict(good, K=-1)))
+    assert paro.lib.paro_rotate_w4_linear_batched(ctypes.cast(arr, ctypes.c_void_p), 1, 128, None, 0, None) == INVALID
+    assert paro.lib.paro_rotate_w4_linear_batched(None, 9, 128, None, 0, None) == INVALID
+    arr9 = (L * 9)(*[L(**dict(good, d_y=(1 << 22) + 4096 * i)) for i in range(9)])
+    assert paro.lib.paro_rotate_w4_linear_batched(ctypes.cast(arr9, ctypes.c_void_p), 9, 128, None, 0, None) == UNSUPPORTED
+    arr = (L * 1)(L(**good))
+    assert paro.lib.paro_rotate_w4_linear_batched(ctypes.cast(arr, ctypes.c_void_p), 1, 128, None, 0, None) == INVALID
+    assert paro.lib.paro_batched_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), 1) == 1024
+    assert paro.lib.paro_rotate_w4_linear_batched(None, 0, 128, None, 0, None) == OK

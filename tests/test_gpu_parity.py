@@ -240,3 +240,51 @@ def test_full_size_decode_layers(cfg):
 def test_full_size_prefill_layer_sampled():
     p = next(config_problems(3, only=["k"]))
     _sampled_check(p, 64, 128)
+
+
+# ---------------------------------------------------------------- batched layer call
+def _batch_case(shapes_m, seed):
+    probs, devs = [], []
+    for i, (d_in, d_out, M) in enumerate(shapes_m):
+        p = linear_problem(seed, i, d_in, d_out, M)
+        tables = dev_tables(p)
+        qw, sc, z = paro.paro_pack_weights(torch.from_numpy(p.W).to(DEV), *tables)
+        x = dev_x(p.x)
+        y = torch.empty(M, d_out, dtype=torch.bfloat16, device=DEV)
+        probs.append(p)
+        devs.append(dict(x=x, tables=tables, qw=qw, sc=sc, z=z, y=y))
+    return probs, devs
+
+
+@pytest.mark.parametrize("shapes_m", [
+    [(1536, 1536, 1), (1536, 256, 1), (1536, 256, 1), (1536, 1536, 1), (1536, 8960, 1), (1536, 8960, 1),
+     (8960, 1536, 1)],
+    [(512, 512, 1), (1024, 272, 3), (4096, 1024, 16), (512, 96, 20), (384, 64, 9)],
+])
+def test_batched_matches_oracle_and_single_calls(shapes_m):
+    probs, devs = _batch_case(shapes_m, 61)
+    layers = [paro.paro_linear(d["x"], *d["tables"], d["qw"], d["sc"], d["z"], d["y"]) for d in devs]
+    paro.paro_rotate_w4_linear_batched(layers)
+    torch.cuda.synchronize()
+    assert paro.paro_get_device_status() == 0
+    rng = np.random.default_rng(0)
+    for p, d in zip(probs, devs):
+        got = host(d["y"])
+        single = host(paro.paro_rotate_w4_linear(d["x"], *d["tables"], d["qw"], d["sc"], d["z"]))
+        cols = np.sort(rng.choice(p.d_out, size=min(256, p.d_out), replace=False))
+        qwn, scn, zn = to_np_pack(d["qw"], d["sc"], d["z"])
+        ref = oracle.linear(oracle.rotate(p.x, p.pairs, p.cos_t, p.sin_t, p.scale),
+                            oracle.dequantize(qwn[cols], scn[cols], zn[cols]))
+        assert_linear_close(got[:, cols], ref)
+        assert_linear_close(got, single)
+
+
+def test_batched_rejects_bad_layer_without_launching():
+    probs, devs = _batch_case([(512, 512, 1), (512, 512, 2)], 62)
+    layers = [paro.paro_linear(d["x"], *d["tables"], d["qw"], d["sc"], d["z"], d["y"]) for d in devs]
+    layers[1].d_out = 520  # not a multiple of 16
+    before = devs[0]["y"].clone()
+    with pytest.raises(paro.ParoError, match="layer 1"):
+        paro.paro_rotate_w4_linear_batched(layers)
+    torch.cuda.synchronize()
+    assert torch.equal(devs[0]["y"], before)  # nothing ran
