@@ -111,7 +111,14 @@ class Linear:
         paro.paro_w4_linear(self.xr, self.qw, self.sc, self.z, out=self.y)
 
     def plain(self, paro):
-        paro.paro_w4_linear(self.x, self.qw0, self.sc0, self.z0, out=self.y)
+        # the same INT4 linear without a transform; with many tokens the fused
+        # call with K = 0 (the transform kernel then only rounds x to fp16, the
+        # input format of the tensor-core kernel), with few the plain call
+        if self.M > 64:
+            paro.paro_rotate_w4_linear(self.x, None, None, None, None, self.qw0, self.sc0, self.z0, out=self.y,
+                                       workspace=self.ws)
+        else:
+            paro.paro_w4_linear(self.x, self.qw0, self.sc0, self.z0, out=self.y)
 
     def rotate(self, paro):
         paro.paro_rotate(self.x, self.pairs, self.cos, self.sin, self.scale, out=self.xr)
@@ -123,7 +130,7 @@ class Linear:
 
 
 # kernels launched per linear of each variant (batched: 2 per call of up to 7 linears)
-LAUNCHES = {"fused": 2, "unfused": 2, "plain": 1, "rotate": 1, "fused_e2e": 2}
+LAUNCHES = {"fused": 2, "unfused": 2, "plain": 1, "rotate": 1, "fused_e2e": 2}  # plain: 2 when M > 64
 BATCH = 7  # linears per batched call (one decoder layer)
 
 

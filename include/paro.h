@@ -184,8 +184,10 @@ PARO_API size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int co
  * caller-owned, undefined between calls).  Results equal count separate calls
  * of paro_rotate_w4_linear.  Every linear is validated before anything is
  * enqueued; the message of paro_last_error() names the failing index.  When no
- * linear has a transform (K == 0 and d_scale == NULL for all), only the INT4
- * linear launch runs, on the bf16 inputs, and d_workspace may be NULL.
+ * linear has a transform (K == 0 and d_scale == NULL for all) and every M is
+ * at most 64, only the INT4-linear launch runs, on the bf16 inputs, and
+ * d_workspace may be NULL; with more tokens the inputs are first rounded to
+ * fp16 into the workspace, as the transform does, for the tensor-core kernel.
  */
 PARO_API paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count, int group_size,
                                                   void* d_workspace, size_t workspace_bytes,

@@ -10,6 +10,7 @@
 #include "paro_internal.cuh"
 #include "w4_gemv.cuh"
 #include "rotate_decode.cuh"
+#include "w4_tc.cuh"
 
 namespace {
 
@@ -99,13 +100,20 @@ paro_status check_weights(const uint32_t* qweight, const uint16_t* scales, const
   return PARO_OK;
 }
 
+// Token count from which the tensor-core (tcgen05) kernel takes over.
+constexpr int kTensorCoreMinM = 128;
+
 // The INT4 linear on x (bf16, or fp16 when x_f16).  With pdl_wait the kernel is
 // launched as a programmatic dependent of the previous kernel in the stream and
 // waits for it before reading x (the weights may be read earlier, so only a
 // previous kernel that does not write them may trigger early).
 cudaError_t launch_linear(const uint16_t* x, bool x_f16, const uint32_t* qweight, const uint16_t* scales,
                           const uint16_t* zeros, uint16_t* y, int M, int d_in, int d_out, cudaStream_t s,
-                          bool pdl_wait) {
+                          bool pdl_wait, int* status) {
+  if (M >= kTensorCoreMinM && status && paro::tc_supported(M, d_in, d_out, x))
+    return paro::launch_w4_tc(x, x_f16, qweight, reinterpret_cast<const __half*>(scales),
+                              reinterpret_cast<const __half*>(zeros), reinterpret_cast<__nv_bfloat16*>(y), M, d_in,
+                              d_out, status, s);
   paro::GemvProblem p = {};
   p.x = x;
   p.qw = qweight;
@@ -255,7 +263,7 @@ paro_status paro_w4_linear(const uint16_t* d_x, const uint32_t* d_qweight, const
       overlap(d_y, yb, d_zeros, (size_t)d_out * (d_in / 128) * 2))
     return fail(PARO_ERR_INVALID_ARG, "y overlaps an input");
   cudaError_t e = launch_linear(d_x, false, d_qweight, d_scales, d_zeros, d_y, M, d_in, d_out,
-                                reinterpret_cast<cudaStream_t>(stream), false);
+                                reinterpret_cast<cudaStream_t>(stream), false, status_ptr());
   return from_cuda(e, "w4 linear launch");
 }
 
@@ -294,7 +302,7 @@ paro_status paro_rotate_w4_linear(const uint16_t* d_x, int K, const uint16_t* d_
                                    true);
   if (e != cudaSuccess) return from_cuda(e, "rotate launch");
   e = launch_linear(static_cast<const uint16_t*>(d_workspace), true, d_qweight, d_scales, d_zeros, d_y, M, d_in,
-                    d_out, s, true);
+                    d_out, s, true, status);
   return from_cuda(e, "w4 linear launch");
 }
 
@@ -364,9 +372,9 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     ++n;
   }
   if (n == 0) return ok();
-  if (any_transform && (!d_workspace || workspace_bytes < need || !aligned(d_workspace, 256)))
+  if ((any_transform || !decode_ok) && (!d_workspace || workspace_bytes < need || !aligned(d_workspace, 256)))
     return fail(PARO_ERR_INVALID_ARG, "workspace must be 256-byte aligned and hold %zu bytes", need);
-  for (int i = 0; i < count && any_transform; ++i) {
+  for (int i = 0; i < count && (any_transform || !decode_ok); ++i) {
     const paro_linear& L = h_layers[i];
     if (L.M == 0) continue;
     if (overlap(d_workspace, need, L.d_x, (size_t)L.M * L.d_in * 2) ||
@@ -375,8 +383,8 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (!any_transform) {
-    // no layer has a transform: the INT4 linear reads the bf16 inputs directly
+  if (!any_transform && decode_ok) {
+    // few tokens and no layer has a transform: the INT4 linear reads the bf16 inputs directly
     for (int i = 0; i < n; ++i) gp[i].x = rp[i].x;
     paro::GemvBatch gb;
     int nt = 1;
@@ -392,11 +400,19 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     e = paro::plan_rot_batch(rp, n, &rb, &R);
     if (e == cudaSuccess) e = paro::launch_rot_batch(rb, R, true, status, s, true);
   } else {
+    // many tokens (or tables the decode kernel cannot take): one transform and one
+    // linear per layer, each linear on the tensor-core kernel when it applies
     e = cudaSuccess;
-    for (int i = 0; i < n && e == cudaSuccess; ++i)
+    for (int i = 0; i < n && e == cudaSuccess; ++i) {
       e = launch_transform(rp[i].x, rp[i].out, true, rp[i].M, rp[i].d, rp[i].K,
                            reinterpret_cast<const uint16_t*>(rp[i].pairs), rp[i].cos_t, rp[i].sin_t, rp[i].scale,
-                           status, s, i == n - 1);
+                           status, s, true);
+      if (e == cudaSuccess)
+        e = launch_linear(gp[i].x, true, gp[i].qw, reinterpret_cast<const uint16_t*>(gp[i].sc),
+                          reinterpret_cast<const uint16_t*>(gp[i].z), reinterpret_cast<uint16_t*>(gp[i].y), gp[i].M,
+                          gp[i].d_in, gp[i].d_out, s, true, status);
+    }
+    return from_cuda(e, "batched launch");
   }
   if (e != cudaSuccess) return from_cuda(e, "batched transform launch");
   paro::GemvBatch gb;

@@ -12,7 +12,8 @@
 // so a pair update moves R values with one vector load/store per channel),
 // applies all K stages there with a barrier between stages, and writes the
 // result once.  HBM sees one read and one write of the rows; the pair and
-// cos/sin tables stream from L2.
+// cos/sin tables stream from L2, each thread fetching its entries of the next
+// stage while it works on the current one.
 #include "paro_internal.cuh"
 
 namespace paro {
@@ -44,9 +45,157 @@ __device__ __forceinline__ void st_vec(float* p, const float (&v)[R]) {
   }
 }
 
+// UP: upper bound on the pairs (and channel pairs) one thread handles per stage.
+template <int R, int MODE, int UP>
+__global__ void __launch_bounds__(512, 2)
+givens_rows_kernel(const void* __restrict__ in, void* __restrict__ out, int M, int d, int K,
+                   const uint32_t* __restrict__ pairs, const float* __restrict__ cos_t,
+                   const float* __restrict__ sin_t, const float* __restrict__ scale, int* status,
+                   int pdl_trigger) {
+  extern __shared__ __align__(16) float xs[];  // [d][R]
+  if (pdl_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  const int row0 = blockIdx.x * R;
+  const int nrows = min(R, M - row0);
+  const int tid = threadIdx.x, nth = blockDim.x;
+  const int half = d >> 1;
+
+  // this thread's pairs of a stage: t = tid + u * nth, u < UP; their table
+  // entries are fetched one stage ahead into registers
+  uint32_t pr[UP];
+  float cs[UP], sn[UP];
+  auto fetch = [&](int k, uint32_t (&p)[UP], float (&c)[UP], float (&s_)[UP]) {
+#pragma unroll
+    for (int u = 0; u < UP; ++u) {
+      const int t = tid + u * nth;
+      if (k < K && t < half) {
+        p[u] = __ldg(pairs + (size_t)k * half + t);
+        c[u] = __ldg(cos_t + (size_t)k * half + t);
+        s_[u] = __ldg(sin_t + (size_t)k * half + t);
+      }
+    }
+  };
+  fetch(0, pr, cs, sn);
+
+  // ---- load: rows -> xs[c][r].  A thread issues the loads of four channel
+  // pairs before their shared stores, so their latencies overlap.
+#pragma unroll
+  for (int u0 = 0; u0 < UP; u0 += 4) {
+    float v0[4][R], v1[4][R];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int cp = tid + (u0 + q) * nth;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        v0[q][r] = 0.f; v1[q][r] = 0.f;
+        if (u0 + q < UP && cp < half && r < nrows) {
+          const size_t off = (size_t)(row0 + r) * d + 2 * cp;
+          if constexpr (MODE == kFoldF32) {
+            const float2 f = *reinterpret_cast<const float2*>(static_cast<const float*>(in) + off);
+            v0[q][r] = f.x; v1[q][r] = f.y;
+          } else {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
+                static_cast<const __nv_bfloat16*>(in) + off));
+            v0[q][r] = f.x; v1[q][r] = f.y;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int cp = tid + (u0 + q) * nth;
+      if (u0 + q < UP && cp < half) {
+        st_vec<R>(xs + (size_t)(2 * cp) * R, v0[q]);
+        st_vec<R>(xs + (size_t)(2 * cp + 1) * R, v1[q]);
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- K stages.  The pairs of a stage are disjoint, so a batch's loads may
+  // all be issued before its stores.
+  constexpr int B = R == 4 ? 2 : 4;
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) {
+    uint32_t npr[UP];
+    float ncs[UP], nsn[UP];
+    fetch(k + 1, npr, ncs, nsn);
+#pragma unroll
+    for (int u0 = 0; u0 < UP; u0 += B) {
+      int ii[B], jj[B];
+      float a[B][R], b[B][R];
+#pragma unroll
+      for (int q = 0; q < B; ++q) {
+        const int u = u0 + q;
+        ii[q] = -1;
+        if (u < UP && tid + u * nth < half) {
+          const int i = pr[u] & 0xFFFF, j = pr[u] >> 16;
+          if (i < d && j < d) { ii[q] = i; jj[q] = j; }
+          else report_status(status, kStatusBadIndex);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < B; ++q)
+        if (ii[q] >= 0) {
+          ld_vec<R>(xs + (size_t)ii[q] * R, a[q]);
+          ld_vec<R>(xs + (size_t)jj[q] * R, b[q]);
+        }
+#pragma unroll
+      for (int q = 0; q < B; ++q)
+        if (ii[q] >= 0) {
+          const float c = cs[u0 + q], s_ = sn[u0 + q];
+          float na[R], nb[R];
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            na[r] = fmaf(c, a[q][r], s_ * b[q][r]);
+            nb[r] = fmaf(-s_, a[q][r], c * b[q][r]);
+          }
+          st_vec<R>(xs + (size_t)ii[q] * R, na);
+          st_vec<R>(xs + (size_t)jj[q] * R, nb);
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < UP; ++u) { pr[u] = npr[u]; cs[u] = ncs[u]; sn[u] = nsn[u]; }
+  }
+
+  // ---- channel scale and store -------------------------------------------------
+#pragma unroll
+  for (int u = 0; u < UP; ++u) {
+    const int cp = tid + u * nth;
+    if (cp >= half) break;
+    const int c = 2 * cp;
+    float f0 = 1.0f, f1 = 1.0f;
+    if (scale) {
+      const float s0 = __ldg(scale + c), s1 = __ldg(scale + c + 1);
+      if constexpr (MODE == kFoldF32) { f0 = s0; f1 = s1; }
+      else { f0 = 1.0f / s0; f1 = 1.0f / s1; }
+    }
+    float v0[R], v1[R];
+    ld_vec<R>(xs + (size_t)c * R, v0);
+    ld_vec<R>(xs + (size_t)(c + 1) * R, v1);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (r < nrows) {
+        const size_t off = (size_t)(row0 + r) * d + c;
+        const float a = v0[r] * f0, b = v1[r] * f1;
+        if constexpr (MODE == kFoldF32) {
+          *reinterpret_cast<float2*>(static_cast<float*>(out) + off) = make_float2(a, b);
+        } else if constexpr (MODE == kActBf16) {
+          *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(out) + off) = __floats2bfloat162_rn(a, b);
+        } else {
+          *reinterpret_cast<__half2*>(static_cast<__half*>(out) + off) = __floats2half2_rn(a, b);
+        }
+      }
+    }
+  }
+}
+
+// Plain variant for wide rows (more than 4 pairs per thread and stage):
+// table entries are read when used.
 template <int R, int MODE>
 __global__ void __launch_bounds__(512)
-givens_rows_kernel(const void* __restrict__ in, void* __restrict__ out, int M, int d, int K,
+givens_rows_simple(const void* __restrict__ in, void* __restrict__ out, int M, int d, int K,
                    const uint32_t* __restrict__ pairs, const float* __restrict__ cos_t,
                    const float* __restrict__ sin_t, const float* __restrict__ scale, int* status,
                    int pdl_trigger) {
@@ -151,36 +300,46 @@ int pick_rows_per_cta(int M, int d) {
   return R;
 }
 
+template <int MODE, int R, int UP>
+cudaError_t launch_rup(const void* in, void* out, int M, int d, int K, const uint32_t* p32, const float* cos_t,
+                       const float* sin_t, const float* scale, int* status, cudaStream_t stream, int trig) {
+  const size_t smem = (size_t)R * d * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(givens_rows_kernel<R, MODE, UP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  givens_rows_kernel<R, MODE, UP><<<(M + R - 1) / R, 512, smem, stream>>>(in, out, M, d, K, p32, cos_t, sin_t, scale,
+                                                                          status, trig);
+  return cudaPeekAtLastError();
+}
+
+template <int MODE, int R>
+cudaError_t launch_r(const void* in, void* out, int M, int d, int K, const uint32_t* p32, const float* cos_t,
+                     const float* sin_t, const float* scale, int* status, cudaStream_t stream, int trig) {
+  const int per = (d / 2 + 511) / 512;  // pairs per thread and stage
+  if (per <= 1) return launch_rup<MODE, R, 1>(in, out, M, d, K, p32, cos_t, sin_t, scale, status, stream, trig);
+  if (per <= 2) return launch_rup<MODE, R, 2>(in, out, M, d, K, p32, cos_t, sin_t, scale, status, stream, trig);
+  if (per <= 4) return launch_rup<MODE, R, 4>(in, out, M, d, K, p32, cos_t, sin_t, scale, status, stream, trig);
+  // wider rows: the register prefetch would spill at two CTAs per SM; read the tables when used
+  const int threads = d >= 2048 ? 512 : 256;
+  const size_t smem = (size_t)R * d * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(givens_rows_simple<R, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  givens_rows_simple<R, MODE><<<(M + R - 1) / R, threads, smem, stream>>>(in, out, M, d, K, p32, cos_t, sin_t,
+                                                                          scale, status, trig);
+  return cudaPeekAtLastError();
+}
+
 template <int MODE>
 cudaError_t launch_givens(const void* in, void* out, int M, int d, int K, const uint16_t* pairs,
                           const float* cos_t, const float* sin_t, const float* scale, int* status,
                           cudaStream_t stream, bool pdl_trigger) {
   const int R = pick_rows_per_cta(M, d);
-  const int threads = d >= 2048 ? 512 : 256;
-  const size_t smem = (size_t)R * d * sizeof(float);
-  const dim3 grid((M + R - 1) / R);
   const uint32_t* p32 = reinterpret_cast<const uint32_t*>(pairs);
   const int trig = pdl_trigger ? 1 : 0;
-  cudaError_t e = cudaSuccess;
-  switch (R) {
-    case 4:
-      e = cudaFuncSetAttribute(givens_rows_kernel<4, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess)
-        givens_rows_kernel<4, MODE><<<grid, threads, smem, stream>>>(in, out, M, d, K, p32, cos_t, sin_t, scale, status, trig);
-      break;
-    case 2:
-      e = cudaFuncSetAttribute(givens_rows_kernel<2, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess)
-        givens_rows_kernel<2, MODE><<<grid, threads, smem, stream>>>(in, out, M, d, K, p32, cos_t, sin_t, scale, status, trig);
-      break;
-    default:
-      e = cudaFuncSetAttribute(givens_rows_kernel<1, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess)
-        givens_rows_kernel<1, MODE><<<grid, threads, smem, stream>>>(in, out, M, d, K, p32, cos_t, sin_t, scale, status, trig);
-      break;
-  }
-  if (e != cudaSuccess) return e;
-  return cudaPeekAtLastError();
+  if (R == 4) return launch_r<MODE, 4>(in, out, M, d, K, p32, cos_t, sin_t, scale, status, stream, trig);
+  if (R == 2) return launch_r<MODE, 2>(in, out, M, d, K, p32, cos_t, sin_t, scale, status, stream, trig);
+  return launch_r<MODE, 1>(in, out, M, d, K, p32, cos_t, sin_t, scale, status, stream, trig);
 }
 
 }  // namespace

@@ -1,0 +1,448 @@
+// Group-wise INT4 weight-only linear for many tokens (prefill) on the 5th-
+// generation tensor cores: y[m][n] = sum_k x[m][k] w^[n][k],
+// w^ = (q - zero) * scale per group of 128 input columns (page "ParoQuant:
+// pairwise rotations that survive deployment", section "From fake
+// quantization to a real TensorRT engine": the group-wise INT4 GEMM operator).
+//
+// One CTA computes a 128-token x 256-output tile, K in steps of 64 through a
+// ring of kStages shared-memory stages:
+//   warp 8, lane 0  TMA: the 128 x 64 fp16 activation tile (128-byte swizzle)
+//                   into stage s, completing on full_a[s]; with bf16
+//                   activations warps 10-17 instead load each token row, round
+//                   it to fp16 and store it in the same swizzled layout (fp16
+//                   operands keep the product error an order of magnitude
+//                   below bf16 ones);
+//   warps 0-7       dequantisation: each thread owns one weight row, loads
+//                   their packed words and scale/zero bits PD steps ahead in a
+//                   register ring, turns every word into
+//                   eight fp16 values (q - zero) * scale in column
+//                   order and stores them in the same 128-byte-swizzled
+//                   K-major layout the tensor core reads; then arrives on
+//                   full_b[s] after a proxy fence;
+//   warp 9, lane 0  MMA: four tcgen05.mma (kind::f16, K = 16 each) per step
+//                   into a 128 x 256 fp32 accumulator in tensor memory, then
+//                   tcgen05.commit to empty[s] (the stage may be refilled once
+//                   the MMAs that read it are done) and, after the last step,
+//                   to acc_full;
+//   warps 0-7       epilogue: tcgen05.ld of their 32 lanes (tokens) and one
+//                   half of the 256 columns, bf16 round, 64-byte stores.
+// Every mbarrier wait is bounded; a wait that gives up sets PARO_ERR_TIMEOUT,
+// stops the pipeline and still releases the tensor memory.
+#include <cuda.h>
+
+#include "paro_internal.cuh"
+#include "w4_tc.cuh"
+
+namespace paro {
+namespace {
+
+constexpr int BM = 256, BN = 128, BK = 64;  // two 128-token MMA halves share each B tile
+constexpr int MH = 128;                       // tokens per MMA (M of one tcgen05.mma)
+constexpr int kStages = 4;
+constexpr int kDqWarps = 8;       // warps 0-7: dequantisation (one weight row per thread), then epilogue
+constexpr int kWarpTma = 8;       // TMA producer, tensor-memory allocation
+constexpr int kWarpMma = 9;       // MMA issuer
+constexpr int kWarpConv = 10;     // warps 10-17: bf16 activations -> fp16 tiles (bf16 input only)
+constexpr int kThreadsTma = 320;
+constexpr int kThreadsConv = 576;
+constexpr int A_BYTES = BM * BK * 2;  // 32 KB
+constexpr int B_BYTES = BN * BK * 2;  // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SMEM_BYTES = kStages * STAGE_BYTES + 1024;  // + alignment slack
+constexpr uint32_t kTmemCols = 256;  // two 128 x 128 fp32 accumulators
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded wait on an mbarrier phase (about a second of SM clock).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_test(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_test(bar, parity))
+    if (clock64() - t0 > (1LL << 31)) return false;
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+// K-major operand in the 128-byte swizzle: rows of 128 bytes (64 fp16), 8-row
+// atoms of 1024 bytes (stride byte offset), start address 1024-aligned per tile.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFF);  // start address
+  d |= (uint64_t)1 << 16;                 // leading byte offset (unused by swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;       // stride byte offset: one 8-row atom
+  d |= (uint64_t)1 << 46;                 // descriptor version (Blackwell)
+  d |= (uint64_t)2 << 61;                 // layout: 128-byte swizzle
+  return d;
+}
+
+__host__ __device__ constexpr uint32_t instr_desc() {
+  // fp32 accumulate, A and B fp16, both K-major, N = BN = 128, M = 128
+  return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(MH >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+               : "memory");
+}
+
+// Eight consecutive 4-bit codes of one word -> eight 16-bit (q - zero) * scale,
+// in column order, as four packed pairs.
+template <bool F16>
+__device__ __forceinline__ void dequant8(uint32_t w, uint32_t zc, uint32_t sc, uint32_t (&out)[4]) {
+  const uint32_t lo = w & 0x0F0F0F0Fu;          // codes 0, 2, 4, 6 in bytes 0..3
+  const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;   // codes 1, 3, 5, 7
+  const uint32_t c0123 = __byte_perm(lo, hi, 0x5140);  // bytes: q0 q1 q2 q3
+  const uint32_t c4567 = __byte_perm(lo, hi, 0x7362);  // bytes: q4 q5 q6 q7
+  constexpr uint32_t kMagic = F16 ? 0x64646464u : 0x43434343u;  // high byte of 1024 (fp16) / 128 (bf16)
+  const uint32_t p01 = __byte_perm(c0123, kMagic, 0x4140);
+  const uint32_t p23 = __byte_perm(c0123, kMagic, 0x4342);
+  const uint32_t p45 = __byte_perm(c4567, kMagic, 0x4140);
+  const uint32_t p67 = __byte_perm(c4567, kMagic, 0x4342);
+  const uint32_t p[4] = {p01, p23, p45, p67};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t d;
+    if constexpr (F16) {
+      asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(p[i]), "r"(zc));
+      asm("mul.rn.f16x2 %0, %1, %2;\n" : "=r"(out[i]) : "r"(d), "r"(sc));
+    } else {
+      asm("sub.rn.bf16x2 %0, %1, %2;\n" : "=r"(d) : "r"(p[i]), "r"(zc));
+      asm("mul.rn.bf16x2 %0, %1, %2;\n" : "=r"(out[i]) : "r"(d), "r"(sc));
+    }
+  }
+}
+
+template <bool XF16>
+__global__ void __launch_bounds__(XF16 ? kThreadsTma : kThreadsConv, 1)
+w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ xraw,
+             const uint32_t* __restrict__ qweight, const __half* __restrict__ scales,
+             const __half* __restrict__ zeros, __nv_bfloat16* __restrict__ y, int M, int d_in, int d_out,
+             int* status) {
+  constexpr bool F16 = true;  // tensor-core operands are fp16 in both variants
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t bars[3 * kStages + 1];
+  __shared__ uint32_t tmem_base_slot;
+  __shared__ int abort_flag;
+
+  // the 128-byte swizzle needs every tile at a 1024-byte aligned shared address
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t b_full_a = smem_u32(&bars[0]);
+  const uint32_t b_full_b = smem_u32(&bars[kStages]);
+  const uint32_t b_empty = smem_u32(&bars[2 * kStages]);
+  const uint32_t b_acc = smem_u32(&bars[3 * kStages]);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  const int nk = d_in / BK;
+  const int G = d_in / kGroup;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(b_full_a + 8 * s, XF16 ? 1 : BM);
+      mbar_init(b_full_b + 8 * s, kDqWarps * 32);
+      mbar_init(b_empty + 8 * s, 1);
+    }
+    mbar_init(b_acc, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == kWarpTma) {  // tensor memory for the accumulator
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_base_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  const uint32_t tmem = tmem_base_slot;
+
+  auto fail = [&]() {
+    report_status(status, kStatusTimeout);
+    atomicExch(&abort_flag, 1);
+  };
+
+  if (warp >= kWarpConv) {
+    // ---------------- bf16 activations -> fp16 tiles (bf16 input only) ---------------
+    if constexpr (!XF16) {
+      const int t = threadIdx.x - kWarpConv * 32;  // row of the 256-token tile
+      const int m = m0 + t;
+      const bool okm = m < M;
+      const uint16_t* xr = xraw + (size_t)(okm ? m : 0) * d_in;
+      constexpr int PX = 2;  // steps of loads in flight
+      uint4 xq[PX][8];
+      auto load_x = [&](int k, uint4 (&v)[8]) {
+        if (k < nk && okm) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) v[c] = __ldg(reinterpret_cast<const uint4*>(xr + k * BK + c * 8));
+        }
+      };
+#pragma unroll
+      for (int j = 0; j < PX - 1; ++j) load_x(j, xq[j]);
+      bool stop = false;
+      for (int kb = 0; kb < nk && !stop; kb += PX) {
+#pragma unroll
+        for (int j = 0; j < PX; ++j) {
+          const int k = kb + j;
+          if (k >= nk) break;
+          load_x(k + PX - 1, xq[(j + PX - 1) % PX]);
+          const int s = k % kStages;
+          if (k >= kStages && !mbar_wait(b_empty + 8 * s, ((k / kStages) - 1) & 1)) fail();
+          if (*(volatile int*)&abort_flag) { stop = true; break; }
+          unsigned char* rowp = smem + s * STAGE_BYTES + t * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 o = make_uint4(0u, 0u, 0u, 0u);
+            if (okm) {
+              const uint32_t in[4] = {xq[j][c].x, xq[j][c].y, xq[j][c].z, xq[j][c].w};
+              uint32_t out[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[e]));
+                const __half2 h = __floats2half2_rn(f.x, f.y);
+                out[e] = *reinterpret_cast<const uint32_t*>(&h);
+              }
+              o = make_uint4(out[0], out[1], out[2], out[3]);
+            }
+            *reinterpret_cast<uint4*>(rowp + ((c ^ (t & 7)) << 4)) = o;
+          }
+          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+          mbar_arrive(b_full_a + 8 * s);
+        }
+      }
+    }
+  } else if (warp == kWarpTma) {
+    // ---------------- TMA producer (fp16 input) ------------------------------------
+    if (XF16 && lane == 0) {
+      for (int k = 0; k < nk; ++k) {
+        const int s = k % kStages;
+        if (k >= kStages && !mbar_wait(b_empty + 8 * s, ((k / kStages) - 1) & 1)) { fail(); break; }
+        if (*(volatile int*)&abort_flag) break;
+        mbar_expect_tx(b_full_a + 8 * s, A_BYTES);
+        tma_load_2d(s_base + s * STAGE_BYTES, &xmap, k * BK, m0, b_full_a + 8 * s);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ---------------- MMA issuer ---------------------------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc();
+      bool ok = true;
+      for (int k = 0; k < nk && ok; ++k) {
+        const int s = k % kStages;
+        const uint32_t par = (k / kStages) & 1;
+        if (!mbar_wait(b_full_a + 8 * s, par) || !mbar_wait(b_full_b + 8 * s, par)) { fail(); ok = false; break; }
+        if (*(volatile int*)&abort_flag) { ok = false; break; }
+        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+        const uint32_t a_addr = s_base + s * STAGE_BYTES, b_addr = a_addr + A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 32);
+#pragma unroll
+          for (int h = 0; h < BM / MH; ++h)  // token half h -> accumulator columns [h * BN, (h + 1) * BN)
+            mma_f16(tmem + h * BN, smem_desc_sw128(a_addr + h * (MH * 128) + kk * 32), bdesc, idesc,
+                    (k > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(b_empty + 8 * s);
+      }
+      mma_commit(b_acc);  // arrives once every MMA issued above has completed
+    }
+  } else {
+    // ---------------- dequantisation (warps 0-3), then epilogue ----------------------
+    const int t = threadIdx.x & (BN - 1);  // row of the tile
+    const int hw = threadIdx.x / BN;        // which half of the row's 64 columns (4 words)
+    const int wpr = d_in >> 3;
+    const int rA = n0 + t;
+    const bool okA = rA < d_out;
+    const uint32_t* qa = qweight + (size_t)(okA ? rA : 0) * wpr + hw * 4;
+    const unsigned short* sA = reinterpret_cast<const unsigned short*>(scales) + (size_t)(okA ? rA : 0) * G;
+    const unsigned short* zA = reinterpret_cast<const unsigned short*>(zeros) + (size_t)(okA ? rA : 0) * G;
+    // register ring: words and raw scale/zero bits of the next PD steps, so that
+    // every load has PD steps of work to land before it is used
+    constexpr int PD = 4;
+    uint4 wq[PD];
+    uint32_t sz[PD][2];
+    auto load_step = [&](int k, uint4& w, uint32_t (&z)[2]) {
+      if (k < nk && okA) {
+        const int grp = (k * BK) / kGroup;
+        w = __ldg(reinterpret_cast<const uint4*>(qa + k * 8));
+        z[0] = __ldg(sA + grp);
+        z[1] = __ldg(zA + grp);
+      }
+    };
+#pragma unroll
+    for (int j = 0; j < PD - 1; ++j) load_step(j, wq[j], sz[j]);
+    bool stop = false;
+    for (int kb = 0; kb < nk && !stop; kb += PD) {
+#pragma unroll
+      for (int j = 0; j < PD; ++j) {
+        const int k = kb + j;
+        if (k >= nk) break;
+        load_step(k + PD - 1, wq[(j + PD - 1) % PD], sz[(j + PD - 1) % PD]);
+        const int s = k % kStages;
+        if (k >= kStages && !mbar_wait(b_empty + 8 * s, ((k / kStages) - 1) & 1)) fail();
+        if (*(volatile int*)&abort_flag) { stop = true; break; }
+        uint32_t zc = 0, sc = 0;
+        if (okA) {
+          const float z = __half2float(__ushort_as_half((unsigned short)sz[j][1]));
+          const __half2 zz = __float2half2_rn(1024.f + z);
+          zc = *reinterpret_cast<const uint32_t*>(&zz);
+          sc = (sz[j][0] & 0xFFFFu) * 0x00010001u;
+        }
+        const uint32_t wv[4] = {wq[j].x, wq[j].y, wq[j].z, wq[j].w};
+        unsigned char* rowp = smem + s * STAGE_BYTES + A_BYTES + t * 128;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {  // 16-byte chunk = 8 columns = one word
+          const int c = hw * 4 + c4;
+          uint32_t o[4] = {0u, 0u, 0u, 0u};
+          if (okA) dequant8<F16>(wv[c4], zc, sc, o);
+          *reinterpret_cast<uint4*>(rowp + ((c ^ (t & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // generic writes -> tensor core reads
+        mbar_arrive(b_full_b + 8 * s);
+      }
+    }
+
+    // ---------------- epilogue -------------------------------------------------------
+    const bool done = mbar_wait(b_acc, 0);
+    if (!done) fail();
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    if (done && !*(volatile int*)&abort_flag) {
+      const int q = warp & 3;                 // TMEM lane quarter this warp may access
+      const int h = warp >> 2;                // token half (accumulator) this warp drains
+      const int m = m0 + h * MH + q * 32 + lane;  // token of this thread's TMEM lane
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * BN);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+              "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+              "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+            : "r"(taddr + c0));
+        asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+        if (m < M && n0 + c0 < d_out) {
+          __nv_bfloat16* dst = y + (size_t)m * d_out + n0 + c0;
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            pk[i] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          // d_out is a multiple of 16: the last 32-column chunk may hold only 16
+          const int nq = (n0 + c0 + 32 <= d_out) ? 4 : 2;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (i < nq)
+              reinterpret_cast<uint4*>(dst)[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+    }
+  }
+
+  // ---------------- teardown --------------------------------------------------------
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  if (XF16 && abort_flag && threadIdx.x == 0) {
+    // let any copies and MMAs still in flight land before the memory goes away
+    for (int s = 0; s < kStages; ++s) {
+      mbar_wait(b_full_a + 8 * s, 0);
+      mbar_wait(b_full_a + 8 * s, 1);
+    }
+    mbar_wait(b_acc, 0);
+  }
+  __syncthreads();
+  if (warp == kWarpTma) {
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool tc_supported(int M, int d_in, int d_out, const void* x) {
+  return M >= 128 && d_in % BK == 0 && d_out % 16 == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 &&
+         ((size_t)d_in * 2) % 16 == 0;
+}
+
+cudaError_t launch_w4_tc(const uint16_t* x, bool x_f16, const uint32_t* qweight, const __half* scales,
+                         const __half* zeros, __nv_bfloat16* y, int M, int d_in, int d_out, int* status,
+                         cudaStream_t stream) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)d_in * 2};
+  const cuuint32_t box[2] = {BK, BM};  // 64 fp16 (128 bytes) x 256 tokens
+  const cuuint32_t elem[2] = {1, 1};
+  CUresult r = enc(&map, x_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<uint16_t*>(x), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  const dim3 grid((d_out + BN - 1) / BN, (M + BM - 1) / BM);
+  cudaError_t e;
+  if (x_f16) {
+    e = cudaFuncSetAttribute(w4_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    w4_tc_kernel<true><<<grid, kThreadsTma, SMEM_BYTES, stream>>>(map, x, qweight, scales, zeros, y, M, d_in, d_out,
+                                                                  status);
+  } else {
+    e = cudaFuncSetAttribute(w4_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    w4_tc_kernel<false><<<grid, kThreadsConv, SMEM_BYTES, stream>>>(map, x, qweight, scales, zeros, y, M, d_in,
+                                                                    d_out, status);
+  }
+  return cudaPeekAtLastError();
+}
+
+}  // namespace paro

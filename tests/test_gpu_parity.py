@@ -288,3 +288,31 @@ def test_batched_rejects_bad_layer_without_launching():
         paro.paro_rotate_w4_linear_batched(layers)
     torch.cuda.synchronize()
     assert torch.equal(devs[0]["y"], before)  # nothing ran
+
+
+# ---------------------------------------------------------------- tensor-core (tcgen05) path, M >= 128
+def _sampled_rows(M, n, seed):
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(M, size=min(n, M), replace=False))
+
+
+@pytest.mark.parametrize("M,d_in,d_out", [(128, 256, 256), (200, 512, 272), (384, 1536, 1024), (129, 4096, 512)])
+def test_w4_linear_tensor_core_bf16(M, d_in, d_out):
+    p = linear_problem(81, M + d_out, d_in, d_out, M)
+    qw, sc, z = _packed(p, rotate=False)
+    got = host(paro.paro_w4_linear(dev_x(p.x), qw, sc, z))
+    rows = _sampled_rows(M, 48, 1)
+    ref = oracle.w4_linear(p.x[rows], *to_np_pack(qw, sc, z))
+    assert_linear_close(got[rows], ref)
+    assert paro.paro_get_device_status() == 0
+
+
+@pytest.mark.parametrize("M,d_in,d_out", [(128, 512, 256), (300, 1536, 272), (640, 4096, 1024)])
+def test_rotate_w4_linear_tensor_core_f16(M, d_in, d_out):
+    p = linear_problem(82, M + d_out, d_in, d_out, M)
+    qw, sc, z = _packed(p)
+    got = host(paro.paro_rotate_w4_linear(dev_x(p.x), *dev_tables(p), qw, sc, z))
+    rows = _sampled_rows(M, 48, 2)
+    ref = oracle.rotate_w4_linear(p.x[rows], p.pairs, p.cos_t, p.sin_t, p.scale, *to_np_pack(qw, sc, z))
+    assert_linear_close(got[rows], ref)
+    assert paro.paro_get_device_status() == 0
