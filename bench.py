@@ -80,13 +80,16 @@ def linear_bytes(d_in, d_out, M, rotate=True, unfused=False):
 class Linear:
     """Device tensors of one linear layer: tables, packed weights (rotated and plain), x, y."""
 
-    def __init__(self, p, dev):
+    def __init__(self, p, dev, plan=True):
         import torch
         import rotation_int4_weight_b200 as paro
         self.d_in, self.d_out, self.M = p.d_in, p.d_out, p.M
-        self.pairs = torch.from_numpy(p.pairs.view(np.int16)).to(dev)
-        self.cos = torch.from_numpy(p.cos_t).to(dev)
-        self.sin = torch.from_numpy(p.sin_t).to(dev)
+        pairs, cos_t, sin_t = p.pairs, p.cos_t, p.sin_t
+        if plan and p.d_in % 64 == 0:  # load-time: conflict-free order of the pairs (same transform)
+            pairs, cos_t, sin_t = paro.paro_plan_pair_order(pairs, cos_t, sin_t)
+        self.pairs = torch.from_numpy(pairs.view(np.int16)).to(dev)
+        self.cos = torch.from_numpy(cos_t).to(dev)
+        self.sin = torch.from_numpy(sin_t).to(dev)
         self.scale = torch.from_numpy(p.scale).to(dev)
         W = device_weights(p, dev)
         ws = torch.empty_like(W)
@@ -170,7 +173,7 @@ class Unit:
         return LAUNCHES[variant] * len(self.lins)
 
 
-def build_layers(config, M, n_layers, rank, dev):
+def build_layers(config, M, n_layers, rank, dev, plan=True):
     name, shapes, M, _, _ = workload(config, M)
     base = 0x5A17 + config + 1000 * rank
     layers = []
@@ -178,7 +181,7 @@ def build_layers(config, M, n_layers, rank, dev):
         lins = []
         for si, (nm, d_in, d_out) in enumerate(shapes):
             p = linear_problem(base, li * 16 + si, d_in, d_out, M, K_STAGES, GROUP, name=nm, host_weights=False)
-            lins.append(Linear(p, dev))
+            lins.append(Linear(p, dev, plan))
         layers.append(lins)
     return layers
 
@@ -399,6 +402,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--variants", default="batched,batched_plain,fused,plain,unfused,rotate")
+    ap.add_argument("--no-plan", action="store_true",
+                    help="use the pair tables as drawn instead of the conflict-free order of paro_plan_pair_order")
     ap.add_argument("--profile", action="store_true",
                     help="run only the listed variants (no end-to-end leg, no CPU baseline): a fixed, short "
                          "launch sequence for ncu; its numbers are not bench values")
@@ -428,7 +433,7 @@ def main():
     hbm, bf16, bf16_sus, peak_kind = peaks()
 
     name, shapes, M, n_layers, stack = workload(args.config, args.M)
-    layers = build_layers(args.config, M, n_layers, rank, dev)
+    layers = build_layers(args.config, M, n_layers, rank, dev, plan=not args.no_plan)
     torch.cuda.synchronize()
     units = [Unit(sum(layers, []), paro)] if stack else [Unit(l, paro) for l in layers]
     step_lins = units[0].lins
@@ -494,7 +499,8 @@ def main():
             "l2": ("inputs larger than L2: each step streams a different layer's weights "
                    f"({len(units)} units, {sum(bytes_of('fused') for _ in units) / 1e9:.2f} GB)") if len(units) > 1
                   else "inputs larger than L2 per step" if step_bytes > 126e6 else "L2-resident (single unit)",
-            "graphs": "each step is one CUDA-graph replay of the per-linear C-ABI calls",
+            "graphs": "each step is one CUDA-graph replay of the step's C-ABI calls",
+            "pair_order": "as drawn" if args.no_plan else "paro_plan_pair_order (conflict-free; same transform)",
         },
         "roofline": {
             "bound": "hbm", "achieved": round(w4_gbs, 1) if w4_gbs else None, "peak": hbm, "unit": "GB/s",

@@ -128,6 +128,25 @@ PARO_API paro_status paro_w4_linear(const uint16_t* d_x, const uint32_t* d_qweig
                            const uint16_t* d_zeros, uint16_t* d_y, int M, int d_in, int d_out,
                            int group_size, paro_stream_t stream);
 
+/*
+ * Host-side, once per layer (no GPU involved): reorders the pairs inside every
+ * stage, flipping some (i, j, cos, sin) into the same rotation (j, i, cos, -sin),
+ * so that every aligned group of 32 consecutive pairs touches 32 different
+ * shared-memory banks with its i channels and 32 with its j channels.  The
+ * output tables describe exactly the same transform (the pairs of a stage are
+ * disjoint, page "ParoQuant: pairwise rotations that survive deployment",
+ * section "A rotation small enough to execute"), so they may replace the input
+ * tables in every call, including paro_pack_weights; the transform kernels then
+ * run without shared-memory bank conflicts on the rows.  Results can differ
+ * from the unplanned tables by fp32 rounding only.
+ * h_pairs [K][d/2][2], h_cos/h_sin [K][d/2]: host input; *_out: host output of
+ * the same shapes, not overlapping the input.  Needs d % 64 == 0
+ * (PARO_ERR_UNSUPPORTED otherwise: keep the original tables); every stage must
+ * be a perfect matching of 0..d-1 (PARO_ERR_INVALID_ARG otherwise).
+ */
+PARO_API paro_status paro_plan_pair_order(const uint16_t* h_pairs, const float* h_cos, const float* h_sin, int K,
+                                          int d, uint16_t* h_pairs_out, float* h_cos_out, float* h_sin_out);
+
 /* Bytes of device workspace paro_rotate_w4_linear needs for M tokens of width d_in. */
 PARO_API size_t paro_workspace_bytes(int M, int d_in);
 

@@ -18,7 +18,7 @@ __all__ = [
     "ParoError", "LIB_PATH", "lib", "paro_weight_layout_version", "paro_workspace_bytes",
     "paro_pack_weights", "paro_rotate", "paro_w4_linear", "paro_rotate_w4_linear",
     "paro_rotate_w4_linear_noalloc", "paro_get_device_status", "EXPORTED", "ParoLinear", "paro_linear",
-    "paro_batched_workspace_bytes", "paro_rotate_w4_linear_batched",
+    "paro_batched_workspace_bytes", "paro_rotate_w4_linear_batched", "paro_plan_pair_order",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libparo.so")
@@ -37,6 +37,7 @@ EXPORTED = {
     "paro_rotate_w4_linear_noalloc": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "paro_batched_workspace_bytes": (_S, [_P, _I]),
     "paro_rotate_w4_linear_batched": (_I, [_P, _I, _I, _P, _S, _P]),
+    "paro_plan_pair_order": (_I, [_P, _P, _P, _I, _I, _P, _P, _P]),
     "paro_get_device_status": (_I, [_P]),
 }
 
@@ -217,6 +218,22 @@ def paro_rotate_w4_linear_batched(layers, *, workspace=None, group_size: int = 1
                                            _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "paro_rotate_w4_linear_batched")
     return workspace
+
+
+def paro_plan_pair_order(pairs, cos_t, sin_t):
+    """Host-side: reorder (and flip) the pairs inside every stage for conflict-free
+    shared-memory access; numpy arrays in ([K, d/2, 2] uint16, [K, d/2] fp32 x2),
+    numpy arrays out describing the same transform."""
+    import numpy as np
+    pairs = np.ascontiguousarray(pairs, dtype=np.uint16)
+    cos_t = np.ascontiguousarray(cos_t, dtype=np.float32)
+    sin_t = np.ascontiguousarray(sin_t, dtype=np.float32)
+    K, half = cos_t.shape
+    po, co, so = np.empty_like(pairs), np.empty_like(cos_t), np.empty_like(sin_t)
+    st = lib.paro_plan_pair_order(pairs.ctypes.data, cos_t.ctypes.data, sin_t.ctypes.data, K, 2 * half,
+                                  po.ctypes.data, co.ctypes.data, so.ctypes.data)
+    _check(st, "paro_plan_pair_order")
+    return po, co, so
 
 
 def paro_get_device_status(stream=None) -> int:

@@ -7,9 +7,9 @@
 // (i, j) with x_i' = c x_i + s x_j, x_j' = -s x_i + c x_j, so every pair of a
 // stage can be updated in parallel without write conflicts.
 //
-// One CTA owns R whole rows.  It stages them in shared memory as fp32 in a
-// channel-major layout xs[channel][R] (the R rows of one channel are adjacent,
-// so a pair update moves R values with one vector load/store per channel),
+// One CTA owns R whole rows.  It stages them in shared memory as fp32, one
+// plane per row (channel c of every row in bank c % 32, so pair tables ordered
+// by paro_plan_pair_order make every access of a warp conflict-free),
 // applies all K stages there with a barrier between stages, and writes the
 // result once.  HBM sees one read and one write of the rows; the pair and
 // cos/sin tables stream from L2, each thread fetching its entries of the next
@@ -21,30 +21,6 @@ namespace {
 
 enum Mode { kActBf16 = 0, kActF16 = 1, kFoldF32 = 2 };
 
-template <int R>
-__device__ __forceinline__ void ld_vec(const float* p, float (&v)[R]) {
-  if constexpr (R == 1) {
-    v[0] = *p;
-  } else if constexpr (R == 2) {
-    float2 t = *reinterpret_cast<const float2*>(p);
-    v[0] = t.x; v[1] = t.y;
-  } else {
-    float4 t = *reinterpret_cast<const float4*>(p);
-    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-  }
-}
-
-template <int R>
-__device__ __forceinline__ void st_vec(float* p, const float (&v)[R]) {
-  if constexpr (R == 1) {
-    *p = v[0];
-  } else if constexpr (R == 2) {
-    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
-  } else {
-    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-  }
-}
-
 // UP: upper bound on the pairs (and channel pairs) one thread handles per stage.
 template <int R, int MODE, int UP>
 __global__ void __launch_bounds__(512, 2)
@@ -52,7 +28,7 @@ givens_rows_kernel(const void* __restrict__ in, void* __restrict__ out, int M, i
                    const uint32_t* __restrict__ pairs, const float* __restrict__ cos_t,
                    const float* __restrict__ sin_t, const float* __restrict__ scale, int* status,
                    int pdl_trigger) {
-  extern __shared__ __align__(16) float xs[];  // [d][R]
+  extern __shared__ __align__(16) float xs[];  // [R][d]
   if (pdl_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int row0 = blockIdx.x * R;
@@ -77,7 +53,7 @@ givens_rows_kernel(const void* __restrict__ in, void* __restrict__ out, int M, i
   };
   fetch(0, pr, cs, sn);
 
-  // ---- load: rows -> xs[c][r].  A thread issues the loads of four channel
+  // ---- load: rows -> xs[r][c].  A thread issues the loads of four channel
   // pairs before their shared stores, so their latencies overlap.
 #pragma unroll
   for (int u0 = 0; u0 < UP; u0 += 4) {
@@ -105,8 +81,9 @@ givens_rows_kernel(const void* __restrict__ in, void* __restrict__ out, int M, i
     for (int q = 0; q < 4; ++q) {
       const int cp = tid + (u0 + q) * nth;
       if (u0 + q < UP && cp < half) {
-        st_vec<R>(xs + (size_t)(2 * cp) * R, v0[q]);
-        st_vec<R>(xs + (size_t)(2 * cp + 1) * R, v1[q]);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          *reinterpret_cast<float2*>(xs + (size_t)r * d + 2 * cp) = make_float2(v0[q][r], v1[q][r]);
       }
     }
   }
@@ -137,8 +114,11 @@ givens_rows_kernel(const void* __restrict__ in, void* __restrict__ out, int M, i
 #pragma unroll
       for (int q = 0; q < B; ++q)
         if (ii[q] >= 0) {
-          ld_vec<R>(xs + (size_t)ii[q] * R, a[q]);
-          ld_vec<R>(xs + (size_t)jj[q] * R, b[q]);
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            a[q][r] = xs[(size_t)r * d + ii[q]];
+            b[q][r] = xs[(size_t)r * d + jj[q]];
+          }
         }
 #pragma unroll
       for (int q = 0; q < B; ++q)
@@ -150,8 +130,11 @@ givens_rows_kernel(const void* __restrict__ in, void* __restrict__ out, int M, i
             na[r] = fmaf(c, a[q][r], s_ * b[q][r]);
             nb[r] = fmaf(-s_, a[q][r], c * b[q][r]);
           }
-          st_vec<R>(xs + (size_t)ii[q] * R, na);
-          st_vec<R>(xs + (size_t)jj[q] * R, nb);
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            xs[(size_t)r * d + ii[q]] = na[r];
+            xs[(size_t)r * d + jj[q]] = nb[r];
+          }
         }
     }
     __syncthreads();
@@ -171,14 +154,12 @@ givens_rows_kernel(const void* __restrict__ in, void* __restrict__ out, int M, i
       if constexpr (MODE == kFoldF32) { f0 = s0; f1 = s1; }
       else { f0 = 1.0f / s0; f1 = 1.0f / s1; }
     }
-    float v0[R], v1[R];
-    ld_vec<R>(xs + (size_t)c * R, v0);
-    ld_vec<R>(xs + (size_t)(c + 1) * R, v1);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       if (r < nrows) {
+        const float2 v = *reinterpret_cast<const float2*>(xs + (size_t)r * d + c);
         const size_t off = (size_t)(row0 + r) * d + c;
-        const float a = v0[r] * f0, b = v1[r] * f1;
+        const float a = v.x * f0, b = v.y * f1;
         if constexpr (MODE == kFoldF32) {
           *reinterpret_cast<float2*>(static_cast<float*>(out) + off) = make_float2(a, b);
         } else if constexpr (MODE == kActBf16) {
@@ -199,14 +180,14 @@ givens_rows_simple(const void* __restrict__ in, void* __restrict__ out, int M, i
                    const uint32_t* __restrict__ pairs, const float* __restrict__ cos_t,
                    const float* __restrict__ sin_t, const float* __restrict__ scale, int* status,
                    int pdl_trigger) {
-  extern __shared__ __align__(16) float xs[];  // [d][R]
+  extern __shared__ __align__(16) float xs[];  // [R][d]
   if (pdl_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int row0 = blockIdx.x * R;
   const int nrows = min(R, M - row0);
   const int tid = threadIdx.x, nth = blockDim.x;
 
-  // ---- load: rows -> xs[c][r] ------------------------------------------------
+  // ---- load: rows -> xs[r][c] ------------------------------------------------
   // Each thread takes two adjacent channels of every row (4-byte bf16 pairs or
   // 8-byte fp32 pairs: a warp reads 128 or 256 contiguous bytes per row) and
   // writes the 2 x R values with vector stores to consecutive channel slots.
@@ -229,8 +210,8 @@ givens_rows_simple(const void* __restrict__ in, void* __restrict__ out, int M, i
         v0[r] = 0.f; v1[r] = 0.f;
       }
     }
-    st_vec<R>(xs + (size_t)(2 * cp) * R, v0);
-    st_vec<R>(xs + (size_t)(2 * cp + 1) * R, v1);
+#pragma unroll
+    for (int r = 0; r < R; ++r) *reinterpret_cast<float2*>(xs + (size_t)r * d + 2 * cp) = make_float2(v0[r], v1[r]);
   }
   __syncthreads();
 
@@ -248,17 +229,12 @@ givens_rows_simple(const void* __restrict__ in, void* __restrict__ out, int M, i
         report_status(status, kStatusBadIndex);
         continue;
       }
-      float a[R], b[R];
-      ld_vec<R>(xs + (size_t)i * R, a);
-      ld_vec<R>(xs + (size_t)j * R, b);
-      float na[R], nb[R];
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        na[r] = fmaf(c, a[r], s * b[r]);
-        nb[r] = fmaf(-s, a[r], c * b[r]);
+        const float a = xs[(size_t)r * d + i], b = xs[(size_t)r * d + j];
+        xs[(size_t)r * d + i] = fmaf(c, a, s * b);
+        xs[(size_t)r * d + j] = fmaf(-s, a, c * b);
       }
-      st_vec<R>(xs + (size_t)i * R, na);
-      st_vec<R>(xs + (size_t)j * R, nb);
     }
     __syncthreads();
   }
@@ -272,14 +248,12 @@ givens_rows_simple(const void* __restrict__ in, void* __restrict__ out, int M, i
       if constexpr (MODE == kFoldF32) { f0 = s0; f1 = s1; }
       else { f0 = 1.0f / s0; f1 = 1.0f / s1; }
     }
-    float v0[R], v1[R];
-    ld_vec<R>(xs + (size_t)c * R, v0);
-    ld_vec<R>(xs + (size_t)(c + 1) * R, v1);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       if (r < nrows) {
+        const float2 v = *reinterpret_cast<const float2*>(xs + (size_t)r * d + c);
         const size_t off = (size_t)(row0 + r) * d + c;
-        const float a = v0[r] * f0, b = v1[r] * f1;
+        const float a = v.x * f0, b = v.y * f1;
         if constexpr (MODE == kFoldF32) {
           *reinterpret_cast<float2*>(static_cast<float*>(out) + off) = make_float2(a, b);
         } else if constexpr (MODE == kActBf16) {

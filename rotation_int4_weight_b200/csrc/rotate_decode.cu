@@ -12,7 +12,8 @@
 // slot as soon as its stage is done.  Bulk copies keep a single SM's stream of
 // table bytes deep without one request per 16 bytes.  Waits are bounded: a
 // stage that never lands is reported as PARO_ERR_TIMEOUT.  The rows themselves live in
-// shared memory as fp32 (channel-major, R rows per channel) after one bulk copy
+// shared memory as fp32 (one plane per row, so channel c sits in bank c % 32
+// for every row) after one bulk copy
 // of the rows and the scales, and each stage is one pass over its disjoint
 // pairs followed by one barrier.
 #include "paro_internal.cuh"
@@ -52,29 +53,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
-template <int R>
-__device__ __forceinline__ void ld_rows(const float* p, float (&v)[R]) {
-  if constexpr (R == 1) {
-    v[0] = *p;
-  } else if constexpr (R == 2) {
-    const float2 t = *reinterpret_cast<const float2*>(p);
-    v[0] = t.x; v[1] = t.y;
-  } else {
-    const float4 t = *reinterpret_cast<const float4*>(p);
-    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-  }
-}
-template <int R>
-__device__ __forceinline__ void st_rows(float* p, const float (&v)[R]) {
-  if constexpr (R == 1) {
-    *p = v[0];
-  } else if constexpr (R == 2) {
-    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
-  } else {
-    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-  }
-}
-
 template <int R, bool F16OUT>
 __global__ void __launch_bounds__(kRotThreads)
 rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_trigger) {
@@ -90,7 +68,8 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
   const int nrows = min(R, P.M - row0);
   const int tid = threadIdx.x;
 
-  // shared memory: xs [d][R] fp32 | x staging [R][d] bf16 | factors [d] fp32 | ring [ring][6d]
+  // shared memory: xs [R][d] fp32 (one plane per row: channel c in bank c % 32) |
+  // x staging [R][d] bf16 | factors [d] fp32 | ring [ring][6d]
   float* xs = reinterpret_cast<float*>(smem);
   __nv_bfloat16* xst = reinterpret_cast<__nv_bfloat16*>(xs + (size_t)d * R);
   float* fac = reinterpret_cast<float*>(xst + (size_t)d * R);
@@ -138,8 +117,8 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
         v0[r] = 0.f; v1[r] = 0.f;
       }
     }
-    st_rows<R>(xs + (size_t)(2 * cp) * R, v0);
-    st_rows<R>(xs + (size_t)(2 * cp + 1) * R, v1);
+#pragma unroll
+    for (int r = 0; r < R; ++r) *reinterpret_cast<float2*>(xs + (size_t)r * d + 2 * cp) = make_float2(v0[r], v1[r]);
     float s0 = 1.f, s1 = 1.f;
     if (P.scale) {
       if (scale_bulk) { s0 = fac[2 * cp]; s1 = fac[2 * cp + 1]; }
@@ -185,8 +164,11 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
 #pragma unroll
         for (int u = 0; u < U; ++u)
           if (ii[u] >= 0) {
-            ld_rows<R>(xs + (size_t)ii[u] * R, a[u]);
-            ld_rows<R>(xs + (size_t)jj[u] * R, b[u]);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              a[u][r] = xs[(size_t)r * d + ii[u]];
+              b[u][r] = xs[(size_t)r * d + jj[u]];
+            }
           }
 #pragma unroll
         for (int u = 0; u < U; ++u)
@@ -197,8 +179,11 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
               na[r] = fmaf(c[u], a[u][r], sn[u] * b[u][r]);
               nb[r] = fmaf(-sn[u], a[u][r], c[u] * b[u][r]);
             }
-            st_rows<R>(xs + (size_t)ii[u] * R, na);
-            st_rows<R>(xs + (size_t)jj[u] * R, nb);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              xs[(size_t)r * d + ii[u]] = na[r];
+              xs[(size_t)r * d + jj[u]] = nb[r];
+            }
           }
       }
     }
@@ -218,19 +203,17 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
   // channel scale and store
   for (int cp = tid; cp < half; cp += kRotThreads) {
     const int c = 2 * cp;
-    float v0[R], v1[R];
-    ld_rows<R>(xs + (size_t)c * R, v0);
-    ld_rows<R>(xs + (size_t)(c + 1) * R, v1);
     const float f0 = fac[c], f1 = fac[c + 1];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       if (r < nrows) {
+        const float2 v = *reinterpret_cast<const float2*>(xs + (size_t)r * d + c);
         const size_t off = (size_t)(row0 + r) * d + c;
         if constexpr (F16OUT)
-          *reinterpret_cast<__half2*>(static_cast<__half*>(P.out) + off) = __floats2half2_rn(v0[r] * f0, v1[r] * f1);
+          *reinterpret_cast<__half2*>(static_cast<__half*>(P.out) + off) = __floats2half2_rn(v.x * f0, v.y * f1);
         else
           *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(P.out) + off) =
-              __floats2bfloat162_rn(v0[r] * f0, v1[r] * f1);
+              __floats2bfloat162_rn(v.x * f0, v.y * f1);
       }
     }
   }

@@ -156,3 +156,45 @@ def test_batched_validation_on_host():
     assert paro.lib.paro_rotate_w4_linear_batched(ctypes.cast(arr, ctypes.c_void_p), 1, 128, None, 0, None) == INVALID
     assert paro.lib.paro_batched_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), 1) == 1024
     assert paro.lib.paro_rotate_w4_linear_batched(None, 0, 128, None, 0, None) == OK
+
+
+# ---------------------------------------------------------------- pair-order planner (host only)
+def _tables(d, K=8, seed=0):
+    import numpy as np
+    from synth import linear_problem
+    p = linear_problem(seed, 1, d, 16, 2, K=K)
+    return p, p.pairs, p.cos_t, p.sin_t
+
+
+@pytest.mark.parametrize("d", [64, 512, 1536, 8960])
+def test_planned_order_is_conflict_free_and_the_same_transform(d):
+    import numpy as np
+    import oracle
+    p, pairs, c, s = _tables(d)
+    po, co, so = paro.paro_plan_pair_order(pairs, c, s)
+    for k in range(pairs.shape[0]):
+        # every aligned group of 32 pairs hits 32 distinct banks with i and with j
+        g = po[k].reshape(-1, 32, 2) % 32
+        assert all(len(set(b[:, 0])) == 32 and len(set(b[:, 1])) == 32 for b in g)
+        # the same set of rotations: each (i, j, c, s) or its flip (j, i, c, -s)
+        orig = {(int(a), int(b)): (float(cc), float(ss)) for (a, b), cc, ss in zip(pairs[k], c[k], s[k])}
+        for (a, b), cc, ss in zip(po[k], co[k], so[k]):
+            if (int(a), int(b)) in orig:
+                assert orig[(int(a), int(b))] == (float(cc), float(ss))
+            else:
+                assert orig[(int(b), int(a))] == (float(cc), -float(ss))
+    # reordering disjoint pairs and flipping them leaves the oracle's result bit-identical
+    assert np.array_equal(oracle.rotate(p.x, pairs, c, s, p.scale), oracle.rotate(p.x, po, co, so, p.scale))
+
+
+def test_planner_rejects_bad_tables():
+    import numpy as np
+    p, pairs, c, s = _tables(512)
+    bad = pairs.copy()
+    bad[2, 5, 0] = bad[2, 6, 1]  # a channel twice in stage 2
+    with pytest.raises(paro.ParoError, match="perfect matching"):
+        paro.paro_plan_pair_order(bad, c, s)
+    p2, pairs2, c2, s2 = _tables(96)  # 96 is not a multiple of 64
+    with pytest.raises(paro.ParoError) as e:
+        paro.paro_plan_pair_order(pairs2, c2, s2)
+    assert e.value.status == UNSUPPORTED

@@ -316,3 +316,18 @@ def test_rotate_w4_linear_tensor_core_f16(M, d_in, d_out):
     ref = oracle.rotate_w4_linear(p.x[rows], p.pairs, p.cos_t, p.sin_t, p.scale, *to_np_pack(qw, sc, z))
     assert_linear_close(got[rows], ref)
     assert paro.paro_get_device_status() == 0
+
+
+# ---------------------------------------------------------------- planned (conflict-free) pair order
+@pytest.mark.parametrize("M,d", [(1, 1536), (4, 4096), (300, 4096), (2, 8960)])
+def test_planned_tables_match_the_oracle(M, d):
+    p = linear_problem(91, M + d, d, 256, M)
+    po, co, so = paro.paro_plan_pair_order(p.pairs, p.cos_t, p.sin_t)
+    tables = (torch.from_numpy(po.view(np.int16)).to(DEV), torch.from_numpy(co).to(DEV),
+              torch.from_numpy(so).to(DEV), torch.from_numpy(p.scale).to(DEV))
+    got = host(paro.paro_rotate(dev_x(p.x), *tables))
+    assert_rotation_close(got, oracle.rotate(p.x, p.pairs, p.cos_t, p.sin_t, p.scale))
+    qw, sc, z = paro.paro_pack_weights(torch.from_numpy(p.W).to(DEV), *tables)
+    y = host(paro.paro_rotate_w4_linear(dev_x(p.x), *tables, qw, sc, z))
+    ref = oracle.rotate_w4_linear(p.x, p.pairs, p.cos_t, p.sin_t, p.scale, *to_np_pack(qw, sc, z))
+    assert_linear_close(y, ref)
