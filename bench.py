@@ -39,6 +39,7 @@ from synth import LAYER_SHAPES, device_weights, linear_problem  # noqa: E402
 METRIC = "rot+W4 linear: decode HBM GB/s (% peak), prefill TFLOP/s, rotation overhead %"
 K_STAGES = 8
 GROUP = 128
+PREFILL_M = 512                          # from this many tokens on the metric is TFLOP/s
 TABLE_BYTES_PER_CH = K_STAGES * 6 + 4   # pairs 4 B + cos/sin 8 B per pair per stage, + fp32 scale
 
 
@@ -173,9 +174,29 @@ class Unit:
         return LAUNCHES[variant] * len(self.lins)
 
 
+def rank_seed(config, rank):
+    """Seed of a rank's inputs: every rank draws its own layers (weak scaling)."""
+    return 0x5A17 + config + 1000 * rank
+
+
+def max_over_ranks(torch, dist, ms, device):
+    """The step time of the whole job: the slowest rank's (all ranks call this)."""
+    if dist is None:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(per_rank_amount, world, ms):
+    """Units all ranks processed per second, each rank doing `per_rank_amount`
+    per step in `ms` milliseconds (the max over ranks)."""
+    return per_rank_amount * world / (ms * 1e-3)
+
+
 def build_layers(config, M, n_layers, rank, dev, plan=True):
     name, shapes, M, _, _ = workload(config, M)
-    base = 0x5A17 + config + 1000 * rank
+    base = rank_seed(config, rank)
     layers = []
     for li in range(n_layers):
         lins = []
@@ -243,11 +264,8 @@ def time_graphs(torch, graphs, steps, warmup, dist=None):
     _replay(graphs, warmup, steps)
     end.record()
     torch.cuda.synchronize()
-    ms = start.elapsed_time(end) / steps
+    ms = max_over_ranks(torch, dist, start.elapsed_time(end) / steps, "cuda")
     if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     return ms
 
@@ -337,12 +355,15 @@ def oracle_problems(config, M):
     return probs, sub_m, M
 
 
-def oracle_run(probs, idx):
+def oracle_run(probs, idx, rows=None):
+    """One oracle linear of the unit (cycling), on its first `rows` output rows
+    (all when None): returns (seconds, algorithmic bytes of the rows run)."""
     import oracle
     p, qw, sc, z = probs[idx % len(probs)]
+    r = p.d_out if rows is None else max(1, min(rows[idx % len(probs)], p.d_out))
     t0 = time.perf_counter()
-    oracle.rotate_w4_linear(p.x, p.pairs, p.cos_t, p.sin_t, p.scale, qw, sc, z)
-    return time.perf_counter() - t0, linear_bytes(p.d_in, p.d_out, p.M)
+    oracle.rotate_w4_linear(p.x, p.pairs, p.cos_t, p.sin_t, p.scale, qw[:r], sc[:r], z[:r])
+    return time.perf_counter() - t0, linear_bytes(p.d_in, r, p.M)
 
 
 def oracle_sample(config, M, seconds=12.0):
@@ -361,32 +382,54 @@ def oracle_sample(config, M, seconds=12.0):
     return tot_b / tot_t / 1e9, _oracle_threads(), sample
 
 
+def reference_rows(probs, steps, warmup, seconds=60.0):
+    """Output rows per oracle step so that `warmup + steps` steps take about
+    `seconds` of CPU time: the cost of a row is measured on one full linear of
+    each shape (untimed), rows are a multiple of 16, at least 16."""
+    per_step = seconds / max(1, steps + warmup)
+    rows = []
+    for i, (p, *_rest) in enumerate(probs):
+        t_full, _ = oracle_run(probs, i)
+        t_row = t_full / p.d_out
+        r = int(per_step / t_row) // 16 * 16
+        rows.append(max(16, min(p.d_out, r)))
+    return rows
+
+
 def run_reference(args):
     """The reference arm: the CPU oracle, timed as it stands on this host's cores.
     Each step runs one linear of the workload's unit (cycling q, k, v, o, gate,
-    up, down), a bounded sample; value = bytes of all timed steps / their time."""
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    up, down) on a bounded sample of its output rows, sized so that the whole
+    run takes about a minute; value = bytes of all timed steps / their time.
+    Under torchrun only rank 0 runs; the other ranks exit without work."""
+    if int(os.environ.get("RANK", "0")) != 0:
         return
     name, shapes, M, _, _ = workload(args.config, args.M)
     probs, sub_m, M = oracle_problems(args.config, args.M)
+    rows = reference_rows(probs, args.steps, args.warmup)
     for i in range(args.warmup):
-        oracle_run(probs, i)
-    tot_t, tot_b = 0.0, 0
+        oracle_run(probs, i, rows)
+    tot_t, tot_b, tot_f = 0.0, 0, 0
     for i in range(args.steps):
-        t, b = oracle_run(probs, args.warmup + i)
+        k = args.warmup + i
+        t, b = oracle_run(probs, k, rows)
+        p = probs[k % len(probs)][0]
         tot_t += t
         tot_b += b
-    value = tot_b / tot_t / 1e9
-    sample = f"{args.steps} steps of one linear each (cycling the {len(probs)} linears), M={sub_m}"
-    out = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
+        tot_f += 2 * p.M * p.d_in * min(rows[k % len(probs)], p.d_out)
+    prefill = M >= PREFILL_M
+    value = tot_f / tot_t / 1e12 if prefill else tot_b / tot_t / 1e9
+    unit = "TFLOP/s" if prefill else "GB/s"
+    sample = (f"{args.steps} steps of one linear each (cycling the {len(probs)} linears), M={sub_m}, "
+              f"first {rows} output rows of each, {tot_t:.1f} s")
+    out = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot_t / args.steps, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": f"{name}: rotate + INT4 linear, M={M}, K={K_STAGES}, group={GROUP} "
                                   f"(fp64 CPU oracle)"},
-           "cpu_baseline": {"kind": "oracle", "value": round(value, 4), "unit": "GB/s", "cores": _oracle_threads(),
+           "cpu_baseline": {"kind": "oracle", "value": round(value, 6), "unit": unit, "cores": _oracle_threads(),
                             "sample": sample},
-           "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+           "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
 
@@ -476,19 +519,19 @@ def main():
 
     ms = results["batched"]
     step_bytes = bytes_of("fused")
-    value = step_bytes * world / (ms * 1e-3) / 1e9
-    e2e_value = (step_bytes + h2d + d2h) * world / (ms_e2e * 1e-3) / 1e9
+    value = whole_job_rate(step_bytes, world, ms) / 1e9
+    e2e_value = whole_job_rate(step_bytes + h2d + d2h, world, ms_e2e) / 1e9
     plain_ms = results.get("plain")
     # dominant kernel: the INT4 linear, timed alone (plain weights, no transform:
     # one launch per batched call when that variant ran, else one per linear)
     w4_ms = results.get("batched_plain", plain_ms)
     w4_gbs = bytes_of("plain") / (w4_ms * 1e-3) / 1e9 if w4_ms else None
     rot_gbs = bytes_of("rotate") / (results["rotate"] * 1e-3) / 1e9 if "rotate" in results else None
-    prefill = M >= 512
+    prefill = M >= PREFILL_M
 
     out = {
         "metric": METRIC,
-        "value": round(value if not prefill else flops_step * world / (ms * 1e-3) / 1e12, 3),
+        "value": round(value if not prefill else whole_job_rate(flops_step, world, ms) / 1e12, 3),
         "unit": "GB/s" if not prefill else "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
