@@ -11,6 +11,7 @@
 #include "w4_gemv.cuh"
 #include "rotate_decode.cuh"
 #include "w4_tc.cuh"
+#include "w4_stream.cuh"
 
 namespace {
 
@@ -306,11 +307,23 @@ paro_status paro_rotate_w4_linear(const uint16_t* d_x, int K, const uint16_t* d_
   return from_cuda(e, "w4 linear launch");
 }
 
+namespace {
+// Bytes of the stream-K kernel's publication flags and partial tiles for these
+// linears (0 when some linear has more tokens than that kernel takes).
+size_t batched_stream_bytes(const paro_linear* h_layers, int count) {
+  int max_m = 0;
+  for (int i = 0; i < count; ++i)
+    if (h_layers[i].M > max_m) max_m = h_layers[i].M;
+  if (max_m < 1 || max_m > paro::kStreamMaxM) return 0;
+  return paro::stream_workspace_bytes(max_m);
+}
+}  // namespace
+
 size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int count) {
   if (!h_layers || count <= 0) return 0;
   size_t b = 0;
   for (int i = 0; i < count; ++i) b += paro_workspace_bytes(h_layers[i].M, h_layers[i].d_in);
-  return b;
+  return b + batched_stream_bytes(h_layers, count);
 }
 
 paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count, int group_size,
@@ -318,7 +331,10 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
   if (count == 0) return ok();
   if (!h_layers || count < 0) return fail(PARO_ERR_INVALID_ARG, "null layer array or negative count");
   if (count > PARO_MAX_BATCH) return fail(PARO_ERR_UNSUPPORTED, "count = %d exceeds %d", count, PARO_MAX_BATCH);
+  // the transformed activations are required; the stream-K kernel's flags and
+  // partial tiles behind them are optional (without them the older kernel runs)
   const size_t need = paro_batched_workspace_bytes(h_layers, count);
+  const size_t xt_need = need - batched_stream_bytes(h_layers, count);
   paro::RotProblem rp[PARO_MAX_BATCH];
   paro::GemvProblem gp[PARO_MAX_BATCH];
   int n = 0;
@@ -372,19 +388,57 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     ++n;
   }
   if (n == 0) return ok();
-  if ((any_transform || !decode_ok) && (!d_workspace || workspace_bytes < need || !aligned(d_workspace, 256)))
+  if ((any_transform || !decode_ok) && (!d_workspace || workspace_bytes < xt_need || !aligned(d_workspace, 256)))
     return fail(PARO_ERR_INVALID_ARG, "workspace must be 256-byte aligned and hold %zu bytes", need);
-  for (int i = 0; i < count && (any_transform || !decode_ok); ++i) {
+  const size_t ws_used = d_workspace ? (workspace_bytes < need ? workspace_bytes : need) : 0;
+  for (int i = 0; i < count && ws_used; ++i) {
     const paro_linear& L = h_layers[i];
     if (L.M == 0) continue;
-    if (overlap(d_workspace, need, L.d_x, (size_t)L.M * L.d_in * 2) ||
-        overlap(d_workspace, need, L.d_y, (size_t)L.M * L.d_out * 2))
+    if (overlap(d_workspace, ws_used, L.d_x, (size_t)L.M * L.d_in * 2) ||
+        overlap(d_workspace, ws_used, L.d_y, (size_t)L.M * L.d_out * 2))
       return fail(PARO_ERR_INVALID_ARG, "layer %d: workspace overlaps x or y", i);
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
+  // the stream-K kernel takes the INT4 linears when every linear has at most 16
+  // tokens and the workspace holds its flags and partial tiles (behind the
+  // transformed activations)
+  const size_t xt_bytes = xt_need;
+  bool use_stream = decode_ok && batched_stream_bytes(h_layers, count) > 0 && d_workspace &&
+                    workspace_bytes >= need && aligned(d_workspace, 256);
+  for (int i = 0; i < n && use_stream; ++i)
+    use_stream = paro::stream_supported(gp[i].M, gp[i].d_in, gp[i].d_out, any_transform ? gp[i].x : rp[i].x,
+                                        gp[i].qw);
+  auto launch_stream = [&](bool x_f16, int* st, bool pdl) -> cudaError_t {
+    const uint16_t* xs[PARO_MAX_BATCH];
+    const uint32_t* qs[PARO_MAX_BATCH];
+    const __half *ss[PARO_MAX_BATCH], *zs[PARO_MAX_BATCH];
+    __nv_bfloat16* ys[PARO_MAX_BATCH];
+    int Ms[PARO_MAX_BATCH], dis[PARO_MAX_BATCH], dos[PARO_MAX_BATCH];
+    for (int i = 0; i < n; ++i) {
+      xs[i] = x_f16 ? gp[i].x : rp[i].x;
+      qs[i] = gp[i].qw;
+      ss[i] = gp[i].sc;
+      zs[i] = gp[i].z;
+      ys[i] = gp[i].y;
+      Ms[i] = gp[i].M;
+      dis[i] = gp[i].d_in;
+      dos[i] = gp[i].d_out;
+    }
+    paro::StreamBatch sb;
+    int nt = 1;
+    cudaError_t err = paro::plan_stream_batch(xs, qs, ss, zs, ys, Ms, dis, dos, n, x_f16,
+                                              static_cast<char*>(d_workspace) + xt_bytes, &sb, &nt);
+    if (err != cudaSuccess) return err;
+    return paro::launch_stream_batch(sb, nt, x_f16, st, s, pdl);
+  };
   if (!any_transform && decode_ok) {
     // few tokens and no layer has a transform: the INT4 linear reads the bf16 inputs directly
+    if (use_stream) {
+      int* status = status_ptr();
+      if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
+      return from_cuda(launch_stream(false, status, false), "batched w4 linear launch");
+    }
     for (int i = 0; i < n; ++i) gp[i].x = rp[i].x;
     paro::GemvBatch gb;
     int nt = 1;
@@ -415,6 +469,7 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     return from_cuda(e, "batched launch");
   }
   if (e != cudaSuccess) return from_cuda(e, "batched transform launch");
+  if (use_stream) return from_cuda(launch_stream(true, status, true), "batched w4 linear launch");
   paro::GemvBatch gb;
   int nt = 1;
   e = paro::plan_gemv_batch(gp, n, true, &gb, &nt);

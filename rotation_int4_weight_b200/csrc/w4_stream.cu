@@ -1,0 +1,770 @@
+// Group-wise INT4 weight-only linear for few tokens (decode), stream-K form:
+//   y[m][n] = sum_k w^[n][k] x[m][k],  w^ = (q - zero) * scale per group of 128 input columns
+// (page "ParoQuant: pairwise rotations that survive deployment", section "From fake
+// quantization to a real TensorRT engine": the group-wise INT4 GEMM operator).
+//
+// With one to sixteen tokens a linear is a stream of packed weights, and a
+// decoder layer's worth of them (tens of MB) lasts only a few microseconds on
+// the whole GPU, so the time goes to filling the memory pipeline and to uneven
+// work.  This kernel therefore splits the weight bytes of all the linears of
+// a launch evenly:
+//   unit   = one 64-row tile x one 128-column group (4 KB of codes), numbered
+//            linear by linear, tile by tile, group by group;
+//   CTA c  = the contiguous units [c U / C, (c + 1) U / C), one CTA per SM;
+//   warp w = a contiguous eighth of its CTA's units.
+// Every warp streams its units through a private ring of D slots: one elected
+// lane issues a TMA tile load of the unit's codes (64 rows x 64 bytes) and two
+// of its activations (the 128 columns of every token, 128-byte swizzle), all
+// completing on the slot's mbarrier; scales and zeros come into registers with
+// the loads of the same unit.  So a warp keeps D units (16 KB of codes) in
+// flight and an SM about 128 KB.
+//
+// Arithmetic, per unit and warp: the codes are the MMA's 16-row side and the
+// tokens its 8-column side (mma.sync m16n8k16, fp32 accumulation).  OR-ing a
+// nibble into the mantissa of 1024 (fp16) or 128 (bf16) gives bias + q exactly;
+// odd nibbles stay in place (x16, or moved one bit: x8) and their activations
+// are pre-divided to match.  One MMA per k-step with constant operands yields,
+// per token, Tb = sum(bias x) in its upper rows and Sx = sum x in its lower
+// rows, shared by the four 16-row tiles of the unit, so
+//   sum (q - z) x = R - Tb - z Sx,  R = the code MMAs' result,
+// and the group scale multiplies that once, all in fp32.
+//
+// Partial sums.  A tile wholly inside one warp's units is written by that warp.
+// A tile split between warps of a CTA is summed in shared memory at the end, in
+// warp order.  A tile split between CTAs goes through the workspace: each CTA
+// writes its partial tile, then counts itself in on the tile's arrival counter;
+// the last to arrive sums the partials in CTA order and writes y.  The counter
+// is a 64-bit word holding (grid id, count): a word left by another launch, or
+// never initialised, is read as count 0, and the last arrival puts the count
+// back to 0, so the workspace needs no clearing between calls.  No thread ever
+// waits for another CTA, and every sum has a fixed order (the result does not
+// depend on timing).
+#include "paro_internal.cuh"
+#include "w4_stream.cuh"
+
+namespace paro {
+namespace {
+
+// Warps per CTA and ring slots per warp, for one (NT = 1) and two (NT = 2)
+// 8-token column tiles; a CTA's registers and shared memory bound both.
+#ifndef PARO_STREAM_W1
+#define PARO_STREAM_W1 12
+#endif
+#ifndef PARO_STREAM_D1
+#define PARO_STREAM_D1 3
+#endif
+#ifndef PARO_STREAM_W2
+#define PARO_STREAM_W2 8
+#endif
+#ifndef PARO_STREAM_D2
+#define PARO_STREAM_D2 3
+#endif
+constexpr int kUnitBytes = kStreamRows * 64;  // 64 rows x 128 codes
+
+template <int NT>
+struct Geo {
+  static constexpr int W = NT == 1 ? PARO_STREAM_W1 : PARO_STREAM_W2;  // warps per CTA
+  static constexpr int D = NT == 1 ? PARO_STREAM_D1 : PARO_STREAM_D2;  // ring slots per warp
+  static constexpr int XB = NT == 1 ? 1024 : 2048;  // bytes per activation box slot (>= 128 M, 1024-aligned)
+  static constexpr int SLOT = kUnitBytes + 2 * XB;
+  static constexpr int PF = 4 * NT * 32 * 4;        // floats of one tile partial (fragment order)
+  static constexpr int SMEM = W * D * SLOT + 1024;
+  static_assert(2 * PF * 4 <= D * SLOT, "a warp's two partial tiles fit in its ring");
+  static_assert(SMEM <= 227 * 1024, "ring exceeds shared memory");
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+// adds expected transaction bytes to the current phase without arriving
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded wait on an mbarrier phase (about a second of SM clock).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_test(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_test(bar, parity))
+    if (clock64() - t0 > (1LL << 31)) return false;
+  return true;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float4 lds128f(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts128f(uint32_t addr, float4 v) {
+  asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
+template <bool F16>
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (F16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+// One packed word -> four operand pairs of exponent-biased codes, exact in the
+// operand type: P[0] = columns (0,4), P[1] = (1,5), P[2] = (2,6), P[3] = (3,7).
+//   fp16: even nibbles give 1024 + q, odd nibbles (left in bits 4..7) 1024 + 16 q;
+//   bf16: even nibbles give 128 + q, odd nibbles (moved to bits 3..6) 128 + 8 q.
+template <bool F16>
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t (&P)[4]) {
+  if constexpr (F16) {
+    const uint32_t w2 = w >> 8;
+    P[0] = (w & 0x000F000Fu) | 0x64006400u;
+    P[1] = (w & 0x00F000F0u) | 0x64006400u;
+    P[2] = (w2 & 0x000F000Fu) | 0x64006400u;
+    P[3] = (w2 & 0x00F000F0u) | 0x64006400u;
+  } else {
+    P[0] = (w & 0x000F000Fu) | 0x43004300u;
+    P[1] = ((w >> 1) & 0x00780078u) | 0x43004300u;
+    P[2] = ((w >> 8) & 0x000F000Fu) | 0x43004300u;
+    P[3] = ((w >> 9) & 0x00780078u) | 0x43004300u;
+  }
+}
+
+template <bool F16>
+__device__ __forceinline__ uint32_t mul2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  if constexpr (F16) asm("mul.rn.f16x2 %0, %1, %2;\n" : "=r"(r) : "r"(a), "r"(b));
+  else asm("mul.rn.bf16x2 %0, %1, %2;\n" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// 8 consecutive activations (4 words) -> pairs (0,4), (1,5), (2,6), (3,7)
+__device__ __forceinline__ void pair_act(const uint4& u, uint32_t (&B)[4]) {
+  B[0] = __byte_perm(u.x, u.z, 0x5410);
+  B[1] = __byte_perm(u.x, u.z, 0x7632);
+  B[2] = __byte_perm(u.y, u.w, 0x5410);
+  B[3] = __byte_perm(u.y, u.w, 0x7632);
+}
+
+// ---- the unit sequence ----------------------------------------------------------
+struct Cur {
+  int pi, tile, grp;
+};
+// The scalar fields of a StreamProblem, copied into shared memory at kernel
+// start: the unit walk indexes problems by a runtime number, and shared memory
+// serves such loads without the dependent round trips of kernel parameters.
+struct Meta {
+  long long unit_begin;
+  const unsigned short* sc;
+  const unsigned short* z;
+  __nv_bfloat16* y;
+  int M, d_out, G, tiles;
+};
+__device__ __forceinline__ void cur_at(const Meta* mp, int count, long long u, Cur& c) {
+  int pi = 0;
+#pragma unroll 1
+  while (pi + 1 < count && u >= mp[pi + 1].unit_begin) ++pi;
+  const long long local = u - mp[pi].unit_begin;
+  c.pi = pi;
+  c.tile = (int)(local / mp[pi].G);
+  c.grp = (int)(local - (long long)c.tile * mp[pi].G);
+}
+__device__ __forceinline__ void cur_next(const Meta* mp, Cur& c) {
+  if (++c.grp == mp[c.pi].G) {
+    c.grp = 0;
+    if (++c.tile == mp[c.pi].tiles) {
+      c.tile = 0;
+      ++c.pi;
+    }
+  }
+}
+// first unit of part i when U units are cut into P contiguous parts
+__device__ __forceinline__ long long part_start(long long i, long long P, long long U) { return i * U / P; }
+// the part holding unit x
+__device__ __forceinline__ long long part_of(long long x, long long P, long long U) { return ((x + 1) * P - 1) / U; }
+
+// lane (g, t) fetches one 16-bit value per row tile: t = 0 scale of row g, t = 1
+// scale of row g + 8, t = 2 zero of row g, t = 3 zero of row g + 8 (rows past
+// d_out read as 0); the four are gathered with shuffles when the unit is computed
+__device__ __forceinline__ void load_sz(const Meta& P, const Cur& c, int g, int t, uint32_t (&r)[4]) {
+  const unsigned short* src = (t & 2) ? P.z : P.sc;
+#pragma unroll
+  for (int rt = 0; rt < 4; ++rt) {
+    const int row = c.tile * kStreamRows + rt * 16 + g + (t & 1) * 8;
+    r[rt] = row < P.d_out ? (uint32_t)__ldg(src + (size_t)row * P.G + c.grp) : 0u;
+  }
+}
+
+template <int NT>
+__device__ __forceinline__ void store_tile(const Meta& P, int tile, int g, int t,
+                                           const float (&v)[4][NT][4]) {
+#pragma unroll
+  for (int rt = 0; rt < 4; ++rt) {
+    const int r0 = tile * kStreamRows + rt * 16 + g;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int m0 = n * 8 + 2 * t;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int row = r0 + (e >> 1) * 8, m = m0 + (e & 1);
+        if (row < P.d_out && m < P.M) P.y[(size_t)m * P.d_out + row] = __float2bfloat16_rn(v[rt][n][e]);
+      }
+    }
+  }
+}
+
+// This launch's grid id: a flag holding it was written by this launch (a word
+// left by an earlier launch, or never written, holds another value).
+__device__ __forceinline__ unsigned long long grid_tag() {
+  unsigned long long gid;
+  asm volatile("mov.u64 %0, %%gridid;\n" : "=l"(gid));
+  return gid;
+}
+__device__ __forceinline__ void st_flag(unsigned long long* f, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(f), "l"(v) : "memory");
+}
+// Bounded wait (about a second of SM clock) for a flag to hold v.
+__device__ bool wait_flag(const unsigned long long* f, unsigned long long v) {
+  const long long t0 = clock64();
+#pragma unroll 1
+  while (true) {
+    unsigned long long x;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];\n" : "=l"(x) : "l"(f) : "memory");
+    if (x == v) return true;
+    if (clock64() - t0 > (1LL << 31)) return false;
+    __nanosleep(64);
+  }
+}
+
+template <bool F16, int NT>
+__global__ void __launch_bounds__(Geo<NT>::W * 32, 1)
+w4_stream_kernel(const __grid_constant__ StreamBatch b, int* status, int pdl_wait) {
+  using Gm = Geo<NT>;
+  constexpr int W = Gm::W, D = Gm::D, SLOT = Gm::SLOT, XB = Gm::XB, PF = Gm::PF;
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t bars[W * D];
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  __shared__ Meta meta[kMaxBatch];
+  if (threadIdx.x < b.count) {
+    const StreamProblem& P = b.p[threadIdx.x];
+    meta[threadIdx.x] = Meta{P.unit_begin, P.sc, P.z, P.y, P.M, P.d_out, P.G, P.tiles};
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&P.qmap)) : "memory");
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&P.xmap)) : "memory");
+  }
+  __syncthreads();
+
+  // ---- this CTA's and this warp's units --------------------------------------------
+  const long long U = b.total_units, C = b.ctas, cta = blockIdx.x;
+  const long long c0 = part_start(cta, C, U), c1 = part_start(cta + 1, C, U), nC = c1 - c0;
+  const long long w0 = c0 + part_start(warp, W, nC), w1 = c0 + part_start(warp + 1, W, nC);
+  const int n = (int)(w1 - w0);
+  const uint32_t ring = sbase + (uint32_t)(warp * D * SLOT);
+  const uint32_t bar0 = smem_u32(&bars[warp * D]);
+
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < D; ++s) mbar_init(bar0 + 8u * s, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncwarp();
+
+  // ---- prologue: codes of the first D units, the scales of the first, then, once
+  // the grid that writes the activations is done, their activations ------------------
+  Cur ic = {0, 0, 0};
+  if (n > 0) cur_at(meta, b.count, w0, ic);
+  Cur cc = ic;  // the unit being computed
+  if (lane == 0) {
+    Cur c = ic;
+#pragma unroll 1
+    for (int s = 0; s < D && s < n; ++s) {
+      mbar_expect_tx(bar0 + 8u * s, (uint32_t)kUnitBytes);
+      tma_load_2d(ring + (uint32_t)(s * SLOT), &b.p[c.pi].qmap, c.grp * 16, c.tile * kStreamRows, bar0 + 8u * s);
+      cur_next(meta, c);
+    }
+  }
+  uint32_t szc[4] = {0u, 0u, 0u, 0u};  // scale and zero bits of the unit being computed
+  if (n > 0) load_sz(meta[cc.pi], cc, g, t, szc);
+  if (pdl_wait) asm volatile("griddepcontrol.wait;\n" ::: "memory");
+#pragma unroll 1
+  for (int s = 0; s < D && s < n; ++s) {
+    if (lane == 0) {
+      const CUtensorMap* xm = &b.p[ic.pi].xmap;
+      const uint32_t sx = ring + (uint32_t)(s * SLOT + kUnitBytes), bar = bar0 + 8u * s;
+      mbar_arrive_expect_tx(bar, (uint32_t)(256 * meta[ic.pi].M));
+      tma_load_2d(sx, xm, ic.grp * 128, 0, bar);
+      tma_load_2d(sx + XB, xm, ic.grp * 128 + 64, 0, bar);
+    }
+    cur_next(meta, ic);
+  }
+
+  // ---- the units ------------------------------------------------------------------
+  float acc[4][NT][4], first[4][NT][4];
+#pragma unroll
+  for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+    for (int m = 0; m < NT; ++m)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) { acc[rt][m][e] = 0.f; first[rt][m][e] = 0.f; }
+
+  int cur_pi = cc.pi, cur_tile = cc.tile;
+  bool ok = true;
+  int done = 0;  // units consumed
+  int slot = 0;
+  uint32_t phase = 0;
+
+  constexpr uint32_t kOddScale = F16 ? 0x2C002C00u : 0x3E003E00u;  // 1/16 or 1/8
+  constexpr uint32_t kBias = F16 ? 0x64006400u : 0x43004300u;      // 1024 / 128
+  constexpr uint32_t kOne = F16 ? 0x3C003C00u : 0x3F803F80u;       // 1
+  constexpr uint32_t kOddUp = F16 ? 0x4C004C00u : 0x41004100u;     // 16 / 8
+  // rows 0-7 of this operand weigh the activations by their codes' bias (Tb),
+  // rows 8-15 by one, undoing the odd columns' pre-division (Sx)
+  const uint32_t aTS[4] = {kBias, kOne, kBias, kOddUp};
+
+#pragma unroll 1
+  for (int i = 0; i < n; ++i) {
+    const Meta& P = meta[cc.pi];
+    if (cc.pi != cur_pi || cc.tile != cur_tile) {
+      // leaving a tile: write it when it lies wholly in this warp's units, else
+      // keep it as this warp's first (split) tile
+      const long long Ub = meta[cur_pi].unit_begin + (long long)cur_tile * meta[cur_pi].G;
+      if (Ub >= w0) {
+        store_tile<NT>(meta[cur_pi], cur_tile, g, t, acc);
+      } else {
+#pragma unroll
+        for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+          for (int m = 0; m < NT; ++m)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) first[rt][m][e] = acc[rt][m][e];
+      }
+#pragma unroll
+      for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+        for (int m = 0; m < NT; ++m)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[rt][m][e] = 0.f;
+      cur_pi = cc.pi;
+      cur_tile = cc.tile;
+    }
+    // scales and zeros of the next unit, one unit ahead of their use
+    Cur nx = cc;
+    uint32_t szn[4] = {0u, 0u, 0u, 0u};
+    if (i + 1 < n) {
+      cur_next(meta, nx);
+      load_sz(meta[nx.pi], nx, g, t, szn);
+    }
+    if (!mbar_wait(bar0 + 8u * slot, phase)) {
+      report_status(status, kStatusTimeout);
+      ok = false;
+      break;
+    }
+    ++done;
+    const uint32_t sw = ring + (uint32_t)slot * SLOT, sx = sw + kUnitBytes;
+    const int mt = P.M;
+
+    // activation fragments: token n*8 + g, columns 32t + 8j .. + 7 of the group,
+    // read from the box of columns 64 (t >> 1) .. + 63 (128-byte swizzle)
+    uint32_t Bf[NT][4][4];
+#pragma unroll
+    for (int m = 0; m < NT; ++m) {
+      const int tok = m * 8 + g;
+      if (tok < mt) {
+        const uint32_t row = sx + (uint32_t)((t >> 1) * XB + tok * 128);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t ch = (uint32_t)(4 * (t & 1) + j) ^ (uint32_t)(tok & 7);
+          pair_act(lds128(row + (ch << 4)), Bf[m][j]);
+          Bf[m][j][1] = mul2<F16>(Bf[m][j][1], kOddScale);
+          Bf[m][j][3] = mul2<F16>(Bf[m][j][3], kOddScale);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) Bf[m][j][e] = 0u;
+      }
+    }
+    // TS[m] = {Tb(token 2t), Tb(2t + 1), Sx(2t), Sx(2t + 1)} of token tile m
+    float TS[NT][4];
+#pragma unroll
+    for (int m = 0; m < NT; ++m) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) TS[m][e] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        mma16816<F16>(TS[m], aTS, Bf[m][j][0], Bf[m][j][1]);
+        mma16816<F16>(TS[m], aTS, Bf[m][j][2], Bf[m][j][3]);
+      }
+    }
+    const int q0 = lane & ~3;
+#pragma unroll
+    for (int rt = 0; rt < 4; ++rt) {
+      // rows rt*16 + g and + 8 of the unit: 64 bytes per row, lane t's 16 bytes
+      const uint32_t wa = sw + (uint32_t)((rt * 16 + g) * 64 + t * 16);
+      const uint4 wg = lds128(wa), wh = lds128(wa + 512u);
+      const float scg = __half2float(__ushort_as_half((unsigned short)__shfl_sync(0xffffffffu, szc[rt], q0)));
+      const float sch = __half2float(__ushort_as_half((unsigned short)__shfl_sync(0xffffffffu, szc[rt], q0 | 1)));
+      const float zg = __half2float(__ushort_as_half((unsigned short)__shfl_sync(0xffffffffu, szc[rt], q0 | 2)));
+      const float zh = __half2float(__ushort_as_half((unsigned short)__shfl_sync(0xffffffffu, szc[rt], q0 | 3)));
+      float R[NT][4];
+#pragma unroll
+      for (int m = 0; m < NT; ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) R[m][e] = 0.f;
+      const uint32_t wgv[4] = {wg.x, wg.y, wg.z, wg.w};
+      const uint32_t whv[4] = {wh.x, wh.y, wh.z, wh.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t Pg[4], Ph[4];
+        unpack_word<F16>(wgv[j], Pg);
+        unpack_word<F16>(whv[j], Ph);
+        const uint32_t a0[4] = {Pg[0], Ph[0], Pg[1], Ph[1]};
+        const uint32_t a1[4] = {Pg[2], Ph[2], Pg[3], Ph[3]};
+#pragma unroll
+        for (int m = 0; m < NT; ++m) {
+          mma16816<F16>(R[m], a0, Bf[m][j][0], Bf[m][j][1]);
+          mma16816<F16>(R[m], a1, Bf[m][j][2], Bf[m][j][3]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < NT; ++m) {
+        acc[rt][m][0] = fmaf(scg, fmaf(-zg, TS[m][2], R[m][0] - TS[m][0]), acc[rt][m][0]);
+        acc[rt][m][1] = fmaf(scg, fmaf(-zg, TS[m][3], R[m][1] - TS[m][1]), acc[rt][m][1]);
+        acc[rt][m][2] = fmaf(sch, fmaf(-zh, TS[m][2], R[m][2] - TS[m][0]), acc[rt][m][2]);
+        acc[rt][m][3] = fmaf(sch, fmaf(-zh, TS[m][3], R[m][3] - TS[m][1]), acc[rt][m][3]);
+      }
+    }
+
+    // refill this slot with unit i + D (the generic-proxy reads above are done
+    // before the asynchronous copy may overwrite the slot)
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    __syncwarp();
+    if (i + D < n) {
+      if (lane == 0) {
+        const StreamProblem& Q = b.p[ic.pi];
+        const uint32_t bar = bar0 + 8u * slot;
+        mbar_arrive_expect_tx(bar, (uint32_t)(kUnitBytes + 256 * meta[ic.pi].M));
+        tma_load_2d(sw, &Q.qmap, ic.grp * 16, ic.tile * kStreamRows, bar);
+        tma_load_2d(sx, &Q.xmap, ic.grp * 128, 0, bar);
+        tma_load_2d(sx + XB, &Q.xmap, ic.grp * 128 + 64, 0, bar);
+      }
+      cur_next(meta, ic);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) szc[e] = szn[e];
+    cc = nx;
+    if (++slot == D) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+  if (!ok) {
+    // let the copies still in flight land (each wait bounded) before leaving the ring
+    for (int j = done; j < n && j < done + D; ++j) mbar_wait(bar0 + 8u * (j % D), (uint32_t)((j / D) & 1));
+  }
+
+  // ---- the last tile, and the partial tiles in shared memory -------------------------
+  // slot 0: the warp's first tile when it began before the warp's units;
+  // slot 1: its last tile when it goes on after them (a tile that does both is slot 0)
+  long long fUb = 0, fUe = 0, lUb = 0, lUe = 0;  // unit ranges of the first and last tile
+  int f_pi = 0, f_tile = 0, l_pi = 0, l_tile = 0;
+  bool f_split = false, l_split = false;
+  if (n > 0) {
+    Cur f;
+    cur_at(meta, b.count, w0, f);
+    f_pi = f.pi;
+    f_tile = f.tile;
+    fUb = meta[f.pi].unit_begin + (long long)f.tile * meta[f.pi].G;
+    fUe = fUb + meta[f.pi].G;
+    l_pi = cur_pi;
+    l_tile = cur_tile;
+    lUb = meta[cur_pi].unit_begin + (long long)cur_tile * meta[cur_pi].G;
+    lUe = lUb + meta[cur_pi].G;
+    f_split = fUb < w0;
+    const bool same = (f_pi == l_pi && f_tile == l_tile);
+    l_split = !same && lUe > w1;
+    if (same) {
+      if (fUb < w0 || fUe > w1) {
+        f_split = true;
+#pragma unroll
+        for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+          for (int m = 0; m < NT; ++m)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) first[rt][m][e] = acc[rt][m][e];
+      } else {
+        store_tile<NT>(meta[l_pi], l_tile, g, t, acc);
+      }
+    } else if (!l_split) {
+      store_tile<NT>(meta[l_pi], l_tile, g, t, acc);
+    }
+  }
+  // the ring is drained: it now holds this warp's partial tiles
+#pragma unroll
+  for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+    for (int m = 0; m < NT; ++m) {
+      const uint32_t off = (uint32_t)(((rt * NT + m) * 32 + lane) * 16);
+      if (f_split) sts128f(ring + off, make_float4(first[rt][m][0], first[rt][m][1], first[rt][m][2], first[rt][m][3]));
+      if (l_split)
+        sts128f(ring + (uint32_t)(PF * 4) + off, make_float4(acc[rt][m][0], acc[rt][m][1], acc[rt][m][2], acc[rt][m][3]));
+    }
+  __syncthreads();
+
+  // ---- combine: the warp holding a split tile's first unit in this CTA sums the
+  // warps' partials in warp order.  A tile that crosses the CTA's bounds then
+  // goes through the workspace: every CTA but the tile's last publishes its
+  // partial and a flag (this launch's grid id) and moves on; the tile's last
+  // CTA waits for the flags of the earlier CTAs, which started no later than
+  // it did, and sums the partials in CTA order.  Publishing comes first (the
+  // warp's last tile), so no warp waits while holding back a partial. ------------
+  const unsigned long long tag = grid_tag();
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const int which = 1 - pass;
+    const bool split = which == 0 ? f_split : l_split;
+    if (!split) continue;
+    const int pi = which == 0 ? f_pi : l_pi, tile = which == 0 ? f_tile : l_tile;
+    const long long Ub = which == 0 ? fUb : lUb, Ue = which == 0 ? fUe : lUe;
+    const long long lo = Ub > c0 ? Ub : c0, hi = Ue < c1 ? Ue : c1;  // the tile's units in this CTA
+    if (c0 + part_of(lo - c0, W, nC) != c0 + warp) continue;     // not the owner
+    const int wlast = (int)part_of(hi - 1 - c0, W, nC);
+    float sum[4][NT][4];
+#pragma unroll
+    for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+      for (int m = 0; m < NT; ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sum[rt][m][e] = 0.f;
+#pragma unroll 1
+    for (int w = warp; w <= wlast; ++w) {
+      const long long ws0 = c0 + part_start(w, W, nC), ws1 = c0 + part_start(w + 1, W, nC);
+      if (ws1 <= ws0) continue;                  // a warp without units
+      const int e = (Ub <= ws0) ? 0 : 1;         // the tile is that warp's first or its last
+      const uint32_t src = sbase + (uint32_t)(w * D * SLOT) + (uint32_t)(e * PF * 4);
+#pragma unroll
+      for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+        for (int m = 0; m < NT; ++m) {
+          const float4 v = lds128f(src + (uint32_t)(((rt * NT + m) * 32 + lane) * 16));
+          sum[rt][m][0] += v.x; sum[rt][m][1] += v.y; sum[rt][m][2] += v.z; sum[rt][m][3] += v.w;
+        }
+    }
+    const Meta& P = meta[pi];
+    if (Ub >= c0 && Ue <= c1) {
+      store_tile<NT>(P, tile, g, t, sum);
+      continue;
+    }
+    if (Ue > c1) {
+      // the tile goes on in a later CTA: publish this CTA's partial, then its flag
+      const int eC = (Ub <= c0) ? 0 : 1;
+      float4* mine = reinterpret_cast<float4*>(b.partials + ((size_t)cta * 2 + eC) * PF);
+#pragma unroll
+      for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+        for (int m = 0; m < NT; ++m)
+          __stcg(mine + (rt * NT + m) * 32 + lane, make_float4(sum[rt][m][0], sum[rt][m][1], sum[rt][m][2], sum[rt][m][3]));
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) st_flag(b.flags + cta * 2 + eC, tag);
+      continue;
+    }
+    // the tile began in an earlier CTA and ends here: add the earlier partials
+    // in CTA order, then this CTA's
+    float tot[4][NT][4];
+#pragma unroll
+    for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+      for (int m = 0; m < NT; ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) tot[rt][m][e] = 0.f;
+    const long long ca = part_of(Ub, C, U);
+#pragma unroll 1
+    for (long long cx = ca; cx < cta; ++cx) {
+      const long long s0 = part_start(cx, C, U);
+      if (part_start(cx + 1, C, U) <= s0) continue;  // a CTA without units
+      const int e = (Ub <= s0) ? 0 : 1;
+      int seen = 1;
+      if (lane == 0) seen = wait_flag(b.flags + cx * 2 + e, tag) ? 1 : 0;
+      seen = __shfl_sync(0xffffffffu, seen, 0);
+      if (!seen) {
+        if (lane == 0) report_status(status, kStatusTimeout);
+        break;
+      }
+      __threadfence();
+      const float4* src = reinterpret_cast<const float4*>(b.partials + ((size_t)cx * 2 + e) * PF);
+#pragma unroll
+      for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+        for (int m = 0; m < NT; ++m) {
+          const float4 v = __ldcg(src + (rt * NT + m) * 32 + lane);
+          tot[rt][m][0] += v.x; tot[rt][m][1] += v.y; tot[rt][m][2] += v.z; tot[rt][m][3] += v.w;
+        }
+    }
+#pragma unroll
+    for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+      for (int m = 0; m < NT; ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) tot[rt][m][e] += sum[rt][m][e];
+    store_tile<NT>(P, tile, g, t, tot);
+  }
+}
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  }
+  return fn;
+}
+
+size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+}  // namespace
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+bool stream_supported(int M, int d_in, int d_out, const void* x, const void* qweight) {
+  return M >= 1 && M <= kStreamMaxM && d_in % kGroup == 0 && d_out >= kStreamRows && d_out % 16 == 0 &&
+         (reinterpret_cast<uintptr_t>(x) & 15) == 0 && (reinterpret_cast<uintptr_t>(qweight) & 15) == 0;
+}
+
+size_t stream_workspace_bytes(int max_m) {
+  const int NT = max_m <= 8 ? 1 : 2;
+  return round256((size_t)device_sm_count() * 2 * 8) + round256((size_t)device_sm_count() * 2 * (4 * NT * 32 * 4) * 4);
+}
+
+cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* qw, const __half* const* sc,
+                              const __half* const* z, __nv_bfloat16* const* y, const int* M, const int* d_in,
+                              const int* d_out, int count, bool x_f16, void* ws, StreamBatch* out, int* nt_out) {
+  if (count < 1 || count > kMaxBatch || !ws) return cudaErrorInvalidValue;
+  EncodeTiled enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  *out = StreamBatch{};
+  int maxM = 0;
+  long long units = 0;
+  for (int i = 0; i < count; ++i) {
+    if (!stream_supported(M[i], d_in[i], d_out[i], x[i], qw[i])) return cudaErrorInvalidValue;
+    maxM = M[i] > maxM ? M[i] : maxM;
+    StreamProblem& p = out->p[i];
+    p.sc = reinterpret_cast<const unsigned short*>(sc[i]);
+    p.z = reinterpret_cast<const unsigned short*>(z[i]);
+    p.y = y[i];
+    p.M = M[i];
+    p.d_in = d_in[i];
+    p.d_out = d_out[i];
+    p.G = d_in[i] / kGroup;
+    p.tiles = (d_out[i] + kStreamRows - 1) / kStreamRows;
+    p.unit_begin = units;
+    units += (long long)p.tiles * p.G;
+    const cuuint32_t unit_strides[2] = {1, 1};
+    {  // codes: uint32 [d_out][d_in / 8], one box = 16 words x 64 rows
+      const cuuint64_t dims[2] = {(cuuint64_t)(d_in[i] / 8), (cuuint64_t)d_out[i]};
+      const cuuint64_t strides[1] = {(cuuint64_t)d_in[i] / 2};
+      const cuuint32_t box[2] = {16, (cuuint32_t)kStreamRows};
+      if (enc(&p.qmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(qw[i]), dims, strides, box,
+              unit_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
+    {  // activations [M][d_in], one box = 64 columns x all M tokens, 128-byte swizzle
+      const cuuint64_t dims[2] = {(cuuint64_t)d_in[i], (cuuint64_t)M[i]};
+      const cuuint64_t strides[1] = {(cuuint64_t)d_in[i] * 2};
+      const cuuint32_t box[2] = {64, (cuuint32_t)M[i]};
+      if (enc(&p.xmap, x_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<uint16_t*>(x[i]), dims, strides, box, unit_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
+  }
+  out->count = count;
+  out->total_units = units;
+  const int W = maxM <= 8 ? Geo<1>::W : Geo<2>::W;
+  const long long want = (units + W - 1) / W;
+  const int sms = device_sm_count();
+  out->ctas = (int)(want < sms ? want : sms);
+  out->flags = static_cast<unsigned long long*>(ws);
+  out->partials = reinterpret_cast<float*>(static_cast<char*>(ws) + round256((size_t)sms * 2 * 8));
+  *nt_out = maxM <= 8 ? 1 : 2;
+  return cudaSuccess;
+}
+
+cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* status, cudaStream_t stream,
+                                bool pdl_wait) {
+  const size_t smem = NT == 1 ? Geo<1>::SMEM : Geo<2>::SMEM;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(b.ctas);
+  cfg.blockDim = dim3((NT == 1 ? Geo<1>::W : Geo<2>::W) * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_wait ? 1 : 0;
+  const int wait = pdl_wait ? 1 : 0;
+  cudaError_t e;
+#define PARO_STREAM_LAUNCH(f16, nt)                                                                       \
+  {                                                                                                       \
+    auto k = w4_stream_kernel<f16, nt>;                                                                   \
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                  \
+    if (e != cudaSuccess) return e;                                                                       \
+    return cudaLaunchKernelEx(&cfg, k, b, status, wait);                                                  \
+  }
+  if (x_f16) {
+    if (NT == 1) PARO_STREAM_LAUNCH(true, 1) else PARO_STREAM_LAUNCH(true, 2)
+  } else {
+    if (NT == 1) PARO_STREAM_LAUNCH(false, 1) else PARO_STREAM_LAUNCH(false, 2)
+  }
+#undef PARO_STREAM_LAUNCH
+}
+
+}  // namespace paro

@@ -1,0 +1,50 @@
+// Problem descriptors of the stream-K INT4 linear for few tokens (w4_stream.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "w4_gemv.cuh"  // kMaxBatch
+
+namespace paro {
+
+constexpr int kStreamMaxM = 16;     // tokens per launch (two 8-token MMA column tiles)
+constexpr int kStreamRows = 64;     // weight rows per tile (four 16-row MMA tiles)
+
+struct StreamProblem {
+  CUtensorMap qmap;            // packed weights, uint32 [d_out][d_in/8], box 16 words x 64 rows
+  CUtensorMap xmap;            // activations [M][d_in] fp16/bf16, box 64 x M, 128-byte swizzle
+  const unsigned short* sc;    // fp16 bits [d_out][d_in/128]
+  const unsigned short* z;     // fp16 bits [d_out][d_in/128]
+  __nv_bfloat16* y;            // [M][d_out]
+  long long unit_begin;        // first unit (one 64-row tile x one 128-column group) of this linear
+  int M, d_in, d_out, G;       // G = d_in / 128
+  int tiles;                   // ceil(d_out / 64)
+};
+
+struct StreamBatch {
+  StreamProblem p[kMaxBatch];
+  long long total_units;
+  unsigned long long* flags;     // two per CTA: its partials' publication flags (workspace)
+  float* partials;               // two tile partials per CTA (workspace)
+  int count;
+  int ctas;
+};
+
+// True when a linear can run on the stream-K kernel (the caller also checks M).
+bool stream_supported(int M, int d_in, int d_out, const void* x, const void* qweight);
+// Workspace bytes of the kernel's publication flags and cross-CTA partial sums.
+size_t stream_workspace_bytes(int max_m);
+// Builds the launch descriptor: tensor maps, unit and tile offsets, the CTA count.
+// x_f16 selects fp16 (else bf16) activations; ws points at stream_workspace_bytes().
+cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* qw, const __half* const* sc,
+                              const __half* const* z, __nv_bfloat16* const* y, const int* M, const int* d_in,
+                              const int* d_out, int count, bool x_f16, void* ws, StreamBatch* out, int* nt_out);
+cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* status, cudaStream_t stream,
+                                bool pdl_wait);
+// Streaming multiprocessors of the current device (cached per device).
+int device_sm_count();
+
+}  // namespace paro

@@ -154,7 +154,12 @@ def test_batched_validation_on_host():
     assert paro.lib.paro_rotate_w4_linear_batched(ctypes.cast(arr9, ctypes.c_void_p), 9, 128, None, 0, None) == UNSUPPORTED
     arr = (L * 1)(L(**good))
     assert paro.lib.paro_rotate_w4_linear_batched(ctypes.cast(arr, ctypes.c_void_p), 1, 128, None, 0, None) == INVALID
-    assert paro.lib.paro_batched_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), 1) == 1024
+    # the transformed activations (1024 bytes), then the stream-K kernel's
+    # counter word (rounded to 256 bytes) and its per-SM partial tiles
+    wb = paro.lib.paro_batched_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), 1)
+    assert wb > 1024 + 256 and wb % 256 == 0
+    too_many = (L * 1)(L(**dict(good, M=17)))
+    assert paro.lib.paro_batched_workspace_bytes(ctypes.cast(too_many, ctypes.c_void_p), 1) == 17 * 1024
     assert paro.lib.paro_rotate_w4_linear_batched(None, 0, 128, None, 0, None) == OK
 
 

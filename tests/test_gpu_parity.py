@@ -331,3 +331,55 @@ def test_planned_tables_match_the_oracle(M, d):
     y = host(paro.paro_rotate_w4_linear(dev_x(p.x), *tables, qw, sc, z))
     ref = oracle.rotate_w4_linear(p.x, p.pairs, p.cos_t, p.sin_t, p.scale, *to_np_pack(qw, sc, z))
     assert_linear_close(y, ref)
+
+
+# ---------------------------------------------------------------- stream-K decode kernel (M <= 16)
+def _stream_case(shapes_m, seed, rotate):
+    probs, devs = [], []
+    for i, (d_in, d_out, M) in enumerate(shapes_m):
+        p = linear_problem(seed, i, d_in, d_out, M)
+        tables = dev_tables(p) if rotate else (None, None, None, None)
+        qw, sc, z = _packed(p, rotate)
+        y = torch.full((M, d_out), float("nan"), dtype=torch.bfloat16, device=DEV)
+        probs.append(p)
+        devs.append(dict(x=dev_x(p.x), tables=tables, qw=qw, sc=sc, z=z, y=y))
+    layers = [paro.paro_linear(d["x"], *d["tables"], d["qw"], d["sc"], d["z"], d["y"]) for d in devs]
+    return probs, devs, layers
+
+
+@pytest.mark.parametrize("rotate", [True, False])
+@pytest.mark.parametrize("shapes_m", [
+    # a Qwen2.5-1.5B-shaped layer at 16 tokens: tiles split between warps and CTAs
+    [(1536, 1536, 16), (1536, 256, 16), (1536, 256, 16), (1536, 1536, 16), (1536, 8960, 16), (1536, 8960, 16),
+     (8960, 1536, 16)],
+    # mixed token counts, ragged output tails (d_out not a multiple of 64)
+    [(512, 80, 1), (1024, 272, 3), (384, 112, 9), (128, 64, 16), (4096, 1040, 8)],
+    # fewer units than warps in the only CTA
+    [(128, 64, 1)],
+    # one row block whose 96 groups are spread over twelve CTAs
+    [(12288, 64, 2)],
+])
+def test_stream_decode_matches_oracle_and_repeats_bit_exactly(shapes_m, rotate):
+    probs, devs, layers = _stream_case(shapes_m, 71, rotate)
+    ws = paro.paro_rotate_w4_linear_batched(layers)
+    torch.cuda.synchronize()
+    assert paro.paro_get_device_status() == 0
+    first = [d["y"].clone() for d in devs]
+    rng = np.random.default_rng(3)
+    for p, d in zip(probs, devs):
+        got = host(d["y"])
+        assert np.isfinite(got).all(), p.name
+        cols = np.sort(rng.choice(p.d_out, size=min(320, p.d_out), replace=False))
+        qwn, scn, zn = to_np_pack(d["qw"], d["sc"], d["z"])
+        xt = oracle.rotate(p.x, p.pairs, p.cos_t, p.sin_t, p.scale) if rotate else p.x
+        ref = oracle.linear(xt, oracle.dequantize(qwn[cols], scn[cols], zn[cols]))
+        assert_linear_close(got[:, cols], ref)
+    # the arrival counters left by the first call are reused as they are: the
+    # second call must give the same bits (fixed summation order)
+    for d in devs:
+        d["y"].fill_(float("nan"))
+    paro.paro_rotate_w4_linear_batched(layers, workspace=ws)
+    torch.cuda.synchronize()
+    assert paro.paro_get_device_status() == 0
+    for f, d in zip(first, devs):
+        assert torch.equal(f.view(torch.int16), d["y"].view(torch.int16))
