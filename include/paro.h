@@ -191,10 +191,10 @@ typedef struct {
 /*
  * Workspace bytes paro_rotate_w4_linear_batched uses for these linears: the
  * transformed activations of every linear (paro_workspace_bytes(M, d_in)
- * each, in order), then, when every M is at most 16, the arrival counters
- * and partial sums of the stream-K INT4 linear (8 bytes per 64-row tile of
- * all the linears, plus 2 partial tiles per SM).  The second part is
- * optional: given only the first, the call runs the older per-block kernel.
+ * each, in order), then, when every M is at most 16, the publication flags
+ * and partial sums of the stream-K INT4 linear (2 flags and 2 partial
+ * 64-row tiles per SM).  The second part is optional: given only the first,
+ * the call runs the older per-block kernel.
  */
 PARO_API size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int count);
 
@@ -214,9 +214,10 @@ PARO_API size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int co
  * at most 64, only the INT4-linear launch runs, on the bf16 inputs, and
  * d_workspace may be NULL; with more tokens the inputs are first rounded to
  * fp16 into the workspace, as the transform does, for the tensor-core kernel.
- * The stream-K kernel's arrival counters need no clearing: a word left by
- * another launch, or never written, counts as zero.  Two calls that may run
- * at the same time need two workspaces.
+ * The stream-K kernel's publication flags need no clearing: a flag holds the
+ * id of the launch that wrote it, so one left by another launch, or never
+ * written, is never taken for this launch's.  Two calls that may run at the
+ * same time need two workspaces.
  */
 PARO_API paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count, int group_size,
                                                   void* d_workspace, size_t workspace_bytes,

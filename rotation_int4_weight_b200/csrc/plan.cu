@@ -18,6 +18,13 @@
 // pairs and the j-side of d/64 pairs.  The resulting bipartite multigraph
 // (i-residue -> j-residue) is d/64-regular and splits into d/64 perfect
 // matchings (Hall / Konig); each matching is one group of 32 pairs.
+//
+// Kernels that keep several rows of a channel side by side (a float2 or float4
+// per channel) access shared memory in phases of 16 or 8 lanes, so each group
+// of 32 is then ordered so that every aligned 16 has distinct i % 16 and
+// j % 16, and every aligned 8 distinct i % 8 and j % 8: n pairs with distinct
+// residues mod n hold every residue mod n/2 twice on each side, a 2-regular
+// bipartite multigraph, which splits into two perfect matchings.
 #include <cstring>
 #include <functional>
 #include <vector>
@@ -92,6 +99,45 @@ bool perfect_matching(const std::vector<Edge>& E, const std::vector<std::vector<
   return true;
 }
 
+// Orders the 2n pairs of `grp` (oriented i -> j, distinct i % 2n and j % 2n)
+// into two halves of n with distinct residues mod n, recursively down to 8.
+void split_phases(std::vector<std::pair<int, int>>& grp) {
+  const int n2 = (int)grp.size(), n = n2 / 2;
+  if (n < 8) return;
+  std::vector<int> left_of_right(n, -1), edge_of_left(n, -1);
+  std::vector<std::vector<int>> out(n);
+  for (int e = 0; e < n2; ++e) out[grp[e].first % n].push_back(e);
+  for (int l = 0; l < n; ++l) {
+    std::vector<bool> seen(n, false);
+    std::function<bool(int)> try_left = [&](int x) -> bool {
+      for (int e : out[x]) {
+        const int r = grp[e].second % n;
+        if (seen[r]) continue;
+        seen[r] = true;
+        if (left_of_right[r] < 0 || try_left(left_of_right[r])) {
+          left_of_right[r] = x;
+          edge_of_left[x] = e;
+          return true;
+        }
+      }
+      return false;
+    };
+    try_left(l);  // a 2-regular bipartite multigraph always has a perfect matching
+  }
+  std::vector<bool> first(n2, false);
+  for (int l = 0; l < n; ++l)
+    if (edge_of_left[l] >= 0) first[edge_of_left[l]] = true;
+  std::vector<std::pair<int, int>> a, b;
+  for (int e = 0; e < n2; ++e) (first[e] ? a : b).push_back(grp[e]);
+  if ((int)a.size() != n) return;  // cannot happen; keep the mod-2n order
+  split_phases(a);
+  split_phases(b);
+  for (int e = 0; e < n; ++e) {
+    grp[e] = a[e];
+    grp[n + e] = b[e];
+  }
+}
+
 }  // namespace
 
 extern "C" paro_status paro_plan_pair_order(const uint16_t* h_pairs, const float* h_cos, const float* h_sin, int K,
@@ -122,8 +168,29 @@ extern "C" paro_status paro_plan_pair_order(const uint16_t* h_pairs, const float
       std::vector<int> m;
       if (!perfect_matching(E, out_edges, m))
         return paro::record_error(PARO_ERR_CUDA, "internal: stage %d has no perfect matching left", k);
+      // the group's pairs, oriented (i, j)
+      std::vector<std::pair<int, int>> grp(kBanks);
+      std::vector<int> edge_at(kBanks);
       for (int l = 0; l < kBanks; ++l) {
-        Edge& e = E[m[l]];
+        const Edge& e = E[m[l]];
+        const int t = e.pair;
+        const int i = e.flip ? P[2 * t + 1] : P[2 * t], j = e.flip ? P[2 * t] : P[2 * t + 1];
+        grp[l] = {i, j};
+      }
+      split_phases(grp);
+      // map each ordered (i, j) back to its edge: i determines the edge within the group
+      for (int l = 0; l < kBanks; ++l) {
+        int found = -1;
+        for (int q = 0; q < kBanks; ++q) {
+          const Edge& e = E[m[q]];
+          const int t = e.pair;
+          const int i = e.flip ? P[2 * t + 1] : P[2 * t];
+          if (i == grp[l].first) { found = m[q]; break; }
+        }
+        edge_at[l] = found;
+      }
+      for (int l = 0; l < kBanks; ++l) {
+        Edge& e = E[edge_at[l]];
         e.used = true;
         const int t = e.pair, o = g * kBanks + l;
         const uint16_t i = P[2 * t], j = P[2 * t + 1];

@@ -178,9 +178,12 @@ def test_planned_order_is_conflict_free_and_the_same_transform(d):
     p, pairs, c, s = _tables(d)
     po, co, so = paro.paro_plan_pair_order(pairs, c, s)
     for k in range(pairs.shape[0]):
-        # every aligned group of 32 pairs hits 32 distinct banks with i and with j
-        g = po[k].reshape(-1, 32, 2) % 32
-        assert all(len(set(b[:, 0])) == 32 and len(set(b[:, 1])) == 32 for b in g)
+        # every aligned group of 32 pairs hits 32 distinct banks with i and with j,
+        # and so does every aligned 16 (8) mod 16 (8): the phases of 8- and
+        # 16-byte shared-memory accesses of channel-major rows
+        for n in (32, 16, 8):
+            g = po[k].reshape(-1, n, 2) % n
+            assert all(len(set(b[:, 0])) == n and len(set(b[:, 1])) == n for b in g), n
         # the same set of rotations: each (i, j, c, s) or its flip (j, i, c, -s)
         orig = {(int(a), int(b)): (float(cc), float(ss)) for (a, b), cc, ss in zip(pairs[k], c[k], s[k])}
         for (a, b), cc, ss in zip(po[k], co[k], so[k]):
