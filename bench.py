@@ -142,7 +142,26 @@ class Unit:
     """The linears of one step; runs them per linear or as batched calls."""
 
     def __init__(self, lins, paro):
+        import torch
         self.lins = lins
+        # the step's inputs and outputs live in one contiguous device buffer each
+        # (every linear's x and y are views into them), so the end-to-end variant
+        # moves them with one host->device and one device->host copy per step
+        dev = lins[0].x.device
+        self.x_all = torch.empty(sum(l.x.numel() for l in lins), dtype=torch.bfloat16, device=dev)
+        self.y_all = torch.empty(sum(l.y.numel() for l in lins), dtype=torch.bfloat16, device=dev)
+        ox = oy = 0
+        for l in lins:
+            nx, ny = l.x.numel(), l.y.numel()
+            vx = self.x_all[ox:ox + nx].view(l.x.shape)
+            vx.copy_(l.x)
+            l.x = vx
+            l.y = self.y_all[oy:oy + ny].view(l.y.shape)
+            ox += nx
+            oy += ny
+        self.x_host = torch.empty(self.x_all.shape, dtype=torch.bfloat16, pin_memory=True)
+        self.x_host.copy_(self.x_all)
+        self.y_host = torch.empty(self.y_all.shape, dtype=torch.bfloat16, pin_memory=True)
         self.calls = []
         for i in range(0, len(lins), BATCH):
             grp = lins[i:i + BATCH]
@@ -154,14 +173,12 @@ class Unit:
 
     def run(self, paro, variant):
         if variant in ("batched", "batched_e2e", "batched_plain"):
+            if variant == "batched_e2e":
+                self.x_all.copy_(self.x_host, non_blocking=True)
             for grp, descs, plain, ws in self.calls:
-                if variant == "batched_e2e":
-                    for l in grp:
-                        l.x.copy_(l.x_host, non_blocking=True)
                 paro.paro_rotate_w4_linear_batched(plain if variant == "batched_plain" else descs, workspace=ws)
-                if variant == "batched_e2e":
-                    for l in grp:
-                        l.y_host.copy_(l.y, non_blocking=True)
+            if variant == "batched_e2e":
+                self.y_host.copy_(self.y_all, non_blocking=True)
         else:
             for lin in self.lins:
                 getattr(lin, variant)(paro)
@@ -514,8 +531,8 @@ def main():
     graphs = capture(torch, paro, units, "batched_e2e")
     ms_e2e = time_graphs(torch, graphs, args.steps, args.warmup, dist)
     del graphs
-    h2d = sum(l.x.numel() * 2 for l in step_lins)
-    d2h = sum(l.y.numel() * 2 for l in step_lins)
+    h2d = units[0].x_all.numel() * 2
+    d2h = units[0].y_all.numel() * 2
 
     ms = results["batched"]
     step_bytes = bytes_of("fused")
@@ -548,8 +565,9 @@ def main():
         "roofline": {
             "bound": "hbm", "achieved": round(w4_gbs, 1) if w4_gbs else None, "peak": hbm, "unit": "GB/s",
             "frac": round(w4_gbs / hbm, 4) if w4_gbs else None, "traffic": None,
-            "kernel": "w4_gemv_kernel (INT4 linear; one launch per batched call of a step's linears), "
-                      "algorithmic bytes / device time",
+            "kernel": ("w4_stream_kernel" if M <= 16 else "w4_gemv_kernel")
+                      + " (INT4 linear; one launch per batched call of a step's linears, timed alone "
+                        "with plain weights), algorithmic bytes / device time",
             "peak_kind": f"{peak_kind} HBM copy bandwidth",
         },
         "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -7,15 +7,13 @@
 // With one or a few token rows the work per stage is tiny and the time goes
 // into fetching the stage tables (12 bytes per pair and stage), so the tables
 // are requested up front: one thread of every CTA issues bulk (TMA) copies of
-// as many whole stages (pairs, cos, sin) as fit in shared memory before the
-// rows are touched, each stage completing on its own mbarrier, and refills a
-// slot as soon as its stage is done.  Bulk copies keep a single SM's stream of
-// table bytes deep without one request per 16 bytes.  Waits are bounded: a
-// stage that never lands is reported as PARO_ERR_TIMEOUT.  The rows themselves live in
-// shared memory as fp32 (one plane per row, so channel c sits in bank c % 32
-// for every row) after one bulk copy
-// of the rows and the scales, and each stage is one pass over its disjoint
-// pairs followed by one barrier.
+// as many whole stages (pairs, cos, sin) as fit in shared memory, each stage
+// completing on its own mbarrier, and a bulk L2 prefetch of all later stages,
+// so that the refill of a slot, issued as soon as its stage is done, waits for
+// L2 rather than HBM.  Waits are bounded: a stage that never lands is reported
+// as PARO_ERR_TIMEOUT.  The rows live in shared memory as fp32 (one plane per
+// row, so channel c sits in bank c % 32 for every row), and each stage is one
+// pass over its disjoint pairs followed by one barrier.
 #include "paro_internal.cuh"
 #include "rotate_decode.cuh"
 
@@ -48,6 +46,9 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     if (clock64() - t0 > (1LL << 31)) return false;
   return true;
 }
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, size_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"((uint32_t)bytes) : "memory");
+}
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
                ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
@@ -69,16 +70,12 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
   const int tid = threadIdx.x;
 
   // shared memory: xs [R][d] fp32 (one plane per row: channel c in bank c % 32) |
-  // x staging [R][d] bf16 | factors [d] fp32 | ring [ring][6d]
+  // ring [ring][6d] of stage tables
   float* xs = reinterpret_cast<float*>(smem);
-  __nv_bfloat16* xst = reinterpret_cast<__nv_bfloat16*>(xs + (size_t)d * R);
-  float* fac = reinterpret_cast<float*>(xst + (size_t)d * R);
-  unsigned char* tab = reinterpret_cast<unsigned char*>(fac + d);
+  unsigned char* tab = reinterpret_cast<unsigned char*>(xs + (size_t)d * R);
   const size_t stage_bytes = (size_t)6 * d;  // pairs | cos | sin
   const uint32_t s_tab = static_cast<uint32_t>(__cvta_generic_to_shared(tab));
   const uint32_t s_bar = static_cast<uint32_t>(__cvta_generic_to_shared(bars));
-  const uint32_t bar_in = s_bar + 8u * kMaxRing;  // rows and scale
-  const bool scale_bulk = P.scale && (reinterpret_cast<uintptr_t>(P.scale) & 15) == 0;
 
   // one thread requests whole stages with bulk copies (three per stage); the
   // stage's mbarrier completes when all 6d bytes have landed
@@ -93,48 +90,46 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
     }
   };
   if (tid == 0) {
-    for (int k = 0; k <= kMaxRing; ++k) mbar_init(s_bar + 8u * k, 1);
+    for (int k = 0; k < kMaxRing; ++k) mbar_init(s_bar + 8u * k, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    const uint32_t in_bytes = (uint32_t)(nrows * 2 * d) + (scale_bulk ? 4u * d : 0u);
-    mbar_expect_tx(bar_in, in_bytes);
-    bulk_g2s(static_cast<uint32_t>(__cvta_generic_to_shared(xst)), P.x + (size_t)row0 * d, (uint32_t)(nrows * 2 * d),
-             bar_in);
-    if (scale_bulk) bulk_g2s(static_cast<uint32_t>(__cvta_generic_to_shared(fac)), P.scale, 4u * d, bar_in);
     for (int k = 0; k < ring; ++k) issue_stage(k);
+    // then the stages beyond the ring go to L2, so that their copies into the
+    // ring later wait for L2 rather than HBM
+    if (K > ring) {
+      const size_t off = (size_t)ring * half, bytes = (size_t)(K - ring) * 2 * d;
+      bulk_prefetch_l2(P.pairs + off, bytes);
+      bulk_prefetch_l2(P.cos_t + off, bytes);
+      bulk_prefetch_l2(P.sin_t + off, bytes);
+    }
+    if (P.scale && (reinterpret_cast<uintptr_t>(P.scale) & 15) == 0) bulk_prefetch_l2(P.scale, (size_t)4 * d);
   }
-  __syncthreads();  // barriers initialised before anyone waits on them
-
-  bool ok = mbar_wait_bounded(bar_in, 0);
-  // rows -> xs as fp32 (channel-major), factors 1/s
-  for (int cp = tid; cp < half && ok; cp += kRotThreads) {
-    float v0[R], v1[R];
+  // rows -> xs as fp32: each thread two adjacent channels of every row, the
+  // loads of LB channel pairs issued before their stores so that their
+  // latencies overlap
+  constexpr int LB = R == 4 ? 2 : (R == 2 ? 4 : 8);
+#pragma unroll 1
+  for (int cp0 = tid; cp0 < half; cp0 += LB * kRotThreads) {
+    __nv_bfloat162 v[LB][R];
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      if (r < nrows) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xst + (size_t)r * d + 2 * cp));
-        v0[r] = f.x; v1[r] = f.y;
-      } else {
-        v0[r] = 0.f; v1[r] = 0.f;
+    for (int q = 0; q < LB; ++q)
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int cp = cp0 + q * kRotThreads;
+        v[q][r] = __floats2bfloat162_rn(0.f, 0.f);
+        if (cp < half && r < nrows)
+          v[q][r] = *reinterpret_cast<const __nv_bfloat162*>(P.x + (size_t)(row0 + r) * d + 2 * cp);
+      }
+#pragma unroll
+    for (int q = 0; q < LB; ++q) {
+      const int cp = cp0 + q * kRotThreads;
+      if (cp < half) {
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          *reinterpret_cast<float2*>(xs + (size_t)r * d + 2 * cp) = __bfloat1622float2(v[q][r]);
       }
     }
-#pragma unroll
-    for (int r = 0; r < R; ++r) *reinterpret_cast<float2*>(xs + (size_t)r * d + 2 * cp) = make_float2(v0[r], v1[r]);
-    float s0 = 1.f, s1 = 1.f;
-    if (P.scale) {
-      if (scale_bulk) { s0 = fac[2 * cp]; s1 = fac[2 * cp + 1]; }
-      else { s0 = __ldg(P.scale + 2 * cp); s1 = __ldg(P.scale + 2 * cp + 1); }
-    }
-    fac[2 * cp] = 1.0f / s0;
-    fac[2 * cp + 1] = 1.0f / s1;
   }
-  if (__syncthreads_or(!ok)) {
-    // the rows never arrived: report, let the stage copies in flight land (bounded), leave
-    report_status(status, kStatusTimeout);
-    if (tid == 0)
-      for (int q = 0; q < K && q < ring; ++q) mbar_wait_bounded(s_bar + 8u * q, 0);
-    __syncthreads();
-    return;
-  }
+  __syncthreads();  // rows staged; barriers initialised before anyone waits on them
 
   // K stages.  The pairs of a stage are disjoint, so the loads of a batch of
   // pairs may all be issued before any of its stores.
@@ -200,28 +195,40 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
     if (tid == 0) issue_stage(k + ring);  // refill the slot this stage used
   }
 
-  // channel scale and store
-  for (int cp = tid; cp < half; cp += kRotThreads) {
-    const int c = 2 * cp;
-    const float f0 = fac[c], f1 = fac[c + 1];
+  // channel scale and store: the scales of LB channel pairs are loaded (from
+  // L2, where the prologue put them) before any of them is used
+#pragma unroll 1
+  for (int cp0 = tid; cp0 < half; cp0 += LB * kRotThreads) {
+    float2 sc[LB];
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      if (r < nrows) {
-        const float2 v = *reinterpret_cast<const float2*>(xs + (size_t)r * d + c);
-        const size_t off = (size_t)(row0 + r) * d + c;
-        if constexpr (F16OUT)
-          *reinterpret_cast<__half2*>(static_cast<__half*>(P.out) + off) = __floats2half2_rn(v.x * f0, v.y * f1);
-        else
-          *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(P.out) + off) =
-              __floats2bfloat162_rn(v.x * f0, v.y * f1);
+    for (int q = 0; q < LB; ++q) {
+      const int cp = cp0 + q * kRotThreads;
+      sc[q] = make_float2(1.0f, 1.0f);
+      if (P.scale && cp < half) sc[q] = make_float2(__ldg(P.scale + 2 * cp), __ldg(P.scale + 2 * cp + 1));
+    }
+#pragma unroll
+    for (int q = 0; q < LB; ++q) {
+      const int cp = cp0 + q * kRotThreads;
+      if (cp >= half) continue;
+      const int c = 2 * cp;
+      const float f0 = 1.0f / sc[q].x, f1 = 1.0f / sc[q].y;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (r < nrows) {
+          const float2 v = *reinterpret_cast<const float2*>(xs + (size_t)r * d + c);
+          const size_t off = (size_t)(row0 + r) * d + c;
+          if constexpr (F16OUT)
+            *reinterpret_cast<__half2*>(static_cast<__half*>(P.out) + off) = __floats2half2_rn(v.x * f0, v.y * f1);
+          else
+            *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(P.out) + off) =
+                __floats2bfloat162_rn(v.x * f0, v.y * f1);
+        }
       }
     }
   }
 }
 
-size_t rot_smem(int d, int R, int ring) {
-  return (size_t)d * R * 4 + (size_t)d * R * 2 + (size_t)d * 4 + (size_t)ring * 6 * d;
-}
+size_t rot_smem(int d, int R, int ring) { return (size_t)d * R * 4 + (size_t)ring * 6 * d; }
 
 }  // namespace
 
@@ -235,9 +242,10 @@ cudaError_t plan_rot_batch(const RotProblem* probs, int count, RotBatch* out, in
   int maxM = 0;
   for (int i = 0; i < count; ++i) maxM = probs[i].M > maxM ? probs[i].M : maxM;
   int R = maxM >= 4 ? 4 : (maxM >= 2 ? 2 : 1);
-  // the widest problem must still hold its rows, factors and one stage
+  // the widest problem must still hold its rows and two stages (one copy in
+  // flight while the other is used)
   for (int i = 0; i < count; ++i)
-    while (R > 1 && rot_smem(probs[i].d, R, 1) > kRotSmemBudget) R >>= 1;
+    while (R > 1 && rot_smem(probs[i].d, R, probs[i].K > 1 ? 2 : 1) > kRotSmemBudget) R >>= 1;
   *out = RotBatch{};
   int ctas = 0;
   for (int i = 0; i < count; ++i) {
