@@ -4,28 +4,32 @@
 // pairwise rotations that survive deployment", section "From fake
 // quantization to a real TensorRT engine": the group-wise INT4 GEMM operator).
 //
-// One CTA computes a 128-token x 256-output tile, K in steps of 64 through a
+// One CTA computes a 256-token x 256-output tile, K in steps of 64 through a
 // ring of kStages shared-memory stages:
-//   warp 8, lane 0  TMA: the 128 x 64 fp16 activation tile (128-byte swizzle)
-//                   into stage s, completing on full_a[s]; with bf16
-//                   activations warps 10-17 instead load each token row, round
-//                   it to fp16 and store it in the same swizzled layout (fp16
-//                   operands keep the product error an order of magnitude
-//                   below bf16 ones);
-//   warps 0-7       dequantisation: each thread owns one weight row, loads
-//                   their packed words and scale/zero bits PD steps ahead in a
-//                   register ring, turns every word into
-//                   eight fp16 values (q - zero) * scale in column
-//                   order and stores them in the same 128-byte-swizzled
-//                   K-major layout the tensor core reads; then arrives on
-//                   full_b[s] after a proxy fence;
-//   warp 9, lane 0  MMA: four tcgen05.mma (kind::f16, K = 16 each) per step
-//                   into a 128 x 256 fp32 accumulator in tensor memory, then
-//                   tcgen05.commit to empty[s] (the stage may be refilled once
-//                   the MMAs that read it are done) and, after the last step,
-//                   to acc_full;
-//   warps 0-7       epilogue: tcgen05.ld of their 32 lanes (tokens) and one
-//                   half of the 256 columns, bf16 round, 64-byte stores.
+//   warp 16, lane 0 TMA: the stage's packed codes (256 rows x 32 bytes, 32-byte
+//                   swizzle), completing on full_c[s], and the 256 x 64 fp16
+//                   activation tile (128-byte swizzle), completing on
+//                   full_a[s]; with bf16 activations warps 18-25 instead load
+//                   each token row, round it to fp16 and store it in the same
+//                   swizzled layout (fp16 operands keep the product error an
+//                   order of magnitude below bf16 ones);
+//   warps 0-15      dequantisation: thread (row t, half h) reads its 16 bytes
+//                   of the stage's codes from shared memory, holds its row's
+//                   scale and zero bits (loaded once per 128-column group, a
+//                   few groups ahead), turns every word into eight fp16 values
+//                   (q - zero) * scale in column order and stores them in the
+//                   128-byte-swizzled K-major layout the tensor core reads;
+//                   then arrives on full_b[s] after a proxy fence;
+//   warp 17, lane 0 MMA: four tcgen05.mma (kind::f16, K = 16, N = 256) per step
+//                   and token half into two 128 x 256 fp32 accumulators in tensor
+//                   memory, then tcgen05.commit to empty[s] (the stage may be
+//                   refilled once the MMAs that read it are done) and, after
+//                   the last step, to acc_full;
+//   warps 0-15      epilogue: tcgen05.ld of their 32 lanes (tokens) and 128
+//                   columns of one accumulator, bf16 round, 64-byte stores.
+// A 256 x 256 tile reads each activation tile once per 256 outputs: the
+// tensor core's shared-memory operand traffic per flop is 3/4 of that of a
+// 256 x 128 tile.
 // Every mbarrier wait is bounded; a wait that gives up sets PARO_ERR_TIMEOUT,
 // stops the pipeline and still releases the tensor memory.
 #include <cuda.h>
@@ -36,20 +40,21 @@
 namespace paro {
 namespace {
 
-constexpr int BM = 256, BN = 128, BK = 64;  // two 128-token MMA halves share each B tile
+constexpr int BM = 256, BN = 256, BK = 64;  // two 128-token MMA halves share each B tile
 constexpr int MH = 128;                       // tokens per MMA (M of one tcgen05.mma)
-constexpr int kStages = 4;
-constexpr int kDqWarps = 8;       // warps 0-7: dequantisation (one weight row per thread), then epilogue
-constexpr int kWarpTma = 8;       // TMA producer, tensor-memory allocation
-constexpr int kWarpMma = 9;       // MMA issuer
-constexpr int kWarpConv = 10;     // warps 10-17: bf16 activations -> fp16 tiles (bf16 input only)
-constexpr int kThreadsTma = 320;
-constexpr int kThreadsConv = 576;
+constexpr int kStages = 3;
+constexpr int kDqWarps = 16;      // warps 0-15: dequantisation (one weight row per thread), then epilogue
+constexpr int kWarpTma = 16;      // TMA producer, tensor-memory allocation
+constexpr int kWarpMma = 17;      // MMA issuer
+constexpr int kWarpConv = 18;     // warps 18-25: bf16 activations -> fp16 tiles (bf16 input only)
+constexpr int kThreadsTma = 576;
+constexpr int kThreadsConv = 832;
 constexpr int A_BYTES = BM * BK * 2;  // 32 KB
-constexpr int B_BYTES = BN * BK * 2;  // 16 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int B_BYTES = BN * BK * 2;  // 32 KB
+constexpr int C_BYTES = BN * BK / 2;  // 8 KB of packed codes (256 rows x 32 bytes, 32-byte swizzle)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
 constexpr int SMEM_BYTES = kStages * STAGE_BYTES + 1024;  // + alignment slack
-constexpr uint32_t kTmemCols = 256;  // two 128 x 128 fp32 accumulators
+constexpr uint32_t kTmemCols = 512;  // two 128 x 256 fp32 accumulators (all of tensor memory)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -99,7 +104,7 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 }
 
 __host__ __device__ constexpr uint32_t instr_desc() {
-  // fp32 accumulate, A and B fp16, both K-major, N = BN = 128, M = 128
+  // fp32 accumulate, A and B fp16, both K-major, N = BN = 256, M = 128
   return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(MH >> 4) << 24);
 }
 
@@ -145,13 +150,14 @@ __device__ __forceinline__ void dequant8(uint32_t w, uint32_t zc, uint32_t sc, u
 
 template <bool XF16>
 __global__ void __launch_bounds__(XF16 ? kThreadsTma : kThreadsConv, 1)
-w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ xraw,
+w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap qmap,
+             const uint16_t* __restrict__ xraw,
              const uint32_t* __restrict__ qweight, const __half* __restrict__ scales,
              const __half* __restrict__ zeros, __nv_bfloat16* __restrict__ y, int M, int d_in, int d_out,
              int* status) {
   constexpr bool F16 = true;  // tensor-core operands are fp16 in both variants
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  __shared__ __align__(8) uint64_t bars[3 * kStages + 1];
+  __shared__ __align__(8) uint64_t bars[4 * kStages + 1];
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
 
@@ -162,6 +168,7 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restric
   const uint32_t b_full_b = smem_u32(&bars[kStages]);
   const uint32_t b_empty = smem_u32(&bars[2 * kStages]);
   const uint32_t b_acc = smem_u32(&bars[3 * kStages]);
+  const uint32_t b_full_c = smem_u32(&bars[3 * kStages + 1]);  // codes of a stage landed
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
@@ -173,6 +180,7 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restric
       mbar_init(b_full_a + 8 * s, XF16 ? 1 : BM);
       mbar_init(b_full_b + 8 * s, kDqWarps * 32);
       mbar_init(b_empty + 8 * s, 1);
+      mbar_init(b_full_c + 8 * s, 1);
     }
     mbar_init(b_acc, 1);
     abort_flag = 0;
@@ -244,14 +252,18 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restric
       }
     }
   } else if (warp == kWarpTma) {
-    // ---------------- TMA producer (fp16 input) ------------------------------------
-    if (XF16 && lane == 0) {
+    // ---------------- TMA producer: packed codes (both variants), fp16 activations ---
+    if (lane == 0) {
       for (int k = 0; k < nk; ++k) {
         const int s = k % kStages;
         if (k >= kStages && !mbar_wait(b_empty + 8 * s, ((k / kStages) - 1) & 1)) { fail(); break; }
         if (*(volatile int*)&abort_flag) break;
-        mbar_expect_tx(b_full_a + 8 * s, A_BYTES);
-        tma_load_2d(s_base + s * STAGE_BYTES, &xmap, k * BK, m0, b_full_a + 8 * s);
+        mbar_expect_tx(b_full_c + 8 * s, C_BYTES);
+        tma_load_2d(s_base + s * STAGE_BYTES + A_BYTES + B_BYTES, &qmap, k * (BK / 8), n0, b_full_c + 8 * s);
+        if (XF16) {
+          mbar_expect_tx(b_full_a + 8 * s, A_BYTES);
+          tma_load_2d(s_base + s * STAGE_BYTES, &xmap, k * BK, m0, b_full_a + 8 * s);
+        }
       }
     }
   } else if (warp == kWarpMma) {
@@ -279,48 +291,54 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restric
       mma_commit(b_acc);  // arrives once every MMA issued above has completed
     }
   } else {
-    // ---------------- dequantisation (warps 0-3), then epilogue ----------------------
+    // ---------------- dequantisation (warps 0-7), then epilogue ----------------------
     const int t = threadIdx.x & (BN - 1);  // row of the tile
     const int hw = threadIdx.x / BN;        // which half of the row's 64 columns (4 words)
-    const int wpr = d_in >> 3;
     const int rA = n0 + t;
     const bool okA = rA < d_out;
-    const uint32_t* qa = qweight + (size_t)(okA ? rA : 0) * wpr + hw * 4;
     const unsigned short* sA = reinterpret_cast<const unsigned short*>(scales) + (size_t)(okA ? rA : 0) * G;
     const unsigned short* zA = reinterpret_cast<const unsigned short*>(zeros) + (size_t)(okA ? rA : 0) * G;
-    // register ring: words and raw scale/zero bits of the next PD steps, so that
-    // every load has PD steps of work to land before it is used
+    // this thread's 16 bytes of the stage's codes: row t holds 32 bytes, its
+    // 16-byte halves swapped on rows with bit 2 set (the 32-byte swizzle)
+    const uint32_t c_off = (uint32_t)(A_BYTES + B_BYTES + t * 32 + ((hw ^ ((t >> 2) & 1)) << 4));
+    // scale and zero bits of a group, PD groups ahead in a register ring
+    constexpr int SPG = kGroup / BK;  // steps per group
     constexpr int PD = 4;
-    uint4 wq[PD];
     uint32_t sz[PD][2];
-    auto load_step = [&](int k, uint4& w, uint32_t (&z)[2]) {
-      if (k < nk && okA) {
-        const int grp = (k * BK) / kGroup;
-        w = __ldg(reinterpret_cast<const uint4*>(qa + k * 8));
-        z[0] = __ldg(sA + grp);
-        z[1] = __ldg(zA + grp);
+    auto load_group = [&](int g, uint32_t (&z)[2]) {
+      if (g < G && okA) {
+        z[0] = __ldg(sA + g);
+        z[1] = __ldg(zA + g);
       }
     };
 #pragma unroll
-    for (int j = 0; j < PD - 1; ++j) load_step(j, wq[j], sz[j]);
+    for (int j = 0; j < PD - 1; ++j) load_group(j, sz[j]);
     bool stop = false;
-    for (int kb = 0; kb < nk && !stop; kb += PD) {
+    for (int kb = 0; kb < nk && !stop; kb += PD * SPG) {
 #pragma unroll
-      for (int j = 0; j < PD; ++j) {
+      for (int j = 0; j < PD * SPG; ++j) {
         const int k = kb + j;
         if (k >= nk) break;
-        load_step(k + PD - 1, wq[(j + PD - 1) % PD], sz[(j + PD - 1) % PD]);
+        const int gj = j / SPG;  // ring slot of this step's group
+        if (j % SPG == 0) load_group(k / SPG + PD - 1, sz[(gj + PD - 1) % PD]);
         const int s = k % kStages;
-        if (k >= kStages && !mbar_wait(b_empty + 8 * s, ((k / kStages) - 1) & 1)) fail();
+        const uint32_t par = (k / kStages) & 1;
+        if (k >= kStages && !mbar_wait(b_empty + 8 * s, par ^ 1)) fail();
+        if (!mbar_wait(b_full_c + 8 * s, par)) fail();
         if (*(volatile int*)&abort_flag) { stop = true; break; }
         uint32_t zc = 0, sc = 0;
         if (okA) {
-          const float z = __half2float(__ushort_as_half((unsigned short)sz[j][1]));
+          const float z = __half2float(__ushort_as_half((unsigned short)sz[gj][1]));
           const __half2 zz = __float2half2_rn(1024.f + z);
           zc = *reinterpret_cast<const uint32_t*>(&zz);
-          sc = (sz[j][0] & 0xFFFFu) * 0x00010001u;
+          sc = (sz[gj][0] & 0xFFFFu) * 0x00010001u;
         }
-        const uint32_t wv[4] = {wq[j].x, wq[j].y, wq[j].z, wq[j].w};
+        uint32_t wv[4];
+        {
+          const uint32_t a = s_base + (uint32_t)(s * STAGE_BYTES) + c_off;
+          asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                       : "=r"(wv[0]), "=r"(wv[1]), "=r"(wv[2]), "=r"(wv[3]) : "r"(a) : "memory");
+        }
         unsigned char* rowp = smem + s * STAGE_BYTES + A_BYTES + t * 128;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {  // 16-byte chunk = 8 columns = one word
@@ -340,11 +358,12 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restric
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
     if (done && !*(volatile int*)&abort_flag) {
       const int q = warp & 3;                 // TMEM lane quarter this warp may access
-      const int h = warp >> 2;                // token half (accumulator) this warp drains
+      const int h = (warp >> 2) & 1;          // token half (accumulator) this warp drains
+      const int cb = (warp >> 3) * (BN / 2);  // and which half of its columns
       const int m = m0 + h * MH + q * 32 + lane;  // token of this thread's TMEM lane
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * BN);
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * BN + cb);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = 0; c0 < BN / 2; c0 += 32) {
         uint32_t v[32];
         asm volatile(
             "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -355,8 +374,9 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restric
               "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
             : "r"(taddr + c0));
         asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-        if (m < M && n0 + c0 < d_out) {
-          __nv_bfloat16* dst = y + (size_t)m * d_out + n0 + c0;
+        const int n = n0 + cb + c0;  // first output column of this chunk
+        if (m < M && n < d_out) {
+          __nv_bfloat16* dst = y + (size_t)m * d_out + n;
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -364,7 +384,7 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restric
             pk[i] = *reinterpret_cast<const uint32_t*>(&b2);
           }
           // d_out is a multiple of 16: the last 32-column chunk may hold only 16
-          const int nq = (n0 + c0 + 32 <= d_out) ? 4 : 2;
+          const int nq = (n + 32 <= d_out) ? 4 : 2;
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             if (i < nq)
@@ -377,11 +397,15 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restric
   // ---------------- teardown --------------------------------------------------------
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
-  if (XF16 && abort_flag && threadIdx.x == 0) {
+  if (abort_flag && threadIdx.x == 0) {
     // let any copies and MMAs still in flight land before the memory goes away
     for (int s = 0; s < kStages; ++s) {
-      mbar_wait(b_full_a + 8 * s, 0);
-      mbar_wait(b_full_a + 8 * s, 1);
+      if (XF16) {
+        mbar_wait(b_full_a + 8 * s, 0);
+        mbar_wait(b_full_a + 8 * s, 1);
+      }
+      mbar_wait(b_full_c + 8 * s, 0);
+      mbar_wait(b_full_c + 8 * s, 1);
     }
     mbar_wait(b_acc, 0);
   }
@@ -429,17 +453,27 @@ cudaError_t launch_w4_tc(const uint16_t* x, bool x_f16, const uint32_t* qweight,
                    const_cast<uint16_t*>(x), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  CUtensorMap qmap;  // packed codes: uint32 [d_out][d_in / 8], one box = 8 words x 128 rows
+  {
+    const cuuint64_t qdims[2] = {(cuuint64_t)(d_in / 8), (cuuint64_t)d_out};
+    const cuuint64_t qstrides[1] = {(cuuint64_t)d_in / 2};
+    const cuuint32_t qbox[2] = {BK / 8, BN};
+    r = enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(qweight), qdims, qstrides, qbox, elem,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
   const dim3 grid((d_out + BN - 1) / BN, (M + BM - 1) / BM);
   cudaError_t e;
   if (x_f16) {
     e = cudaFuncSetAttribute(w4_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    w4_tc_kernel<true><<<grid, kThreadsTma, SMEM_BYTES, stream>>>(map, x, qweight, scales, zeros, y, M, d_in, d_out,
+    w4_tc_kernel<true><<<grid, kThreadsTma, SMEM_BYTES, stream>>>(map, qmap, x, qweight, scales, zeros, y, M, d_in, d_out,
                                                                   status);
   } else {
     e = cudaFuncSetAttribute(w4_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    w4_tc_kernel<false><<<grid, kThreadsConv, SMEM_BYTES, stream>>>(map, x, qweight, scales, zeros, y, M, d_in,
+    w4_tc_kernel<false><<<grid, kThreadsConv, SMEM_BYTES, stream>>>(map, qmap, x, qweight, scales, zeros, y, M, d_in,
                                                                     d_out, status);
   }
   return cudaPeekAtLastError();
