@@ -454,18 +454,25 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     e = paro::plan_rot_batch(rp, n, &rb, &R);
     if (e == cudaSuccess) e = paro::launch_rot_batch(rb, R, true, status, s, true);
   } else {
-    // many tokens (or tables the decode kernel cannot take): one transform and one
-    // linear per layer, each linear on the tensor-core kernel when it applies
+    // many tokens (or tables the decode kernel cannot take): every transform, then
+    // one persistent tensor-core launch over all linears it takes (their tiles
+    // balanced over the SMs together); any other linear on its own
     e = cudaSuccess;
-    for (int i = 0; i < n && e == cudaSuccess; ++i) {
+    for (int i = 0; i < n && e == cudaSuccess; ++i)
       e = launch_transform(rp[i].x, rp[i].out, true, rp[i].M, rp[i].d, rp[i].K,
                            reinterpret_cast<const uint16_t*>(rp[i].pairs), rp[i].cos_t, rp[i].sin_t, rp[i].scale,
-                           status, s, true);
-      if (e == cudaSuccess)
+                           status, s, false);
+    paro::TcLinear tl[PARO_MAX_BATCH];
+    int ntc = 0;
+    for (int i = 0; i < n && e == cudaSuccess; ++i) {
+      if (gp[i].M >= kTensorCoreMinM && paro::tc_supported(gp[i].M, gp[i].d_in, gp[i].d_out, gp[i].x))
+        tl[ntc++] = paro::TcLinear{gp[i].x, gp[i].qw, gp[i].sc, gp[i].z, gp[i].y, gp[i].M, gp[i].d_in, gp[i].d_out};
+      else
         e = launch_linear(gp[i].x, true, gp[i].qw, reinterpret_cast<const uint16_t*>(gp[i].sc),
                           reinterpret_cast<const uint16_t*>(gp[i].z), reinterpret_cast<uint16_t*>(gp[i].y), gp[i].M,
-                          gp[i].d_in, gp[i].d_out, s, true, status);
+                          gp[i].d_in, gp[i].d_out, s, false, status);
     }
+    if (e == cudaSuccess && ntc > 0) e = paro::launch_w4_tc_batch(tl, ntc, true, status, s);
     return from_cuda(e, "batched launch");
   }
   if (e != cudaSuccess) return from_cuda(e, "batched transform launch");

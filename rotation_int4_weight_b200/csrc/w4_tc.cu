@@ -36,6 +36,7 @@
 
 #include "paro_internal.cuh"
 #include "w4_tc.cuh"
+#include "w4_stream.cuh"  // device_sm_count
 
 namespace paro {
 namespace {
@@ -148,18 +149,45 @@ __device__ __forceinline__ void dequant8(uint32_t w, uint32_t zc, uint32_t sc, u
   }
 }
 
+// Per-linear scalars of a launch, copied into shared memory at kernel start
+// (the tile walk indexes linears by a runtime number).
+struct TcMeta {
+  const uint16_t* xraw;
+  const unsigned short* sc;
+  const unsigned short* z;
+  __nv_bfloat16* y;
+  int M, d_in, d_out, n_tiles, tile_begin;
+};
+
+// The j-th tile of this CTA, or -1: tiles go out in rounds of gridDim.x, in
+// ascending CTA order on even rounds and descending order on odd ones, so that
+// the CTAs given the first (longest) tiles get the last partial round least.
+__device__ __forceinline__ int tile_of(int j, int total) {
+  const int G = (int)gridDim.x, c = (int)blockIdx.x;
+  const int t = j * G + ((j & 1) ? (G - 1 - c) : c);
+  return t < total ? t : -1;
+}
+struct TileInfo {
+  int pi, m0, n0, nk;
+};
+__device__ __forceinline__ TileInfo tile_info(const TcMeta* mt, int count, int t) {
+  int pi = 0;
+#pragma unroll 1
+  while (pi + 1 < count && t >= mt[pi + 1].tile_begin) ++pi;
+  const int local = t - mt[pi].tile_begin;
+  const int mtile = local / mt[pi].n_tiles, ntile = local - mtile * mt[pi].n_tiles;
+  return TileInfo{pi, mtile * BM, ntile * BN, mt[pi].d_in / BK};
+}
+
 template <bool XF16>
 __global__ void __launch_bounds__(XF16 ? kThreadsTma : kThreadsConv, 1)
-w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap qmap,
-             const uint16_t* __restrict__ xraw,
-             const uint32_t* __restrict__ qweight, const __half* __restrict__ scales,
-             const __half* __restrict__ zeros, __nv_bfloat16* __restrict__ y, int M, int d_in, int d_out,
-             int* status) {
+w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
   constexpr bool F16 = true;  // tensor-core operands are fp16 in both variants
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  __shared__ __align__(8) uint64_t bars[4 * kStages + 1];
+  __shared__ __align__(8) uint64_t bars[4 * kStages + 2];
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
+  __shared__ TcMeta meta[kTcMaxBatch];
 
   // the 128-byte swizzle needs every tile at a 1024-byte aligned shared address
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -167,14 +195,19 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ C
   const uint32_t b_full_a = smem_u32(&bars[0]);
   const uint32_t b_full_b = smem_u32(&bars[kStages]);
   const uint32_t b_empty = smem_u32(&bars[2 * kStages]);
-  const uint32_t b_acc = smem_u32(&bars[3 * kStages]);
-  const uint32_t b_full_c = smem_u32(&bars[3 * kStages + 1]);  // codes of a stage landed
+  const uint32_t b_full_c = smem_u32(&bars[3 * kStages]);    // codes of a stage landed
+  const uint32_t b_acc_full = smem_u32(&bars[4 * kStages]);  // a tile's accumulator is complete
+  const uint32_t b_acc_empty = smem_u32(&bars[4 * kStages + 1]);  // ... and has been read out
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-  const int nk = d_in / BK;
-  const int G = d_in / kGroup;
+  const int total = b.total_tiles, count = b.count;
 
+  if (threadIdx.x < count) {
+    const TcProblem& P = b.p[threadIdx.x];
+    meta[threadIdx.x] = TcMeta{P.xraw, P.sc, P.z, P.y, P.M, P.d_in, P.d_out, P.n_tiles, P.tile_begin};
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&P.qmap)) : "memory");
+    if (XF16) asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&P.xmap)) : "memory");
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(b_full_a + 8 * s, XF16 ? 1 : BM);
@@ -182,11 +215,12 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ C
       mbar_init(b_empty + 8 * s, 1);
       mbar_init(b_full_c + 8 * s, 1);
     }
-    mbar_init(b_acc, 1);
+    mbar_init(b_acc_full, 1);
+    mbar_init(b_acc_empty, kDqWarps * 32);
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (warp == kWarpTma) {  // tensor memory for the accumulator
+  if (warp == kWarpTma) {  // tensor memory for the accumulators
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_base_slot)),
                  "r"(kTmemCols)
                  : "memory");
@@ -201,68 +235,89 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ C
     report_status(status, kStatusTimeout);
     atomicExch(&abort_flag, 1);
   };
+  auto aborted = [&]() { return *(volatile int*)&abort_flag != 0; };
 
   if (warp >= kWarpConv) {
     // ---------------- bf16 activations -> fp16 tiles (bf16 input only) ---------------
     if constexpr (!XF16) {
       const int t = threadIdx.x - kWarpConv * 32;  // row of the 256-token tile
-      const int m = m0 + t;
-      const bool okm = m < M;
-      const uint16_t* xr = xraw + (size_t)(okm ? m : 0) * d_in;
-      constexpr int PX = 2;  // steps of loads in flight
-      uint4 xq[PX][8];
-      auto load_x = [&](int k, uint4 (&v)[8]) {
-        if (k < nk && okm) {
-#pragma unroll
-          for (int c = 0; c < 8; ++c) v[c] = __ldg(reinterpret_cast<const uint4*>(xr + k * BK + c * 8));
-        }
-      };
-#pragma unroll
-      for (int j = 0; j < PX - 1; ++j) load_x(j, xq[j]);
+      int it = 0;
       bool stop = false;
-      for (int kb = 0; kb < nk && !stop; kb += PX) {
+#pragma unroll 1
+      for (int j = 0; !stop; ++j) {
+        const int T = tile_of(j, total);
+        if (T < 0) break;
+        const TileInfo ti = tile_info(meta, count, T);
+        const TcMeta& P = meta[ti.pi];
+        const int m = ti.m0 + t;
+        const bool okm = m < P.M;
+        const uint16_t* xr = P.xraw + (size_t)(okm ? m : 0) * P.d_in;
+        constexpr int PX = 2;  // steps of loads in flight
+        uint4 xq[PX][8];
+        auto load_x = [&](int k, uint4 (&v)[8]) {
+          if (k < ti.nk && okm) {
 #pragma unroll
-        for (int j = 0; j < PX; ++j) {
-          const int k = kb + j;
-          if (k >= nk) break;
-          load_x(k + PX - 1, xq[(j + PX - 1) % PX]);
-          const int s = k % kStages;
-          if (k >= kStages && !mbar_wait(b_empty + 8 * s, ((k / kStages) - 1) & 1)) fail();
-          if (*(volatile int*)&abort_flag) { stop = true; break; }
-          unsigned char* rowp = smem + s * STAGE_BYTES + t * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4 o = make_uint4(0u, 0u, 0u, 0u);
-            if (okm) {
-              const uint32_t in[4] = {xq[j][c].x, xq[j][c].y, xq[j][c].z, xq[j][c].w};
-              uint32_t out[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[e]));
-                const __half2 h = __floats2half2_rn(f.x, f.y);
-                out[e] = *reinterpret_cast<const uint32_t*>(&h);
-              }
-              o = make_uint4(out[0], out[1], out[2], out[3]);
-            }
-            *reinterpret_cast<uint4*>(rowp + ((c ^ (t & 7)) << 4)) = o;
+            for (int c = 0; c < 8; ++c) v[c] = __ldg(reinterpret_cast<const uint4*>(xr + k * BK + c * 8));
           }
-          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-          mbar_arrive(b_full_a + 8 * s);
+        };
+#pragma unroll
+        for (int q = 0; q < PX - 1; ++q) load_x(q, xq[q]);
+#pragma unroll 1
+        for (int kb = 0; kb < ti.nk && !stop; kb += PX) {
+#pragma unroll
+          for (int q = 0; q < PX; ++q) {
+            const int k = kb + q;
+            if (k >= ti.nk) break;
+            load_x(k + PX - 1, xq[(q + PX - 1) % PX]);
+            const int s = it % kStages;
+            if (it >= kStages && !mbar_wait(b_empty + 8 * s, ((it / kStages) - 1) & 1)) fail();
+            if (aborted()) { stop = true; break; }
+            unsigned char* rowp = smem + s * STAGE_BYTES + t * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint4 o = make_uint4(0u, 0u, 0u, 0u);
+              if (okm) {
+                const uint32_t in[4] = {xq[q][c].x, xq[q][c].y, xq[q][c].z, xq[q][c].w};
+                uint32_t out[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[e]));
+                  const __half2 h = __floats2half2_rn(f.x, f.y);
+                  out[e] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+                o = make_uint4(out[0], out[1], out[2], out[3]);
+              }
+              *reinterpret_cast<uint4*>(rowp + ((c ^ (t & 7)) << 4)) = o;
+            }
+            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            mbar_arrive(b_full_a + 8 * s);
+            ++it;
+          }
         }
       }
     }
   } else if (warp == kWarpTma) {
     // ---------------- TMA producer: packed codes (both variants), fp16 activations ---
     if (lane == 0) {
-      for (int k = 0; k < nk; ++k) {
-        const int s = k % kStages;
-        if (k >= kStages && !mbar_wait(b_empty + 8 * s, ((k / kStages) - 1) & 1)) { fail(); break; }
-        if (*(volatile int*)&abort_flag) break;
-        mbar_expect_tx(b_full_c + 8 * s, C_BYTES);
-        tma_load_2d(s_base + s * STAGE_BYTES + A_BYTES + B_BYTES, &qmap, k * (BK / 8), n0, b_full_c + 8 * s);
-        if (XF16) {
-          mbar_expect_tx(b_full_a + 8 * s, A_BYTES);
-          tma_load_2d(s_base + s * STAGE_BYTES, &xmap, k * BK, m0, b_full_a + 8 * s);
+      int it = 0;
+      bool stop = false;
+#pragma unroll 1
+      for (int j = 0; !stop; ++j) {
+        const int T = tile_of(j, total);
+        if (T < 0) break;
+        const TileInfo ti = tile_info(meta, count, T);
+        const TcProblem& P = b.p[ti.pi];
+#pragma unroll 1
+        for (int k = 0; k < ti.nk; ++k, ++it) {
+          const int s = it % kStages;
+          if (it >= kStages && !mbar_wait(b_empty + 8 * s, ((it / kStages) - 1) & 1)) { fail(); stop = true; break; }
+          if (aborted()) { stop = true; break; }
+          mbar_expect_tx(b_full_c + 8 * s, C_BYTES);
+          tma_load_2d(s_base + s * STAGE_BYTES + A_BYTES + B_BYTES, &P.qmap, k * (BK / 8), ti.n0, b_full_c + 8 * s);
+          if (XF16) {
+            mbar_expect_tx(b_full_a + 8 * s, A_BYTES);
+            tma_load_2d(s_base + s * STAGE_BYTES, &P.xmap, k * BK, ti.m0, b_full_a + 8 * s);
+          }
         }
       }
     }
@@ -270,127 +325,152 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ C
     // ---------------- MMA issuer ---------------------------------------------------
     if (lane == 0) {
       constexpr uint32_t idesc = instr_desc();
+      int it = 0;
       bool ok = true;
-      for (int k = 0; k < nk && ok; ++k) {
-        const int s = k % kStages;
-        const uint32_t par = (k / kStages) & 1;
-        if (!mbar_wait(b_full_a + 8 * s, par) || !mbar_wait(b_full_b + 8 * s, par)) { fail(); ok = false; break; }
-        if (*(volatile int*)&abort_flag) { ok = false; break; }
+#pragma unroll 1
+      for (int j = 0; ok; ++j) {
+        const int T = tile_of(j, total);
+        if (T < 0) break;
+        const TileInfo ti = tile_info(meta, count, T);
+        // the previous tile's accumulators must have been read out
+        if (j > 0 && !mbar_wait(b_acc_empty, (j - 1) & 1)) { fail(); ok = false; break; }
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-        const uint32_t a_addr = s_base + s * STAGE_BYTES, b_addr = a_addr + A_BYTES;
+#pragma unroll 1
+        for (int k = 0; k < ti.nk; ++k, ++it) {
+          const int s = it % kStages;
+          const uint32_t par = (it / kStages) & 1;
+          if (!mbar_wait(b_full_a + 8 * s, par) || !mbar_wait(b_full_b + 8 * s, par)) { fail(); ok = false; break; }
+          if (aborted()) { ok = false; break; }
+          asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+          const uint32_t a_addr = s_base + s * STAGE_BYTES, b_addr = a_addr + A_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 32);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 32);
 #pragma unroll
-          for (int h = 0; h < BM / MH; ++h)  // token half h -> accumulator columns [h * BN, (h + 1) * BN)
-            mma_f16(tmem + h * BN, smem_desc_sw128(a_addr + h * (MH * 128) + kk * 32), bdesc, idesc,
-                    (k > 0 || kk > 0) ? 1u : 0u);
+            for (int h = 0; h < BM / MH; ++h)  // token half h -> accumulator columns [h * BN, (h + 1) * BN)
+              mma_f16(tmem + h * BN, smem_desc_sw128(a_addr + h * (MH * 128) + kk * 32), bdesc, idesc,
+                      (k > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(b_empty + 8 * s);
         }
-        mma_commit(b_empty + 8 * s);
+        if (ok) mma_commit(b_acc_full);  // arrives once every MMA of the tile has completed
       }
-      mma_commit(b_acc);  // arrives once every MMA issued above has completed
     }
   } else {
-    // ---------------- dequantisation (warps 0-7), then epilogue ----------------------
+    // ---------------- dequantisation (warps 0-15), then each tile's epilogue ----------
     const int t = threadIdx.x & (BN - 1);  // row of the tile
     const int hw = threadIdx.x / BN;        // which half of the row's 64 columns (4 words)
-    const int rA = n0 + t;
-    const bool okA = rA < d_out;
-    const unsigned short* sA = reinterpret_cast<const unsigned short*>(scales) + (size_t)(okA ? rA : 0) * G;
-    const unsigned short* zA = reinterpret_cast<const unsigned short*>(zeros) + (size_t)(okA ? rA : 0) * G;
-    // this thread's 16 bytes of the stage's codes: row t holds 32 bytes, its
+    // this thread's 16 bytes of a stage's codes: row t holds 32 bytes, its
     // 16-byte halves swapped on rows with bit 2 set (the 32-byte swizzle)
     const uint32_t c_off = (uint32_t)(A_BYTES + B_BYTES + t * 32 + ((hw ^ ((t >> 2) & 1)) << 4));
-    // scale and zero bits of a group, PD groups ahead in a register ring
     constexpr int SPG = kGroup / BK;  // steps per group
-    constexpr int PD = 4;
-    uint32_t sz[PD][2];
-    auto load_group = [&](int g, uint32_t (&z)[2]) {
-      if (g < G && okA) {
-        z[0] = __ldg(sA + g);
-        z[1] = __ldg(zA + g);
-      }
-    };
-#pragma unroll
-    for (int j = 0; j < PD - 1; ++j) load_group(j, sz[j]);
+    constexpr int PD = 4;             // groups of scale/zero bits in flight
+    int it = 0;
     bool stop = false;
-    for (int kb = 0; kb < nk && !stop; kb += PD * SPG) {
-#pragma unroll
-      for (int j = 0; j < PD * SPG; ++j) {
-        const int k = kb + j;
-        if (k >= nk) break;
-        const int gj = j / SPG;  // ring slot of this step's group
-        if (j % SPG == 0) load_group(k / SPG + PD - 1, sz[(gj + PD - 1) % PD]);
-        const int s = k % kStages;
-        const uint32_t par = (k / kStages) & 1;
-        if (k >= kStages && !mbar_wait(b_empty + 8 * s, par ^ 1)) fail();
-        if (!mbar_wait(b_full_c + 8 * s, par)) fail();
-        if (*(volatile int*)&abort_flag) { stop = true; break; }
-        uint32_t zc = 0, sc = 0;
-        if (okA) {
-          const float z = __half2float(__ushort_as_half((unsigned short)sz[gj][1]));
-          const __half2 zz = __float2half2_rn(1024.f + z);
-          zc = *reinterpret_cast<const uint32_t*>(&zz);
-          sc = (sz[gj][0] & 0xFFFFu) * 0x00010001u;
-        }
-        uint32_t wv[4];
-        {
-          const uint32_t a = s_base + (uint32_t)(s * STAGE_BYTES) + c_off;
-          asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
-                       : "=r"(wv[0]), "=r"(wv[1]), "=r"(wv[2]), "=r"(wv[3]) : "r"(a) : "memory");
-        }
-        unsigned char* rowp = smem + s * STAGE_BYTES + A_BYTES + t * 128;
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {  // 16-byte chunk = 8 columns = one word
-          const int c = hw * 4 + c4;
-          uint32_t o[4] = {0u, 0u, 0u, 0u};
-          if (okA) dequant8<F16>(wv[c4], zc, sc, o);
-          *reinterpret_cast<uint4*>(rowp + ((c ^ (t & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // generic writes -> tensor core reads
-        mbar_arrive(b_full_b + 8 * s);
-      }
-    }
-
-    // ---------------- epilogue -------------------------------------------------------
-    const bool done = mbar_wait(b_acc, 0);
-    if (!done) fail();
-    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-    if (done && !*(volatile int*)&abort_flag) {
-      const int q = warp & 3;                 // TMEM lane quarter this warp may access
-      const int h = (warp >> 2) & 1;          // token half (accumulator) this warp drains
-      const int cb = (warp >> 3) * (BN / 2);  // and which half of its columns
-      const int m = m0 + h * MH + q * 32 + lane;  // token of this thread's TMEM lane
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * BN + cb);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN / 2; c0 += 32) {
-        uint32_t v[32];
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-              "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-              "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-            : "r"(taddr + c0));
-        asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-        const int n = n0 + cb + c0;  // first output column of this chunk
-        if (m < M && n < d_out) {
-          __nv_bfloat16* dst = y + (size_t)m * d_out + n;
-          uint32_t pk[16];
+    for (int j = 0; !stop; ++j) {
+      const int T = tile_of(j, total);
+      if (T < 0) break;
+      const TileInfo ti = tile_info(meta, count, T);
+      const TcMeta& P = meta[ti.pi];
+      const int G = P.d_in / kGroup;
+      const int rA = ti.n0 + t;
+      const bool okA = rA < P.d_out;
+      const unsigned short* sA = P.sc + (size_t)(okA ? rA : 0) * G;
+      const unsigned short* zA = P.z + (size_t)(okA ? rA : 0) * G;
+      uint32_t sz[PD][2];
+      auto load_group = [&](int g, uint32_t (&z)[2]) {
+        if (g < G && okA) {
+          z[0] = __ldg(sA + g);
+          z[1] = __ldg(zA + g);
+        }
+      };
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            pk[i] = *reinterpret_cast<const uint32_t*>(&b2);
+      for (int q = 0; q < PD - 1; ++q) load_group(q, sz[q]);
+#pragma unroll 1
+      for (int kb = 0; kb < ti.nk && !stop; kb += PD * SPG) {
+#pragma unroll
+        for (int q = 0; q < PD * SPG; ++q) {
+          const int k = kb + q;
+          if (k >= ti.nk) break;
+          const int gj = q / SPG;  // ring slot of this step's group
+          if (q % SPG == 0) load_group(k / SPG + PD - 1, sz[(gj + PD - 1) % PD]);
+          const int s = it % kStages;
+          const uint32_t par = (it / kStages) & 1;
+          if (it >= kStages && !mbar_wait(b_empty + 8 * s, par ^ 1)) fail();
+          if (!mbar_wait(b_full_c + 8 * s, par)) fail();
+          if (aborted()) { stop = true; break; }
+          uint32_t zc = 0, sc = 0;
+          if (okA) {
+            const float z = __half2float(__ushort_as_half((unsigned short)sz[gj][1]));
+            const __half2 zz = __float2half2_rn(1024.f + z);
+            zc = *reinterpret_cast<const uint32_t*>(&zz);
+            sc = (sz[gj][0] & 0xFFFFu) * 0x00010001u;
           }
-          // d_out is a multiple of 16: the last 32-column chunk may hold only 16
-          const int nq = (n + 32 <= d_out) ? 4 : 2;
+          uint32_t wv[4];
+          {
+            const uint32_t a = s_base + (uint32_t)(s * STAGE_BYTES) + c_off;
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                         : "=r"(wv[0]), "=r"(wv[1]), "=r"(wv[2]), "=r"(wv[3]) : "r"(a) : "memory");
+          }
+          unsigned char* rowp = smem + s * STAGE_BYTES + A_BYTES + t * 128;
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            if (i < nq)
-              reinterpret_cast<uint4*>(dst)[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int c4 = 0; c4 < 4; ++c4) {  // 16-byte chunk = 8 columns = one word
+            const int c = hw * 4 + c4;
+            uint32_t o[4] = {0u, 0u, 0u, 0u};
+            if (okA) dequant8<F16>(wv[c4], zc, sc, o);
+            *reinterpret_cast<uint4*>(rowp + ((c ^ (t & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // generic writes -> tensor core reads
+          mbar_arrive(b_full_b + 8 * s);
+          ++it;
         }
       }
+      if (stop) break;
+
+      // ---------------- epilogue of this tile --------------------------------------
+      if (!mbar_wait(b_acc_full, j & 1)) { fail(); break; }
+      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+      if (!aborted()) {
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int h = (warp >> 2) & 1;          // token half (accumulator) this warp drains
+        const int cb = (warp >> 3) * (BN / 2);  // and which half of its columns
+        const int m = ti.m0 + h * MH + q * 32 + lane;  // token of this thread's TMEM lane
+        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * BN + cb);
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN / 2; c0 += 32) {
+          uint32_t v[32];
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+              "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+                "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+                "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+              : "r"(taddr + c0));
+          asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+          const int n = ti.n0 + cb + c0;  // first output column of this chunk
+          if (m < P.M && n < P.d_out) {
+            __nv_bfloat16* dst = P.y + (size_t)m * P.d_out + n;
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const __nv_bfloat162 b2 =
+                  __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              pk[i] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            // d_out is a multiple of 16: the last 32-column chunk may hold only 16
+            const int nq = (n + 32 <= P.d_out) ? 4 : 2;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (i < nq)
+                reinterpret_cast<uint4*>(dst)[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      }
+      asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+      mbar_arrive(b_acc_empty);  // the MMA warp may overwrite the accumulators
     }
   }
 
@@ -406,8 +486,9 @@ w4_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ C
       }
       mbar_wait(b_full_c + 8 * s, 0);
       mbar_wait(b_full_c + 8 * s, 1);
+      mbar_wait(b_empty + 8 * s, 0);
+      mbar_wait(b_empty + 8 * s, 1);
     }
-    mbar_wait(b_acc, 0);
   }
   __syncthreads();
   if (warp == kWarpTma) {
@@ -439,44 +520,79 @@ bool tc_supported(int M, int d_in, int d_out, const void* x) {
          ((size_t)d_in * 2) % 16 == 0;
 }
 
-cudaError_t launch_w4_tc(const uint16_t* x, bool x_f16, const uint32_t* qweight, const __half* scales,
-                         const __half* zeros, __nv_bfloat16* y, int M, int d_in, int d_out, int* status,
-                         cudaStream_t stream) {
+cudaError_t launch_w4_tc_batch(const TcLinear* lins, int count, bool x_f16, int* status, cudaStream_t stream) {
+  if (count < 1 || count > kTcMaxBatch) return cudaErrorInvalidValue;
   EncodeTiled enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
-  CUtensorMap map;
-  const cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)d_in * 2};
-  const cuuint32_t box[2] = {BK, BM};  // 64 fp16 (128 bytes) x 256 tokens
-  const cuuint32_t elem[2] = {1, 1};
-  CUresult r = enc(&map, x_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                   const_cast<uint16_t*>(x), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  CUtensorMap qmap;  // packed codes: uint32 [d_out][d_in / 8], one box = 8 words x 128 rows
-  {
-    const cuuint64_t qdims[2] = {(cuuint64_t)(d_in / 8), (cuuint64_t)d_out};
-    const cuuint64_t qstrides[1] = {(cuuint64_t)d_in / 2};
-    const cuuint32_t qbox[2] = {BK / 8, BN};
-    r = enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(qweight), qdims, qstrides, qbox, elem,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  // the linears with the longest K (slowest tiles) first, otherwise in call order
+  int order[kTcMaxBatch];
+  for (int i = 0; i < count; ++i) {
+    int j = i;
+    while (j > 0 && lins[order[j - 1]].d_in < lins[i].d_in) {
+      order[j] = order[j - 1];
+      --j;
+    }
+    order[j] = i;
   }
-  const dim3 grid((d_out + BN - 1) / BN, (M + BM - 1) / BM);
+  TcBatch b{};
+  int tiles = 0;
+  const cuuint32_t elem[2] = {1, 1};
+  for (int oi = 0; oi < count; ++oi) {
+    const TcLinear& L = lins[order[oi]];
+    if (!tc_supported(L.M, L.d_in, L.d_out, L.x)) return cudaErrorInvalidValue;
+    TcProblem& P = b.p[oi];
+    {  // activations [M][d_in]: box 64 columns x 256 tokens, 128-byte swizzle
+      const cuuint64_t dims[2] = {(cuuint64_t)L.d_in, (cuuint64_t)L.M};
+      const cuuint64_t strides[1] = {(cuuint64_t)L.d_in * 2};
+      const cuuint32_t box[2] = {BK, BM};
+      if (enc(&P.xmap, x_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<uint16_t*>(L.x), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
+    {  // packed codes uint32 [d_out][d_in / 8]: box 8 words x 256 rows, 32-byte swizzle
+      const cuuint64_t dims[2] = {(cuuint64_t)(L.d_in / 8), (cuuint64_t)L.d_out};
+      const cuuint64_t strides[1] = {(cuuint64_t)L.d_in / 2};
+      const cuuint32_t box[2] = {BK / 8, BN};
+      if (enc(&P.qmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(L.qweight), dims, strides, box,
+              elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
+    P.xraw = L.x;
+    P.sc = reinterpret_cast<const unsigned short*>(L.scales);
+    P.z = reinterpret_cast<const unsigned short*>(L.zeros);
+    P.y = L.y;
+    P.M = L.M;
+    P.d_in = L.d_in;
+    P.d_out = L.d_out;
+    P.n_tiles = (L.d_out + BN - 1) / BN;
+    P.tile_begin = tiles;
+    tiles += ((L.M + BM - 1) / BM) * P.n_tiles;
+  }
+  b.count = count;
+  b.total_tiles = tiles;
+  const int sms = device_sm_count();
+  const int grid = tiles < sms ? tiles : sms;
   cudaError_t e;
   if (x_f16) {
     e = cudaFuncSetAttribute(w4_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    w4_tc_kernel<true><<<grid, kThreadsTma, SMEM_BYTES, stream>>>(map, qmap, x, qweight, scales, zeros, y, M, d_in, d_out,
-                                                                  status);
+    w4_tc_kernel<true><<<grid, kThreadsTma, SMEM_BYTES, stream>>>(b, status);
   } else {
     e = cudaFuncSetAttribute(w4_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    w4_tc_kernel<false><<<grid, kThreadsConv, SMEM_BYTES, stream>>>(map, qmap, x, qweight, scales, zeros, y, M, d_in,
-                                                                    d_out, status);
+    w4_tc_kernel<false><<<grid, kThreadsConv, SMEM_BYTES, stream>>>(b, status);
   }
   return cudaPeekAtLastError();
+}
+
+cudaError_t launch_w4_tc(const uint16_t* x, bool x_f16, const uint32_t* qweight, const __half* scales,
+                         const __half* zeros, __nv_bfloat16* y, int M, int d_in, int d_out, int* status,
+                         cudaStream_t stream) {
+  const TcLinear L{x, qweight, scales, zeros, y, M, d_in, d_out};
+  return launch_w4_tc_batch(&L, 1, x_f16, status, stream);
 }
 
 }  // namespace paro

@@ -383,3 +383,27 @@ def test_stream_decode_matches_oracle_and_repeats_bit_exactly(shapes_m, rotate):
     assert paro.paro_get_device_status() == 0
     for f, d in zip(first, devs):
         assert torch.equal(f.view(torch.int16), d["y"].view(torch.int16))
+
+
+# ---------------------------------------------------------------- grouped tensor-core launch (batched, M >= 128)
+@pytest.mark.parametrize("shapes_m", [
+    # mixed K, ragged token counts and ragged output tails in one launch
+    [(512, 272, 128), (1536, 528, 300), (4096, 1024, 200)],
+    # more tiles than SMs: every CTA walks several tiles, the longest K first
+    [(4096, 14336, 640), (4096, 1024, 640), (14336, 512, 384)],
+])
+def test_batched_prefill_grouped_matches_oracle_and_single_calls(shapes_m):
+    probs, devs = _batch_case(shapes_m, 63)
+    layers = [paro.paro_linear(d["x"], *d["tables"], d["qw"], d["sc"], d["z"], d["y"]) for d in devs]
+    paro.paro_rotate_w4_linear_batched(layers)
+    torch.cuda.synchronize()
+    assert paro.paro_get_device_status() == 0
+    for i, (p, d) in enumerate(zip(probs, devs)):
+        got = host(d["y"])
+        assert np.isfinite(got).all(), p.name
+        rows = _sampled_rows(p.M, 24, 7 + i)
+        ref = oracle.rotate_w4_linear(p.x[rows], p.pairs, p.cos_t, p.sin_t, p.scale, *to_np_pack(d["qw"], d["sc"], d["z"]))
+        assert_linear_close(got[rows], ref)
+        # a tile's sum does not depend on the launch it ran in
+        single = paro.paro_rotate_w4_linear(d["x"], *d["tables"], d["qw"], d["sc"], d["z"])
+        assert torch.equal(single.view(torch.int16), d["y"].view(torch.int16))
