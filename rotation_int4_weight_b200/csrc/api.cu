@@ -452,7 +452,7 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     paro::RotBatch rb;
     int R = 1;
     e = paro::plan_rot_batch(rp, n, &rb, &R);
-    if (e == cudaSuccess) e = paro::launch_rot_batch(rb, R, true, status, s, true);
+    if (e == cudaSuccess) e = paro::launch_rot_batch(rb, R, true, status, s, true, true);
   } else {
     // many tokens (or tables the decode kernel cannot take): every transform, then
     // one persistent tensor-core launch over all linears it takes (their tiles

@@ -56,7 +56,7 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 
 template <int R, bool F16OUT>
 __global__ void __launch_bounds__(kRotThreads)
-rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_trigger) {
+rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_trigger, int pdl_wait) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ __align__(8) uint64_t bars[kMaxRing + 1];
   if (pdl_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -103,6 +103,10 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
     }
     if (P.scale && (reinterpret_cast<uintptr_t>(P.scale) & 15) == 0) bulk_prefetch_l2(P.scale, (size_t)4 * d);
   }
+  // launched as a programmatic dependent: the tables above may be fetched while
+  // the previous kernel finishes; the rows (which it may have written) and the
+  // output (which it may still read) wait for it to complete
+  if (pdl_wait) asm volatile("griddepcontrol.wait;\n" ::: "memory");
   // rows -> xs as fp32: each thread two adjacent channels of every row, the
   // loads of LB channel pairs issued before their stores so that their
   // latencies overlap
@@ -265,21 +269,30 @@ cudaError_t plan_rot_batch(const RotProblem* probs, int count, RotBatch* out, in
 }
 
 cudaError_t launch_rot_batch(const RotBatch& b, int R, bool f16_out, int* status, cudaStream_t stream,
-                             bool pdl_trigger) {
+                             bool pdl_trigger, bool pdl_wait) {
   size_t smem = 0;
   for (int i = 0; i < b.count; ++i) {
     const size_t s = rot_smem(b.p[i].d, R, b.p[i].ring);
     smem = s > smem ? s : smem;
   }
-  const int trig = pdl_trigger ? 1 : 0;
+  const int trig = pdl_trigger ? 1 : 0, wait = pdl_wait ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(b.total_ctas);
+  cfg.blockDim = dim3(kRotThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_wait ? 1 : 0;
   cudaError_t e;
 #define PARO_ROT_LAUNCH(r, f16)                                                                     \
   {                                                                                                 \
     auto k = rot_decode_kernel<r, f16>;                                                             \
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);            \
     if (e != cudaSuccess) return e;                                                                 \
-    k<<<b.total_ctas, kRotThreads, smem, stream>>>(b, status, trig);                                \
-    return cudaPeekAtLastError();                                                                   \
+    return cudaLaunchKernelEx(&cfg, k, b, status, trig, wait);                                      \
   }
   if (f16_out) {
     if (R == 4) PARO_ROT_LAUNCH(4, true) else if (R == 2) PARO_ROT_LAUNCH(2, true) else PARO_ROT_LAUNCH(1, true)

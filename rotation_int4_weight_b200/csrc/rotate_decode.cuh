@@ -31,7 +31,10 @@ struct RotBatch {
 // (d % 8 == 0 and 16-byte aligned tables, since stages are copied in 16-byte pieces).
 bool rot_decode_supported(int d, const void* pairs, const void* cos_t, const void* sin_t);
 cudaError_t plan_rot_batch(const RotProblem* probs, int count, RotBatch* out, int* R_out);
+// pdl_trigger: let the next kernel launch early; pdl_wait: launched as a
+// programmatic dependent, fetches its tables early and waits for the previous
+// kernel before it reads the rows or writes the output.
 cudaError_t launch_rot_batch(const RotBatch& b, int R, bool f16_out, int* status, cudaStream_t stream,
-                             bool pdl_trigger);
+                             bool pdl_trigger, bool pdl_wait = false);
 
 }  // namespace paro

@@ -272,6 +272,9 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, int* status, int pdl_wai
   __shared__ __align__(8) uint64_t bars[W * D];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  // a programmatic dependent (the next call's transform) may start its table
+  // fetches as SMs free up; it waits for this grid before touching its data
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   __shared__ Meta meta[kMaxBatch];
   if (threadIdx.x < b.count) {
     const StreamProblem& P = b.p[threadIdx.x];
