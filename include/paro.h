@@ -212,8 +212,11 @@ PARO_API size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int co
  * enqueued; the message of paro_last_error() names the failing index.  When no
  * linear has a transform (K == 0 and d_scale == NULL for all) and every M is
  * at most 64, only the INT4-linear launch runs, on the bf16 inputs, and
- * d_workspace may be NULL; with more tokens the inputs are first rounded to
- * fp16 into the workspace, as the transform does, for the tensor-core kernel.
+ * d_workspace may be NULL; with more tokens, one tensor-core launch rounds
+ * the bf16 inputs to fp16 itself when every linear has at least 128 tokens,
+ * else the inputs are first rounded to fp16 into the workspace, as the
+ * transform does.  With many tokens the INT4 linears of all layers run as one
+ * persistent tensor-core launch after the transforms.
  * The stream-K kernel's publication flags need no clearing: a flag holds the
  * id of the launch that wrote it, so one left by another launch, or never
  * written, is never taken for this launch's.  Two calls that may run at the

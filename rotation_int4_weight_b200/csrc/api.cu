@@ -448,6 +448,17 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
   }
   int* status = status_ptr();
   if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
+  if (!any_transform) {
+    // many tokens and no layer has a transform: when the tensor-core kernel takes
+    // every linear, one launch rounds the bf16 inputs to fp16 tiles itself
+    bool all_tc = true;
+    paro::TcLinear tl[PARO_MAX_BATCH];
+    for (int i = 0; i < n && all_tc; ++i) {
+      all_tc = rp[i].M >= kTensorCoreMinM && paro::tc_supported(rp[i].M, rp[i].d, gp[i].d_out, rp[i].x);
+      tl[i] = paro::TcLinear{rp[i].x, gp[i].qw, gp[i].sc, gp[i].z, gp[i].y, gp[i].M, gp[i].d_in, gp[i].d_out};
+    }
+    if (all_tc) return from_cuda(paro::launch_w4_tc_batch(tl, n, false, status, s), "batched w4 linear launch");
+  }
   if (decode_ok) {
     paro::RotBatch rb;
     int R = 1;

@@ -126,29 +126,44 @@ givens_cm_kernel(const void* __restrict__ in, void* __restrict__ out, int M, int
   if (K > 0) fetch(pr, cs, sn);
 
   // ---- load: two adjacent channels of every row per thread (a warp reads 128
-  // or 256 contiguous bytes of each row), stored as two channel vectors
+  // or 256 contiguous bytes of each row), stored as two channel vectors.  The
+  // loads of LB consecutive channel pairs are issued before their stores, so
+  // their DRAM latencies overlap.
+  constexpr int LB = MODE == kFoldF32 ? 2 : 4;
 #pragma unroll 1
-  for (int cp = tid; cp < half; cp += NTH) {
-    V v0, v1;
+  for (int cp0 = tid; cp0 < half; cp0 += LB * NTH) {
+    float2 f[LB][R];
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      float f0 = 0.f, f1 = 0.f;
-      if (r < nrows) {
-        const size_t off = (size_t)(row0 + r) * d + 2 * cp;
-        if constexpr (MODE == kFoldF32) {
-          const float2 f = __ldg(reinterpret_cast<const float2*>(static_cast<const float*>(in) + off));
-          f0 = f.x; f1 = f.y;
-        } else {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
-              static_cast<const __nv_bfloat16*>(in) + off));
-          f0 = f.x; f1 = f.y;
+    for (int q = 0; q < LB; ++q) {
+      const int cp = cp0 + q * NTH;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        f[q][r] = make_float2(0.f, 0.f);
+        if (cp < half && r < nrows) {
+          const size_t off = (size_t)(row0 + r) * d + 2 * cp;
+          if constexpr (MODE == kFoldF32) {
+            f[q][r] = __ldg(reinterpret_cast<const float2*>(static_cast<const float*>(in) + off));
+          } else {
+            f[q][r] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
+                static_cast<const __nv_bfloat16*>(in) + off));
+          }
         }
       }
-      vset(v0, r, f0);
-      vset(v1, r, f1);
     }
-    xs[2 * cp] = v0;
-    xs[2 * cp + 1] = v1;
+#pragma unroll
+    for (int q = 0; q < LB; ++q) {
+      const int cp = cp0 + q * NTH;
+      if (cp < half) {
+        V v0, v1;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          vset(v0, r, f[q][r].x);
+          vset(v1, r, f[q][r].y);
+        }
+        xs[2 * cp] = v0;
+        xs[2 * cp + 1] = v1;
+      }
+    }
   }
   __syncthreads();
 

@@ -9,10 +9,10 @@
 //   warp 16, lane 0 TMA: the stage's packed codes (256 rows x 32 bytes, 32-byte
 //                   swizzle), completing on full_c[s], and the 256 x 64 fp16
 //                   activation tile (128-byte swizzle), completing on
-//                   full_a[s]; with bf16 activations warps 18-25 instead load
-//                   each token row, round it to fp16 and store it in the same
-//                   swizzled layout (fp16 operands keep the product error an
-//                   order of magnitude below bf16 ones);
+//                   full_a[s]; bf16 activations land the same way (on
+//                   full_raw[s]) and warps 18-25 round them to fp16 in place
+//                   (fp16 operands keep the product error an order of
+//                   magnitude below bf16 ones);
 //   warps 0-15      dequantisation: thread (row t, half h) reads its 16 bytes
 //                   of the stage's codes from shared memory, holds its row's
 //                   scale and zero bits (loaded once per 128-column group, a
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(XF16 ? kThreadsTma : kThreadsConv, 1)
 w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
   constexpr bool F16 = true;  // tensor-core operands are fp16 in both variants
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  __shared__ __align__(8) uint64_t bars[4 * kStages + 2];
+  __shared__ __align__(8) uint64_t bars[5 * kStages + 2];
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
   __shared__ TcMeta meta[kTcMaxBatch];
@@ -198,6 +198,7 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
   const uint32_t b_full_c = smem_u32(&bars[3 * kStages]);    // codes of a stage landed
   const uint32_t b_acc_full = smem_u32(&bars[4 * kStages]);  // a tile's accumulator is complete
   const uint32_t b_acc_empty = smem_u32(&bars[4 * kStages + 1]);  // ... and has been read out
+  const uint32_t b_full_raw = smem_u32(&bars[4 * kStages + 2]);   // bf16 activation tile landed
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = b.total_tiles, count = b.count;
@@ -206,7 +207,7 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
     const TcProblem& P = b.p[threadIdx.x];
     meta[threadIdx.x] = TcMeta{P.xraw, P.sc, P.z, P.y, P.M, P.d_in, P.d_out, P.n_tiles, P.tile_begin};
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&P.qmap)) : "memory");
-    if (XF16) asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&P.xmap)) : "memory");
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&P.xmap)) : "memory");
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -214,6 +215,7 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
       mbar_init(b_full_b + 8 * s, kDqWarps * 32);
       mbar_init(b_empty + 8 * s, 1);
       mbar_init(b_full_c + 8 * s, 1);
+      mbar_init(b_full_raw + 8 * s, 1);
     }
     mbar_init(b_acc_full, 1);
     mbar_init(b_acc_empty, kDqWarps * 32);
@@ -238,9 +240,12 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
   auto aborted = [&]() { return *(volatile int*)&abort_flag != 0; };
 
   if (warp >= kWarpConv) {
-    // ---------------- bf16 activations -> fp16 tiles (bf16 input only) ---------------
+    // ---------------- bf16 activations -> fp16, in place (bf16 input only) -----------
+    // The TMA put the stage's bf16 tile in the A slot in the same swizzled layout
+    // the tensor core reads; every 16-byte chunk holds 8 consecutive columns of
+    // one token, so converting each chunk where it lies keeps the layout.
     if constexpr (!XF16) {
-      const int t = threadIdx.x - kWarpConv * 32;  // row of the 256-token tile
+      const int t = threadIdx.x - kWarpConv * 32;  // 0 .. 255
       int it = 0;
       bool stop = false;
 #pragma unroll 1
@@ -248,51 +253,34 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
         const int T = tile_of(j, total);
         if (T < 0) break;
         const TileInfo ti = tile_info(meta, count, T);
-        const TcMeta& P = meta[ti.pi];
-        const int m = ti.m0 + t;
-        const bool okm = m < P.M;
-        const uint16_t* xr = P.xraw + (size_t)(okm ? m : 0) * P.d_in;
-        constexpr int PX = 2;  // steps of loads in flight
-        uint4 xq[PX][8];
-        auto load_x = [&](int k, uint4 (&v)[8]) {
-          if (k < ti.nk && okm) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) v[c] = __ldg(reinterpret_cast<const uint4*>(xr + k * BK + c * 8));
-          }
-        };
-#pragma unroll
-        for (int q = 0; q < PX - 1; ++q) load_x(q, xq[q]);
 #pragma unroll 1
-        for (int kb = 0; kb < ti.nk && !stop; kb += PX) {
+        for (int k = 0; k < ti.nk; ++k, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(b_full_raw + 8 * s, (it / kStages) & 1)) { fail(); stop = true; break; }
+          if (aborted()) { stop = true; break; }
+          const uint32_t a0 = s_base + (uint32_t)(s * STAGE_BYTES);
+          uint32_t v[A_BYTES / 16 / (BM)][4];  // the chunks of this thread
 #pragma unroll
-          for (int q = 0; q < PX; ++q) {
-            const int k = kb + q;
-            if (k >= ti.nk) break;
-            load_x(k + PX - 1, xq[(q + PX - 1) % PX]);
-            const int s = it % kStages;
-            if (it >= kStages && !mbar_wait(b_empty + 8 * s, ((it / kStages) - 1) & 1)) fail();
-            if (aborted()) { stop = true; break; }
-            unsigned char* rowp = smem + s * STAGE_BYTES + t * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              uint4 o = make_uint4(0u, 0u, 0u, 0u);
-              if (okm) {
-                const uint32_t in[4] = {xq[q][c].x, xq[q][c].y, xq[q][c].z, xq[q][c].w};
-                uint32_t out[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[e]));
-                  const __half2 h = __floats2half2_rn(f.x, f.y);
-                  out[e] = *reinterpret_cast<const uint32_t*>(&h);
-                }
-                o = make_uint4(out[0], out[1], out[2], out[3]);
-              }
-              *reinterpret_cast<uint4*>(rowp + ((c ^ (t & 7)) << 4)) = o;
-            }
-            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-            mbar_arrive(b_full_a + 8 * s);
-            ++it;
+          for (int q = 0; q < A_BYTES / 16 / BM; ++q) {
+            const uint32_t a = a0 + (uint32_t)((t + q * BM) * 16);
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                         : "=r"(v[q][0]), "=r"(v[q][1]), "=r"(v[q][2]), "=r"(v[q][3]) : "r"(a) : "memory");
           }
+#pragma unroll
+          for (int q = 0; q < A_BYTES / 16 / BM; ++q) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v[q][e]));
+              const __half2 h = __floats2half2_rn(f.x, f.y);
+              v[q][e] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            const uint32_t a = a0 + (uint32_t)((t + q * BM) * 16);
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(a), "r"(v[q][0]), "r"(v[q][1]), "r"(v[q][2]),
+                         "r"(v[q][3])
+                         : "memory");
+          }
+          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+          mbar_arrive(b_full_a + 8 * s);
         }
       }
     }
@@ -314,10 +302,11 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
           if (aborted()) { stop = true; break; }
           mbar_expect_tx(b_full_c + 8 * s, C_BYTES);
           tma_load_2d(s_base + s * STAGE_BYTES + A_BYTES + B_BYTES, &P.qmap, k * (BK / 8), ti.n0, b_full_c + 8 * s);
-          if (XF16) {
-            mbar_expect_tx(b_full_a + 8 * s, A_BYTES);
-            tma_load_2d(s_base + s * STAGE_BYTES, &P.xmap, k * BK, ti.m0, b_full_a + 8 * s);
-          }
+          // fp16 activations complete the stage's A tile; bf16 ones land first and
+          // are converted in place by the conversion warps
+          const uint32_t bar_a = XF16 ? b_full_a + 8 * s : b_full_raw + 8 * s;
+          mbar_expect_tx(bar_a, A_BYTES);
+          tma_load_2d(s_base + s * STAGE_BYTES, &P.xmap, k * BK, ti.m0, bar_a);
         }
       }
     }
@@ -480,10 +469,9 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
   if (abort_flag && threadIdx.x == 0) {
     // let any copies and MMAs still in flight land before the memory goes away
     for (int s = 0; s < kStages; ++s) {
-      if (XF16) {
-        mbar_wait(b_full_a + 8 * s, 0);
-        mbar_wait(b_full_a + 8 * s, 1);
-      }
+      const uint32_t bar_a = XF16 ? b_full_a : b_full_raw;
+      mbar_wait(bar_a + 8 * s, 0);
+      mbar_wait(bar_a + 8 * s, 1);
       mbar_wait(b_full_c + 8 * s, 0);
       mbar_wait(b_full_c + 8 * s, 1);
       mbar_wait(b_empty + 8 * s, 0);

@@ -407,3 +407,20 @@ def test_batched_prefill_grouped_matches_oracle_and_single_calls(shapes_m):
         # a tile's sum does not depend on the launch it ran in
         single = paro.paro_rotate_w4_linear(d["x"], *d["tables"], d["qw"], d["sc"], d["z"])
         assert torch.equal(single.view(torch.int16), d["y"].view(torch.int16))
+
+
+def test_batched_prefill_plain_bf16_grouped():
+    """No transforms, every linear on the tensor cores: one launch reads the bf16 inputs."""
+    shapes_m = [(4096, 1040, 256), (1536, 528, 300), (512, 256, 128)]
+    probs, devs, layers = _stream_case(shapes_m, 64, rotate=False)
+    paro.paro_rotate_w4_linear_batched(layers)
+    torch.cuda.synchronize()
+    assert paro.paro_get_device_status() == 0
+    for i, (p, d) in enumerate(zip(probs, devs)):
+        got = host(d["y"])
+        assert np.isfinite(got).all(), p.name
+        rows = _sampled_rows(p.M, 24, 11 + i)
+        ref = oracle.w4_linear(p.x[rows], *to_np_pack(d["qw"], d["sc"], d["z"]))
+        assert_linear_close(got[rows], ref)
+        single = paro.paro_w4_linear(d["x"], d["qw"], d["sc"], d["z"])
+        assert torch.equal(single.view(torch.int16), d["y"].view(torch.int16))
