@@ -21,6 +21,9 @@ namespace paro {
 namespace {
 
 constexpr int kRotThreads = 1024;
+// warp 31 fetches the stage tables; the other 31 warps rotate
+constexpr int kProducer = kRotThreads - 32;
+constexpr int kCompute = kRotThreads - 32;
 constexpr int kMaxRing = 8;
 constexpr size_t kRotSmemBudget = 227 * 1024 - 256;
 
@@ -37,10 +40,19 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
       : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
   return ok != 0;
 }
+// non-blocking test of the same phase (cheaper than try_wait when the phase has
+// long completed, the usual case for the stages after the first)
+__device__ __forceinline__ bool mbar_done(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
 // Waits for phase `parity` of an mbarrier; gives up after about a second of
 // SM clock (then returns false and the caller reports PARO_ERR_TIMEOUT).
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
-  if (mbar_test(bar, parity)) return true;
+  if (mbar_done(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_test(bar, parity))
     if (clock64() - t0 > (1LL << 31)) return false;
@@ -54,7 +66,9 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
-template <int R, bool F16OUT>
+// R token rows per CTA; UP pairs per thread and round of a stage (0: the
+// default for R, 4 for one or two rows and 2 for four)
+template <int R, bool F16OUT, int UP>
 __global__ void __launch_bounds__(kRotThreads)
 rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_trigger, int pdl_wait) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -89,7 +103,7 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
       bulk_g2s(base + 4u * d, P.sin_t + (size_t)k * half, 2u * d, bar);
     }
   };
-  if (tid == 0) {
+  if (tid == kProducer) {
     for (int k = 0; k < kMaxRing; ++k) mbar_init(s_bar + 8u * k, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     for (int k = 0; k < ring; ++k) issue_stage(k);
@@ -133,25 +147,32 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
       }
     }
   }
-  __syncthreads();  // rows staged; barriers initialised before anyone waits on them
+  // The producer waits for each stage's table before the CTA barrier that
+  // starts the stage, so that the barrier also tells the other threads that
+  // the table has landed; it refills a slot as soon as the barrier after its
+  // stage has passed.  With one slot the next stage can only be requested once
+  // the current one is done, which costs a second barrier per stage.
+  bool ok = true;
+  if (tid == kProducer && K > 0) ok = mbar_wait_bounded(s_bar, 0u);
+  int failed = __syncthreads_or(!ok);  // also: rows staged
+  int issued = ring < K ? ring : K;    // stages requested so far (producer)
 
   // K stages.  The pairs of a stage are disjoint, so the loads of a batch of
   // pairs may all be issued before any of its stores.
-  constexpr int U = R == 4 ? 2 : 4;
+  constexpr int U = UP > 0 ? UP : (R == 4 ? 2 : 4);
 #pragma unroll 1
-  for (int k = 0; k < K; ++k) {
-    const bool arrived = mbar_wait_bounded(s_bar + 8u * (k % ring), (uint32_t)((k / ring) & 1));
-    if (arrived) {
+  for (int k = 0; k < K && !failed; ++k) {
+    if (tid < kCompute) {
       const unsigned char* st = tab + (size_t)(k % ring) * stage_bytes;
       const uint32_t* pk = reinterpret_cast<const uint32_t*>(st);
       const float* ck = reinterpret_cast<const float*>(st + 2 * d);
       const float* sk = reinterpret_cast<const float*>(st + 4 * d);
-      for (int t0 = tid; t0 < half; t0 += U * kRotThreads) {
+      for (int t0 = tid; t0 < half; t0 += U * kCompute) {
         int ii[U], jj[U];
         float c[U], sn[U], a[U][R], b[U][R];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-          const int t = t0 + u * kRotThreads;
+          const int t = t0 + u * kCompute;
           ii[u] = -1;
           if (t < half) {
             const uint32_t pr = pk[t];
@@ -185,18 +206,34 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
             }
           }
       }
+    } else if (tid == kProducer && ring > 1) {
+      // stage k - 1's slot is free since the barrier that started this stage
+      if (k >= 1 && k - 1 + ring < K) {
+        issue_stage(k - 1 + ring);
+        ++issued;
+      }
+      if (k + 1 < K) ok = mbar_wait_bounded(s_bar + 8u * ((k + 1) % ring), (uint32_t)(((k + 1) / ring) & 1));
     }
-    if (__syncthreads_or(!arrived)) {
-      // a stage never arrived: report, let this CTA's copies in flight land
-      // (each wait bounded again), then leave
+    failed = __syncthreads_or(!ok);
+    if (ring == 1 && k + 1 < K && !failed) {
+      if (tid == kProducer) {
+        issue_stage(k + 1);
+        ++issued;
+        ok = mbar_wait_bounded(s_bar, (uint32_t)((k + 1) & 1));
+      }
+      failed = __syncthreads_or(!ok);
+    }
+  }
+  if (failed) {
+    // a stage never arrived: report, let the latest copy of every slot land
+    // (each wait bounded again), then leave
+    if (tid == kProducer) {
       report_status(status, kStatusTimeout);
-      if (tid == 0)
-        for (int q = k; q < K && q < k + ring; ++q)
-          mbar_wait_bounded(s_bar + 8u * (q % ring), (uint32_t)((q / ring) & 1));
-      __syncthreads();
-      return;
+      for (int q = issued > ring ? issued - ring : 0; q < issued; ++q)
+        mbar_wait_bounded(s_bar + 8u * (q % ring), (uint32_t)((q / ring) & 1));
     }
-    if (tid == 0) issue_stage(k + ring);  // refill the slot this stage used
+    __syncthreads();
+    return;
   }
 
   // channel scale and store: the scales of LB channel pairs are loaded (from
@@ -287,17 +324,41 @@ cudaError_t launch_rot_batch(const RotBatch& b, int R, bool f16_out, int* status
   cfg.attrs = attr;
   cfg.numAttrs = pdl_wait ? 1 : 0;
   cudaError_t e;
-#define PARO_ROT_LAUNCH(r, f16)                                                                     \
+#define PARO_ROT_LAUNCH(r, f16, up)                                                                 \
   {                                                                                                 \
-    auto k = rot_decode_kernel<r, f16>;                                                             \
+    auto k = rot_decode_kernel<r, f16, up>;                                                         \
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);            \
     if (e != cudaSuccess) return e;                                                                 \
     return cudaLaunchKernelEx(&cfg, k, b, status, trig, wait);                                      \
   }
+  // enough pairs per thread that a stage of the widest problem is one round of
+  // loads and stores, within the registers each row count leaves (one row: up
+  // to 8; two rows: 5; four rows: 3)
+  int max_half = 0;
+  for (int i = 0; i < b.count; ++i) max_half = b.p[i].d / 2 > max_half ? b.p[i].d / 2 : max_half;
+  const int rounds = (max_half + kCompute - 1) / kCompute;  // pairs per thread in one round
   if (f16_out) {
-    if (R == 4) PARO_ROT_LAUNCH(4, true) else if (R == 2) PARO_ROT_LAUNCH(2, true) else PARO_ROT_LAUNCH(1, true)
+    if (R == 4) {
+      if (rounds == 3) PARO_ROT_LAUNCH(4, true, 3) else PARO_ROT_LAUNCH(4, true, 0)
+    } else if (R == 2) {
+      if (rounds == 5) PARO_ROT_LAUNCH(2, true, 5) else PARO_ROT_LAUNCH(2, true, 0)
+    } else {
+      if (rounds == 5) PARO_ROT_LAUNCH(1, true, 5)
+      else if (rounds == 6 || rounds == 7) PARO_ROT_LAUNCH(1, true, 7)
+      else if (rounds >= 8) PARO_ROT_LAUNCH(1, true, 8)
+      else PARO_ROT_LAUNCH(1, true, 0)
+    }
   } else {
-    if (R == 4) PARO_ROT_LAUNCH(4, false) else if (R == 2) PARO_ROT_LAUNCH(2, false) else PARO_ROT_LAUNCH(1, false)
+    if (R == 4) {
+      if (rounds == 3) PARO_ROT_LAUNCH(4, false, 3) else PARO_ROT_LAUNCH(4, false, 0)
+    } else if (R == 2) {
+      if (rounds == 5) PARO_ROT_LAUNCH(2, false, 5) else PARO_ROT_LAUNCH(2, false, 0)
+    } else {
+      if (rounds == 5) PARO_ROT_LAUNCH(1, false, 5)
+      else if (rounds == 6 || rounds == 7) PARO_ROT_LAUNCH(1, false, 7)
+      else if (rounds >= 8) PARO_ROT_LAUNCH(1, false, 8)
+      else PARO_ROT_LAUNCH(1, false, 0)
+    }
   }
 #undef PARO_ROT_LAUNCH
 }
