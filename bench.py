@@ -37,6 +37,33 @@ sys.path.insert(0, ROOT)
 from synth import LAYER_SHAPES, device_weights, linear_problem  # noqa: E402
 
 METRIC = "rot+W4 linear: decode HBM GB/s (% peak), prefill TFLOP/s, rotation overhead %"
+
+# DRAM bytes (read + write) per launch of the kernel the roofline times, from
+# one ncu capture of `bench.py --profile --variants batched_plain --config N`
+# (metrics dram__bytes_read.sum, dram__bytes_write.sum; first of three launches
+# after four skipped; profiles/int4_linear_traffic.md), with the sha256 prefix
+# of the kernel's sources at capture time: once the sources change, the figure
+# no longer describes the kernel and the bench reports null.
+TRAFFIC = {
+    1: {"bytes": 24962048, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "61544feaebafd768"},
+    2: {"bytes": 128262144 + 4700160, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "61544feaebafd768"},
+    3: {"bytes": 346587136 + 137527040, "src": ("w4_tc.cu", "w4_tc.cuh"), "sha": "a093d18620409e5a"},
+    4: {"bytes": 25537536, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "61544feaebafd768"},
+}
+
+
+def measured_traffic(config, M):
+    """The captured DRAM bytes per launch of this config's timed kernel, or None
+    when the workload is not the captured one or the kernel changed since."""
+    import hashlib
+    t = TRAFFIC.get(config)
+    if t is None or M is not None:
+        return None
+    h = hashlib.sha256()
+    for f in t["src"]:
+        with open(os.path.join(ROOT, "rotation_int4_weight_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return t["bytes"] if h.hexdigest()[:16] == t["sha"] else None
 K_STAGES = 8
 GROUP = 128
 PREFILL_M = 512                          # from this many tokens on the metric is TFLOP/s
@@ -543,6 +570,10 @@ def main():
     # one launch per batched call when that variant ran, else one per linear)
     w4_ms = results.get("batched_plain", plain_ms)
     w4_gbs = bytes_of("plain") / (w4_ms * 1e-3) / 1e9 if w4_ms else None
+    # launches of the timed kernel per step (one per batched call), for the
+    # per-launch figures next to the captured traffic
+    w4_launches = units[0].launches("batched_plain") if "batched_plain" in results else len(step_lins)
+    traffic = measured_traffic(args.config, args.M)
     rot_gbs = bytes_of("rotate") / (results["rotate"] * 1e-3) / 1e9 if "rotate" in results else None
     prefill = M >= PREFILL_M
 
@@ -564,7 +595,8 @@ def main():
         },
         "roofline": {
             "bound": "hbm", "achieved": round(w4_gbs, 1) if w4_gbs else None, "peak": hbm, "unit": "GB/s",
-            "frac": round(w4_gbs / hbm, 4) if w4_gbs else None, "traffic": None,
+            "frac": round(w4_gbs / hbm, 4) if w4_gbs else None, "traffic": traffic,
+            "algorithmic_bytes_per_launch": int(bytes_of("plain") / w4_launches),
             "kernel": ("w4_stream_kernel" if M <= 16 else "w4_gemv_kernel")
                       + " (INT4 linear; one launch per batched call of a step's linears, timed alone "
                         "with plain weights), algorithmic bytes / device time",
@@ -590,7 +622,8 @@ def main():
     if prefill:
         out["roofline"] = {"bound": "tensor", "achieved": round(flops_step / (w4_ms * 1e-3) / 1e12, 2),
                            "peak": bf16, "unit": "TFLOP/s",
-                           "frac": round(flops_step / (w4_ms * 1e-3) / 1e12 / bf16, 4), "traffic": None,
+                           "frac": round(flops_step / (w4_ms * 1e-3) / 1e12 / bf16, 4), "traffic": traffic,
+                           "algorithmic_bytes_per_launch": int(bytes_of("plain") / w4_launches),
                            "kernel": "INT4 linear, 2*M*d_in*d_out / device time",
                            "peak_kind": f"{peak_kind} bf16 dense (f16 operands: same nominal rate)"}
     if rank == 0 and not args.no_cpu:
