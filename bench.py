@@ -40,15 +40,15 @@ METRIC = "rot+W4 linear: decode HBM GB/s (% peak), prefill TFLOP/s, rotation ove
 
 # DRAM bytes (read + write) per launch of the kernel the roofline times, from
 # one ncu capture of `bench.py --profile --variants batched_plain --config N`
-# (metrics dram__bytes_read.sum, dram__bytes_write.sum; first of three launches
-# after four skipped; profiles/int4_linear_traffic.md), with the sha256 prefix
+# (metrics dram__bytes_read.sum, dram__bytes_write.sum; the first launch after
+# four skipped; profiles/int4_linear_traffic.md), with the sha256 prefix
 # of the kernel's sources at capture time: once the sources change, the figure
 # no longer describes the kernel and the bench reports null.
 TRAFFIC = {
-    1: {"bytes": 24966400, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "68319bfbe7923afb"},
-    2: {"bytes": 132598784 + 3795200, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "68319bfbe7923afb"},
+    1: {"bytes": 24966656, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "9c1800dd14202664"},
+    2: {"bytes": 132635648 + 5437952, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "9c1800dd14202664"},
     3: {"bytes": 346587136 + 137527040, "src": ("w4_tc.cu", "w4_tc.cuh"), "sha": "a093d18620409e5a"},
-    4: {"bytes": 25537536, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "68319bfbe7923afb"},
+    4: {"bytes": 25538048, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "9c1800dd14202664"},
 }
 
 
@@ -214,7 +214,9 @@ class Unit:
         if variant == "batched_plain":
             return len(self.calls)
         if variant.startswith("batched"):
-            return 2 * len(self.calls)
+            # one token per linear: the transforms run inside the INT4 kernel (one
+            # launch per call); otherwise a transform launch and an INT4 launch
+            return (1 if all(l.M == 1 for l in self.lins) else 2) * len(self.calls)
         return LAUNCHES[variant] * len(self.lins)
 
 

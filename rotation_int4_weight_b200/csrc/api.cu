@@ -409,7 +409,7 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
   for (int i = 0; i < n && use_stream; ++i)
     use_stream = paro::stream_supported(gp[i].M, gp[i].d_in, gp[i].d_out, any_transform ? gp[i].x : rp[i].x,
                                         gp[i].qw);
-  auto launch_stream = [&](bool x_f16, int* st, bool pdl) -> cudaError_t {
+  auto plan_stream = [&](bool x_f16, int reserved, paro::StreamBatch* sb, int* nt) -> cudaError_t {
     const uint16_t* xs[PARO_MAX_BATCH];
     const uint32_t* qs[PARO_MAX_BATCH];
     const __half *ss[PARO_MAX_BATCH], *zs[PARO_MAX_BATCH];
@@ -425,10 +425,13 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
       dis[i] = gp[i].d_in;
       dos[i] = gp[i].d_out;
     }
+    return paro::plan_stream_batch(xs, qs, ss, zs, ys, Ms, dis, dos, n, x_f16,
+                                   static_cast<char*>(d_workspace) + xt_bytes, sb, nt, reserved);
+  };
+  auto launch_stream = [&](bool x_f16, int* st, bool pdl) -> cudaError_t {
     paro::StreamBatch sb;
     int nt = 1;
-    cudaError_t err = paro::plan_stream_batch(xs, qs, ss, zs, ys, Ms, dis, dos, n, x_f16,
-                                              static_cast<char*>(d_workspace) + xt_bytes, &sb, &nt);
+    cudaError_t err = plan_stream(x_f16, 0, &sb, &nt);
     if (err != cudaSuccess) return err;
     return paro::launch_stream_batch(sb, nt, x_f16, st, s, pdl);
   };
@@ -458,6 +461,17 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
       tl[i] = paro::TcLinear{rp[i].x, gp[i].qw, gp[i].sc, gp[i].z, gp[i].y, gp[i].M, gp[i].d_in, gp[i].d_out};
     }
     if (all_tc) return from_cuda(paro::launch_w4_tc_batch(tl, n, false, status, s), "batched w4 linear launch");
+  }
+  if (decode_ok && use_stream && paro::fused_supported(rp, n)) {
+    // one token per linear: the transforms run in the INT4 kernel's first CTAs
+    // (one per linear) and each linear's arithmetic waits only for its own x~
+    paro::RotBatch rb;
+    paro::StreamBatch sb;
+    int nt = 1;
+    e = paro::plan_fused_rot(rp, n, &rb);
+    if (e == cudaSuccess) e = plan_stream(true, rb.count, &sb, &nt);
+    if (e == cudaSuccess) e = paro::launch_fused_batch(sb, rb, status, s, true);
+    return from_cuda(e, "batched fused launch");
   }
   if (decode_ok) {
     paro::RotBatch rb;

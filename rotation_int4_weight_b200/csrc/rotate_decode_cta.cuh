@@ -1,0 +1,265 @@
+// One CTA of the few-token activation transform x~ = diag(1/s) R_K ... R_1 x
+// (page "ParoQuant: pairwise rotations that survive deployment", section "A
+// rotation small enough to execute": disjoint channel pairs per stage, each
+// rotated by x_i' = c x_i + s x_j, x_j' = -s x_i + c x_j; channel scale last),
+// shared by the transform kernel (rotate_decode.cu) and the decode INT4 linear
+// that runs the transform in its own first CTAs (w4_stream.cu).
+//
+// The CTA stages its R rows as fp32 planes (channel c in bank c % 32 for every
+// row).  Its last warp streams the stage tables (pairs, cos, sin: 12 bytes a
+// pair) by bulk copies through a ring of mbarrier slots, L2-prefetches the
+// stages beyond the ring, and waits for each stage's table before the CTA
+// barrier that starts the stage, so the barrier also tells the other warps that
+// the table has landed; they rotate the pairs, U per thread and round, loads
+// before stores.  Waits are bounded: a stage that never lands is reported as
+// PARO_ERR_TIMEOUT and the CTA returns false without writing.
+#pragma once
+
+#include "paro_internal.cuh"
+#include "rotate_decode.cuh"
+
+namespace paro {
+namespace rotdec {
+
+constexpr int kRotMaxRing = 8;
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+// non-blocking test of the same phase (cheaper than try_wait when the phase has
+// long completed, the usual case for the stages after the first)
+__device__ __forceinline__ bool mbar_done(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Waits for phase `parity` of an mbarrier; gives up after about a second of
+// SM clock (then returns false and the caller reports PARO_ERR_TIMEOUT).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_done(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_test(bar, parity))
+    if (clock64() - t0 > (1LL << 31)) return false;
+  return true;
+}
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, size_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"((uint32_t)bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+
+// Transforms rows row0 .. row0 + R - 1 of problem P with NTHR threads; smem
+// holds d R 4 + ring 6 d bytes (16-byte aligned), bars kRotMaxRing mbarriers.
+// Returns true when the rows were written (uniform over the CTA).
+template <int R, bool F16OUT, int U, int NTHR>
+__device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, unsigned char* smem, uint64_t* bars,
+                                               int* status, bool pdl_wait) {
+  constexpr int kProd = NTHR - 32;  // the table-fetching thread (lane 0 of the last warp)
+  constexpr int kComp = NTHR - 32;  // rotating threads
+  const int d = P.d, K = P.K, half = d >> 1, ring = P.ring;
+  const int nrows = min(R, P.M - row0);
+  const int tid = threadIdx.x;
+
+  // shared memory: xs [R][d] fp32 (one plane per row: channel c in bank c % 32) |
+  // ring [ring][6d] of stage tables
+  float* xs = reinterpret_cast<float*>(smem);
+  unsigned char* tab = reinterpret_cast<unsigned char*>(xs + (size_t)d * R);
+  const size_t stage_bytes = (size_t)6 * d;  // pairs | cos | sin
+  const uint32_t s_tab = static_cast<uint32_t>(__cvta_generic_to_shared(tab));
+  const uint32_t s_bar = static_cast<uint32_t>(__cvta_generic_to_shared(bars));
+
+  // one thread requests whole stages with bulk copies (three per stage); the
+  // stage's mbarrier completes when all 6d bytes have landed
+  auto issue_stage = [&](int k) {
+    if (k < K) {
+      const int slot = k % ring;
+      const uint32_t base = s_tab + (uint32_t)(slot * stage_bytes), bar = s_bar + 8u * slot;
+      mbar_expect_tx(bar, (uint32_t)stage_bytes);
+      bulk_g2s(base, P.pairs + (size_t)k * half, 2u * d, bar);
+      bulk_g2s(base + 2u * d, P.cos_t + (size_t)k * half, 2u * d, bar);
+      bulk_g2s(base + 4u * d, P.sin_t + (size_t)k * half, 2u * d, bar);
+    }
+  };
+  if (tid == kProd) {
+    for (int k = 0; k < kRotMaxRing; ++k) mbar_init(s_bar + 8u * k, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    for (int k = 0; k < ring; ++k) issue_stage(k);
+    // then the stages beyond the ring go to L2, so that their copies into the
+    // ring later wait for L2 rather than HBM
+    if (K > ring) {
+      const size_t off = (size_t)ring * half, bytes = (size_t)(K - ring) * 2 * d;
+      bulk_prefetch_l2(P.pairs + off, bytes);
+      bulk_prefetch_l2(P.cos_t + off, bytes);
+      bulk_prefetch_l2(P.sin_t + off, bytes);
+    }
+    if (P.scale && (reinterpret_cast<uintptr_t>(P.scale) & 15) == 0) bulk_prefetch_l2(P.scale, (size_t)4 * d);
+  }
+  // launched as a programmatic dependent: the tables above may be fetched while
+  // the previous kernel finishes; the rows (which it may have written) and the
+  // output (which it may still read) wait for it to complete
+  if (pdl_wait) asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  // rows -> xs as fp32: each thread two adjacent channels of every row, the
+  // loads of LB channel pairs issued before their stores so that their
+  // latencies overlap
+  constexpr int LB = R == 4 ? 2 : (R == 2 ? 4 : 8);
+#pragma unroll 1
+  for (int cp0 = tid; cp0 < half; cp0 += LB * NTHR) {
+    __nv_bfloat162 v[LB][R];
+#pragma unroll
+    for (int q = 0; q < LB; ++q)
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int cp = cp0 + q * NTHR;
+        v[q][r] = __floats2bfloat162_rn(0.f, 0.f);
+        if (cp < half && r < nrows)
+          v[q][r] = *reinterpret_cast<const __nv_bfloat162*>(P.x + (size_t)(row0 + r) * d + 2 * cp);
+      }
+#pragma unroll
+    for (int q = 0; q < LB; ++q) {
+      const int cp = cp0 + q * NTHR;
+      if (cp < half) {
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          *reinterpret_cast<float2*>(xs + (size_t)r * d + 2 * cp) = __bfloat1622float2(v[q][r]);
+      }
+    }
+  }
+  // The producer waits for each stage's table before the CTA barrier that
+  // starts the stage, so that the barrier also tells the other threads that
+  // the table has landed; it refills a slot as soon as the barrier after its
+  // stage has passed.  With one slot the next stage can only be requested once
+  // the current one is done, which costs a second barrier per stage.
+  bool ok = true;
+  if (tid == kProd && K > 0) ok = mbar_wait_bounded(s_bar, 0u);
+  int failed = __syncthreads_or(!ok);  // also: rows staged
+  int issued = ring < K ? ring : K;    // stages requested so far (producer)
+
+  // K stages.  The pairs of a stage are disjoint, so the loads of a batch of
+  // pairs may all be issued before any of its stores.
+#pragma unroll 1
+  for (int k = 0; k < K && !failed; ++k) {
+    if (tid < kComp) {
+      const unsigned char* st = tab + (size_t)(k % ring) * stage_bytes;
+      const uint32_t* pk = reinterpret_cast<const uint32_t*>(st);
+      const float* ck = reinterpret_cast<const float*>(st + 2 * d);
+      const float* sk = reinterpret_cast<const float*>(st + 4 * d);
+      for (int t0 = tid; t0 < half; t0 += U * kComp) {
+        int ii[U], jj[U];
+        float c[U], sn[U], a[U][R], b[U][R];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int t = t0 + u * kComp;
+          ii[u] = -1;
+          if (t < half) {
+            const uint32_t pr = pk[t];
+            const int i = pr & 0xFFFF, j = pr >> 16;
+            if (i < d && j < d) { ii[u] = i; jj[u] = j; c[u] = ck[t]; sn[u] = sk[t]; }
+            else report_status(status, kStatusBadIndex);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (ii[u] >= 0) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              a[u][r] = xs[(size_t)r * d + ii[u]];
+              b[u][r] = xs[(size_t)r * d + jj[u]];
+            }
+          }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (ii[u] >= 0) {
+            float na[R], nb[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              na[r] = fmaf(c[u], a[u][r], sn[u] * b[u][r]);
+              nb[r] = fmaf(-sn[u], a[u][r], c[u] * b[u][r]);
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              xs[(size_t)r * d + ii[u]] = na[r];
+              xs[(size_t)r * d + jj[u]] = nb[r];
+            }
+          }
+      }
+    } else if (tid == kProd && ring > 1) {
+      // stage k - 1's slot is free since the barrier that started this stage
+      if (k >= 1 && k - 1 + ring < K) {
+        issue_stage(k - 1 + ring);
+        ++issued;
+      }
+      if (k + 1 < K) ok = mbar_wait_bounded(s_bar + 8u * ((k + 1) % ring), (uint32_t)(((k + 1) / ring) & 1));
+    }
+    failed = __syncthreads_or(!ok);
+    if (ring == 1 && k + 1 < K && !failed) {
+      if (tid == kProd) {
+        issue_stage(k + 1);
+        ++issued;
+        ok = mbar_wait_bounded(s_bar, (uint32_t)((k + 1) & 1));
+      }
+      failed = __syncthreads_or(!ok);
+    }
+  }
+  if (failed) {
+    // a stage never arrived: report, let the latest copy of every slot land
+    // (each wait bounded again), then leave
+    if (tid == kProd) {
+      report_status(status, kStatusTimeout);
+      for (int q = issued > ring ? issued - ring : 0; q < issued; ++q)
+        mbar_wait_bounded(s_bar + 8u * (q % ring), (uint32_t)((q / ring) & 1));
+    }
+    __syncthreads();
+    return false;
+  }
+
+  // channel scale and store: the scales of LB channel pairs are loaded (from
+  // L2, where the prologue put them) before any of them is used
+#pragma unroll 1
+  for (int cp0 = tid; cp0 < half; cp0 += LB * NTHR) {
+    float2 sc[LB];
+#pragma unroll
+    for (int q = 0; q < LB; ++q) {
+      const int cp = cp0 + q * NTHR;
+      sc[q] = make_float2(1.0f, 1.0f);
+      if (P.scale && cp < half) sc[q] = make_float2(__ldg(P.scale + 2 * cp), __ldg(P.scale + 2 * cp + 1));
+    }
+#pragma unroll
+    for (int q = 0; q < LB; ++q) {
+      const int cp = cp0 + q * NTHR;
+      if (cp >= half) continue;
+      const int c = 2 * cp;
+      const float f0 = 1.0f / sc[q].x, f1 = 1.0f / sc[q].y;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (r < nrows) {
+          const float2 v = *reinterpret_cast<const float2*>(xs + (size_t)r * d + c);
+          const size_t off = (size_t)(row0 + r) * d + c;
+          if constexpr (F16OUT)
+            *reinterpret_cast<__half2*>(static_cast<__half*>(P.out) + off) = __floats2half2_rn(v.x * f0, v.y * f1);
+          else
+            *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(P.out) + off) =
+                __floats2bfloat162_rn(v.x * f0, v.y * f1);
+        }
+      }
+    }
+  }
+  return true;
+}
+
+}  // namespace rotdec
+}  // namespace paro

@@ -41,6 +41,7 @@
 // depend on timing).
 #include "paro_internal.cuh"
 #include "w4_stream.cuh"
+#include "rotate_decode_cta.cuh"
 
 namespace paro {
 namespace {
@@ -88,6 +89,9 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -266,9 +270,14 @@ __device__ bool wait_flag(const unsigned long long* f, unsigned long long v) {
   }
 }
 
-template <bool F16, int NT>
+// FU > 0: the fused form (one token per linear): CTAs 0 .. rb.count - 1 run the
+// activation transform of one linear each, FU pairs per thread and round, and
+// publish a flag holding this launch's grid id once its x~ is written; the
+// INT4 CTAs request a linear's activations only after its flag.
+template <bool F16, int NT, int FU>
 __global__ void __launch_bounds__(Geo<NT>::W * 32, 1)
-w4_stream_kernel(const __grid_constant__ StreamBatch b, int* status, int pdl_wait) {
+w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ RotBatch rb, int* status,
+                 int pdl_wait) {
   using Gm = Geo<NT>;
   constexpr int W = Gm::W, D = Gm::D, SLOT = Gm::SLOT, XB = Gm::XB, PF = Gm::PF;
   extern __shared__ unsigned char smem_raw[];
@@ -278,6 +287,22 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, int* status, int pdl_wai
   // a programmatic dependent (the next call's transform) may start its table
   // fetches as SMs free up; it waits for this grid before touching its data
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  const int T = FU > 0 ? rb.count : 0;  // transform CTAs
+  if constexpr (FU > 0) {
+    if ((int)blockIdx.x < T) {
+      __shared__ __align__(8) uint64_t tbars[rotdec::kRotMaxRing];
+      const bool done = rotdec::rot_decode_cta<1, true, FU, W * 32>(
+          rb.p[blockIdx.x], 0, smem_raw + (sbase - smem_u32(smem_raw)), tbars, status, pdl_wait != 0);
+      if (done) {
+        // every thread's x~ stores, then the flag (the INT4 CTAs read x~ through
+        // the asynchronous proxy after seeing it)
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) st_flag(b.xflags + blockIdx.x, grid_tag());
+      }
+      return;
+    }
+  }
   __shared__ Meta meta[kMaxBatch];
   if (threadIdx.x < b.count) {
     const StreamProblem& P = b.p[threadIdx.x];
@@ -288,7 +313,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, int* status, int pdl_wai
   __syncthreads();
 
   // ---- this CTA's and this warp's units --------------------------------------------
-  const long long U = b.total_units, C = b.ctas, cta = blockIdx.x;
+  const long long U = b.total_units, C = b.ctas, cta = (long long)blockIdx.x - T;
   const long long c0 = part_start(cta, C, U), c1 = part_start(cta + 1, C, U), nC = c1 - c0;
   const long long w0 = c0 + part_start(warp, W, nC), w1 = c0 + part_start(warp + 1, W, nC);
   const int n = (int)(w1 - w0);
@@ -319,14 +344,42 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, int* status, int pdl_wai
   uint32_t szc[4] = {0u, 0u, 0u, 0u};  // scale and zero bits of the unit being computed
   if (n > 0) load_sz(meta[cc.pi], cc, g, t, szc);
   if (pdl_wait) asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  // the activations of the unit in slot s (with the slot's arrival; its codes
+  // were requested without one)
+  auto issue_x = [&](const Cur& c, int s) {
+    const CUtensorMap* xm = &b.p[c.pi].xmap;
+    const uint32_t sx = ring + (uint32_t)(s * SLOT + kUnitBytes), bar = bar0 + 8u * s;
+    mbar_arrive_expect_tx(bar, (uint32_t)(256 * meta[c.pi].M));
+    tma_load_2d(sx, xm, c.grp * 128, 0, bar);
+    tma_load_2d(sx + XB, xm, c.grp * 128 + 64, 0, bar);
+  };
+  // fused form (lane 0): linears whose x~ flag was seen, and slots whose
+  // activations are still to be requested
+  uint32_t xready = 0u, xpend = 0u;
+  const unsigned long long xtag = grid_tag();
+  auto x_ready = [&](int pi, bool block) -> bool {
+    if (FU == 0 || ((xready >> pi) & 1u)) return true;
+    bool seen;
+    if (block) {
+      seen = wait_flag(b.xflags + pi, xtag);
+      if (!seen) report_status(status, kStatusTimeout);
+    } else {
+      unsigned long long v;
+      asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];\n" : "=l"(v) : "l"(b.xflags + pi) : "memory");
+      seen = v == xtag;
+    }
+    if (!seen) return false;
+    // acquire the transform CTA's x~, then order the TMA reads after it
+    __threadfence();
+    asm volatile("fence.proxy.async.global;\n" ::: "memory");
+    xready |= 1u << pi;
+    return true;
+  };
 #pragma unroll 1
   for (int s = 0; s < D && s < n; ++s) {
     if (lane == 0) {
-      const CUtensorMap* xm = &b.p[ic.pi].xmap;
-      const uint32_t sx = ring + (uint32_t)(s * SLOT + kUnitBytes), bar = bar0 + 8u * s;
-      mbar_arrive_expect_tx(bar, (uint32_t)(256 * meta[ic.pi].M));
-      tma_load_2d(sx, xm, ic.grp * 128, 0, bar);
-      tma_load_2d(sx + XB, xm, ic.grp * 128 + 64, 0, bar);
+      if (x_ready(ic.pi, false)) issue_x(ic, s);
+      else xpend |= 1u << s;
     }
     cur_next(meta, ic);
   }
@@ -386,6 +439,17 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, int* status, int pdl_wai
     if (i + 1 < n) {
       cur_next(meta, nx);
       load_sz(meta[nx.pi], nx, g, t, szn);
+    }
+    if constexpr (FU > 0) {
+      // the unit's activations were deferred: wait (bounded) for its linear's x~
+      if (lane == 0 && ((xpend >> slot) & 1u)) {
+        // (on a timeout the slot still gets its arrival, so that its phase
+        // completes once the codes have landed; the status says the result is void)
+        if (x_ready(cc.pi, true)) issue_x(cc, slot);
+        else mbar_arrive(bar0 + 8u * slot);
+        xpend &= ~(1u << slot);
+      }
+      __syncwarp();
     }
     if (!mbar_wait(bar0 + 8u * slot, phase)) {
       report_status(status, kStatusTimeout);
@@ -477,10 +541,18 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, int* status, int pdl_wai
       if (lane == 0) {
         const StreamProblem& Q = b.p[ic.pi];
         const uint32_t bar = bar0 + 8u * slot;
-        mbar_arrive_expect_tx(bar, (uint32_t)(kUnitBytes + 256 * meta[ic.pi].M));
-        tma_load_2d(sw, &Q.qmap, ic.grp * 16, ic.tile * kStreamRows, bar);
-        tma_load_2d(sx, &Q.xmap, ic.grp * 128, 0, bar);
-        tma_load_2d(sx + XB, &Q.xmap, ic.grp * 128 + 64, 0, bar);
+        if (x_ready(ic.pi, false)) {
+          mbar_arrive_expect_tx(bar, (uint32_t)(kUnitBytes + 256 * meta[ic.pi].M));
+          tma_load_2d(sw, &Q.qmap, ic.grp * 16, ic.tile * kStreamRows, bar);
+          tma_load_2d(sx, &Q.xmap, ic.grp * 128, 0, bar);
+          tma_load_2d(sx + XB, &Q.xmap, ic.grp * 128 + 64, 0, bar);
+        } else {
+          // fused form, x~ not written yet: the codes now, the activations (and
+          // the slot's arrival) when the unit comes up
+          mbar_expect_tx(bar, (uint32_t)kUnitBytes);
+          tma_load_2d(sw, &Q.qmap, ic.grp * 16, ic.tile * kStreamRows, bar);
+          xpend |= 1u << slot;
+        }
       }
       cur_next(meta, ic);
     }
@@ -493,7 +565,12 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, int* status, int pdl_wai
     }
   }
   if (!ok) {
-    // let the copies still in flight land (each wait bounded) before leaving the ring
+    // let the copies still in flight land (each wait bounded) before leaving the
+    // ring; slots whose activations were never requested get their arrival first
+    if (lane == 0)
+      for (int q = 0; q < D; ++q)
+        if ((xpend >> q) & 1u) mbar_arrive(bar0 + 8u * q);
+    __syncwarp();
     for (int j = done; j < n && j < done + D; ++j) mbar_wait(bar0 + 8u * (j % D), (uint32_t)((j / D) & 1));
   }
 
@@ -684,12 +761,14 @@ bool stream_supported(int M, int d_in, int d_out, const void* x, const void* qwe
 
 size_t stream_workspace_bytes(int max_m) {
   const int NT = max_m <= 8 ? 1 : 2;
-  return round256((size_t)device_sm_count() * 2 * 8) + round256((size_t)device_sm_count() * 2 * (4 * NT * 32 * 4) * 4);
+  return round256((size_t)device_sm_count() * 2 * 8) + round256((size_t)device_sm_count() * 2 * (4 * NT * 32 * 4) * 4) +
+         round256((size_t)kMaxBatch * 8);
 }
 
 cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* qw, const __half* const* sc,
                               const __half* const* z, __nv_bfloat16* const* y, const int* M, const int* d_in,
-                              const int* d_out, int count, bool x_f16, void* ws, StreamBatch* out, int* nt_out) {
+                              const int* d_out, int count, bool x_f16, void* ws, StreamBatch* out, int* nt_out,
+                              int reserved_ctas) {
   if (count < 1 || count > kMaxBatch || !ws) return cudaErrorInvalidValue;
   EncodeTiled enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
@@ -736,9 +815,14 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
   const int W = maxM <= 8 ? Geo<1>::W : Geo<2>::W;
   const long long want = (units + W - 1) / W;
   const int sms = device_sm_count();
-  out->ctas = (int)(want < sms ? want : sms);
+  const int avail = sms - reserved_ctas;
+  if (avail < 1) return cudaErrorInvalidValue;
+  out->ctas = (int)(want < avail ? want : avail);
   out->flags = static_cast<unsigned long long*>(ws);
   out->partials = reinterpret_cast<float*>(static_cast<char*>(ws) + round256((size_t)sms * 2 * 8));
+  out->xflags = reinterpret_cast<unsigned long long*>(
+      static_cast<char*>(ws) + round256((size_t)sms * 2 * 8) +
+      round256((size_t)sms * 2 * (4 * (maxM <= 8 ? 1 : 2) * 32 * 4) * 4));
   *nt_out = maxM <= 8 ? 1 : 2;
   return cudaSuccess;
 }
@@ -758,12 +842,13 @@ cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* s
   cfg.numAttrs = pdl_wait ? 1 : 0;
   const int wait = pdl_wait ? 1 : 0;
   cudaError_t e;
+  const RotBatch none{};
 #define PARO_STREAM_LAUNCH(f16, nt)                                                                       \
   {                                                                                                       \
-    auto k = w4_stream_kernel<f16, nt>;                                                                   \
+    auto k = w4_stream_kernel<f16, nt, 0>;                                                                \
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                  \
     if (e != cudaSuccess) return e;                                                                       \
-    return cudaLaunchKernelEx(&cfg, k, b, status, wait);                                                  \
+    return cudaLaunchKernelEx(&cfg, k, b, none, status, wait);                                            \
   }
   if (x_f16) {
     if (NT == 1) PARO_STREAM_LAUNCH(true, 1) else PARO_STREAM_LAUNCH(true, 2)
@@ -771,6 +856,85 @@ cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* s
     if (NT == 1) PARO_STREAM_LAUNCH(false, 1) else PARO_STREAM_LAUNCH(false, 2)
   }
 #undef PARO_STREAM_LAUNCH
+}
+
+// ---- fused form -----------------------------------------------------------------------
+namespace {
+// dynamic shared memory of the fused kernel: the INT4 CTAs' rings, or a
+// transform CTA's row and stage slots after the 1024-byte alignment, whichever
+// is larger, within 227 KB less the kernel's static shared memory
+constexpr size_t kFusedSmemBudget = 227 * 1024 - 2048;
+size_t fused_rot_smem(int d, int ring) { return 1024 + (size_t)d * 4 + (size_t)ring * 6 * d; }
+// pairs per thread and round of the transform CTAs (W1 - 1 rotating warps)
+int fused_u(const RotBatch& rb) {
+  int max_half = 0;
+  for (int i = 0; i < rb.count; ++i) max_half = rb.p[i].d / 2 > max_half ? rb.p[i].d / 2 : max_half;
+  const int comp = Geo<1>::W * 32 - 32;
+  const int rounds = (max_half + comp - 1) / comp;
+  return rounds <= 4 ? 4 : (rounds <= 8 ? 8 : (rounds <= 10 ? 10 : 8));
+}
+}  // namespace
+
+bool fused_supported(const RotProblem* probs, int count) {
+  if (count < 1 || count > kMaxBatch) return false;
+  for (int i = 0; i < count; ++i) {
+    const RotProblem& p = probs[i];
+    if (p.M != 1 || p.d % 8 != 0 || p.K < 0 || p.K > 16 || fused_rot_smem(p.d, 1) > kFusedSmemBudget) return false;
+    if (p.K > 0 && ((reinterpret_cast<uintptr_t>(p.pairs) | reinterpret_cast<uintptr_t>(p.cos_t) |
+                     reinterpret_cast<uintptr_t>(p.sin_t)) & 15) != 0)
+      return false;
+  }
+  return true;
+}
+
+cudaError_t plan_fused_rot(const RotProblem* probs, int count, RotBatch* out) {
+  if (!fused_supported(probs, count)) return cudaErrorInvalidValue;
+  *out = RotBatch{};
+  for (int i = 0; i < count; ++i) {
+    RotProblem p = probs[i];
+    int ring = p.K < 1 ? 1 : (p.K > rotdec::kRotMaxRing ? rotdec::kRotMaxRing : p.K);
+    while (ring > 1 && fused_rot_smem(p.d, ring) > kFusedSmemBudget) --ring;
+    p.ring = ring;
+    p.cta_begin = i;
+    out->p[i] = p;
+  }
+  out->count = count;
+  out->total_ctas = count;
+  return cudaSuccess;
+}
+
+cudaError_t launch_fused_batch(const StreamBatch& b, const RotBatch& rb, int* status, cudaStream_t stream,
+                               bool pdl_wait) {
+  static_assert(sizeof(StreamBatch) + sizeof(RotBatch) + 16 <= 4096, "kernel parameters");
+  size_t smem = Geo<1>::SMEM;
+  for (int i = 0; i < rb.count; ++i) {
+    const size_t s = fused_rot_smem(rb.p[i].d, rb.p[i].ring);
+    smem = s > smem ? s : smem;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rb.count + b.ctas);
+  cfg.blockDim = dim3(Geo<1>::W * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_wait ? 1 : 0;
+  const int wait = pdl_wait ? 1 : 0;
+  const int u = fused_u(rb);
+  cudaError_t e;
+#define PARO_FUSED_LAUNCH(fu)                                                                             \
+  {                                                                                                       \
+    auto k = w4_stream_kernel<true, 1, fu>;                                                               \
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                  \
+    if (e != cudaSuccess) return e;                                                                       \
+    return cudaLaunchKernelEx(&cfg, k, b, rb, status, wait);                                              \
+  }
+  if (u == 4) PARO_FUSED_LAUNCH(4)
+  else if (u == 10) PARO_FUSED_LAUNCH(10)
+  else PARO_FUSED_LAUNCH(8)
+#undef PARO_FUSED_LAUNCH
 }
 
 }  // namespace paro

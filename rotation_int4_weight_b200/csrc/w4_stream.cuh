@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include "w4_gemv.cuh"  // kMaxBatch
+#include "rotate_decode.cuh"
 
 namespace paro {
 
@@ -29,8 +30,9 @@ struct StreamBatch {
   long long total_units;
   unsigned long long* flags;     // two per CTA: its partials' publication flags (workspace)
   float* partials;               // two tile partials per CTA (workspace)
+  unsigned long long* xflags;    // fused form: one per linear, set when its x~ is written (workspace)
   int count;
-  int ctas;
+  int ctas;                      // CTAs of the INT4 linear (after the transform CTAs in the fused form)
 };
 
 // True when a linear can run on the stream-K kernel (the caller also checks M).
@@ -41,9 +43,22 @@ size_t stream_workspace_bytes(int max_m);
 // x_f16 selects fp16 (else bf16) activations; ws points at stream_workspace_bytes().
 cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* qw, const __half* const* sc,
                               const __half* const* z, __nv_bfloat16* const* y, const int* M, const int* d_in,
-                              const int* d_out, int count, bool x_f16, void* ws, StreamBatch* out, int* nt_out);
+                              const int* d_out, int count, bool x_f16, void* ws, StreamBatch* out, int* nt_out,
+                              int reserved_ctas = 0);
 cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* status, cudaStream_t stream,
                                 bool pdl_wait);
+
+// The fused form for one token per linear: the kernel's first rb.count CTAs
+// each run the activation transform of one linear (writing its fp16 x~, the
+// activations b reads) and then publish a flag; the other CTAs run the INT4
+// linear, requesting a linear's activations once its flag is set, so their
+// weight streaming and the transforms overlap and a linear's arithmetic waits
+// only for its own transform.  b must come from plan_stream_batch with
+// reserved_ctas = rb.count and x_f16; rb from plan_fused_rot.
+bool fused_supported(const RotProblem* probs, int count);
+cudaError_t plan_fused_rot(const RotProblem* probs, int count, RotBatch* out);
+cudaError_t launch_fused_batch(const StreamBatch& b, const RotBatch& rb, int* status, cudaStream_t stream,
+                               bool pdl_wait);
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
 

@@ -385,6 +385,47 @@ def test_stream_decode_matches_oracle_and_repeats_bit_exactly(shapes_m, rotate):
         assert torch.equal(f.view(torch.int16), d["y"].view(torch.int16))
 
 
+# ---------------------------------------------------------------- fused decode (one token per linear)
+# With every linear at M = 1 the batched call runs the transforms in the INT4
+# kernel's first CTAs (one per linear), which publish x~ with a flag that the
+# INT4 CTAs wait for before requesting a linear's activations.
+@pytest.mark.parametrize("spec", [
+    # (d_in, d_out, K, transform): the widest linears take two-slot and one-slot
+    # stage rings inside the fused kernel; one linear has no transform (its x is
+    # only rounded to fp16); ragged output tails
+    [(14336, 272, 8, True), (16384, 64, 16, True), (512, 80, 0, False), (1536, 1040, 3, True)],
+    # the most linears a call takes: eight transform CTAs
+    [(512, 64, 8, True), (1024, 128, 2, True), (384, 96, 8, True), (2048, 64, 1, True),
+     (512, 208, 8, True), (640, 64, 5, True), (4096, 64, 8, True), (128, 64, 8, True)],
+])
+def test_fused_decode_matches_oracle_and_repeats_bit_exactly(spec):
+    probs, devs = [], []
+    for i, (d_in, d_out, K, rot) in enumerate(spec):
+        p = linear_problem(83, i, d_in, d_out, 1, K=K)
+        tables = dev_tables(p) if rot else (None, None, None, None)
+        qw, sc, z = _packed(p, rot)
+        y = torch.full((1, d_out), float("nan"), dtype=torch.bfloat16, device=DEV)
+        probs.append((p, rot))
+        devs.append(dict(x=dev_x(p.x), tables=tables, qw=qw, sc=sc, z=z, y=y))
+    layers = [paro.paro_linear(d["x"], *d["tables"], d["qw"], d["sc"], d["z"], d["y"]) for d in devs]
+    ws = paro.paro_rotate_w4_linear_batched(layers)
+    torch.cuda.synchronize()
+    assert paro.paro_get_device_status() == 0
+    first = [d["y"].clone() for d in devs]
+    for (p, rot), d in zip(probs, devs):
+        got = host(d["y"])
+        xt = oracle.rotate(p.x, p.pairs, p.cos_t, p.sin_t, p.scale) if rot else p.x
+        ref = oracle.linear(xt, oracle.dequantize(*to_np_pack(d["qw"], d["sc"], d["z"])))
+        assert_linear_close(got, ref)
+    for d in devs:
+        d["y"].fill_(float("nan"))
+    paro.paro_rotate_w4_linear_batched(layers, workspace=ws)
+    torch.cuda.synchronize()
+    assert paro.paro_get_device_status() == 0
+    for f, d in zip(first, devs):
+        assert torch.equal(f.view(torch.int16), d["y"].view(torch.int16))
+
+
 # ---------------------------------------------------------------- grouped tensor-core launch (batched, M >= 128)
 @pytest.mark.parametrize("shapes_m", [
     # mixed K, ragged token counts and ragged output tails in one launch
