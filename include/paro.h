@@ -193,15 +193,16 @@ typedef struct {
  * transformed activations of every linear (paro_workspace_bytes(M, d_in)
  * each, in order), then, when every M is at most 16, the publication flags
  * and partial sums of the stream-K INT4 linear (2 flags and 2 partial
- * 64-row tiles per SM).  The second part is optional: given only the first,
- * the call runs the older per-block kernel.
+ * 64-row tiles per SM, and one flag per linear for the fused form below).
+ * The second part is optional: given only the first, the call runs the older
+ * per-block kernel.
  */
 PARO_API size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int count);
 
 /*
  * Runs paro_rotate_w4_linear for up to PARO_MAX_BATCH independent linears with
- * two kernel launches in all (one transform launch, one INT4-linear launch),
- * e.g. the seven linears of one decoder layer; each linear has its own
+ * at most two kernel launches in all (one transform launch, one INT4-linear
+ * launch), e.g. the seven linears of one decoder layer; each linear has its own
  * transform ("one rotation operator plus one group-wise INT4 GEMM operator for
  * each layer", page "ParoQuant: pairwise rotations that survive deployment",
  * section "From fake quantization to a real TensorRT engine").  h_layers is a
@@ -216,7 +217,11 @@ PARO_API size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int co
  * the bf16 inputs to fp16 itself when every linear has at least 128 tokens,
  * else the inputs are first rounded to fp16 into the workspace, as the
  * transform does.  With many tokens the INT4 linears of all layers run as one
- * persistent tensor-core launch after the transforms.
+ * persistent tensor-core launch after the transforms.  When every linear has
+ * one token (M == 1) and the full workspace is given, the call is one launch:
+ * its first CTAs transform one linear each into the workspace and publish a
+ * flag, and the INT4 CTAs request a linear's activations once its flag is set
+ * (each linear's arithmetic waits for its own transform only).
  * The stream-K kernel's publication flags need no clearing: a flag holds the
  * id of the launch that wrote it, so one left by another launch, or never
  * written, is never taken for this launch's.  Two calls that may run at the
