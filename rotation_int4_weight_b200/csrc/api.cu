@@ -106,8 +106,9 @@ constexpr int kTensorCoreMinM = 128;
 
 // The INT4 linear on x (bf16, or fp16 when x_f16).  With pdl_wait the kernel is
 // launched as a programmatic dependent of the previous kernel in the stream and
-// waits for it before reading x (the weights may be read earlier, so only a
-// previous kernel that does not write them may trigger early).
+// waits for it before reading x or writing y (the weights may be read earlier,
+// so only a previous kernel that does not write them may trigger early: in this
+// library the INT4 and transform kernels trigger, the weight packing does not).
 cudaError_t launch_linear(const uint16_t* x, bool x_f16, const uint32_t* qweight, const uint16_t* scales,
                           const uint16_t* zeros, uint16_t* y, int M, int d_in, int d_out, cudaStream_t s,
                           bool pdl_wait, int* status) {
@@ -263,8 +264,10 @@ paro_status paro_w4_linear(const uint16_t* d_x, const uint32_t* d_qweight, const
       overlap(d_y, yb, d_scales, (size_t)d_out * (d_in / 128) * 2) ||
       overlap(d_y, yb, d_zeros, (size_t)d_out * (d_in / 128) * 2))
     return fail(PARO_ERR_INVALID_ARG, "y overlaps an input");
+  // a programmatic dependent of the previous kernel: only this library's INT4 and
+  // transform kernels trigger early, and none of them writes weights
   cudaError_t e = launch_linear(d_x, false, d_qweight, d_scales, d_zeros, d_y, M, d_in, d_out,
-                                reinterpret_cast<cudaStream_t>(stream), false, status_ptr());
+                                reinterpret_cast<cudaStream_t>(stream), true, status_ptr());
   return from_cuda(e, "w4 linear launch");
 }
 
@@ -440,13 +443,13 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     if (use_stream) {
       int* status = status_ptr();
       if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
-      return from_cuda(launch_stream(false, status, false), "batched w4 linear launch");
+      return from_cuda(launch_stream(false, status, true), "batched w4 linear launch");
     }
     for (int i = 0; i < n; ++i) gp[i].x = rp[i].x;
     paro::GemvBatch gb;
     int nt = 1;
     e = paro::plan_gemv_batch(gp, n, false, &gb, &nt);
-    if (e == cudaSuccess) e = paro::launch_gemv_batch(gb, nt, s, false);
+    if (e == cudaSuccess) e = paro::launch_gemv_batch(gb, nt, s, true);
     return from_cuda(e, "batched w4 linear launch");
   }
   int* status = status_ptr();
