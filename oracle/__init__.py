@@ -18,3 +18,4 @@ from .paro import (  # noqa: F401
     pack_weights,
     check_stage_disjoint,
 )
+from .backward import rotate_backward  # noqa: F401,E402
