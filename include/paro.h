@@ -117,6 +117,33 @@ PARO_API paro_status paro_rotate(const uint16_t* d_x, uint16_t* d_x_rot, int M, 
                         const float* d_scale, paro_stream_t stream);
 
 /*
+ * Gradients of the activation-side transform x~ = diag(1/s) R_K ... R_1 x for
+ * an upstream gradient G = dL/dx~ (page "ParoQuant: Pairwise Rotation
+ * Quantization for Efficient Reasoning LLM Inference", abstract: the Givens
+ * rotations and the channel-wise scaling are optimizable; the pages print no
+ * backward pass, and this is the chain rule of the forward transform):
+ *   dx = dL/dx,  dtheta[k][p] = dL/dtheta of pair p of stage k,  dscale = dL/ds,
+ * with (c, s) = (cos, sin) of the angle and x', h the stage's output and its
+ * gradient: dtheta = sum over tokens of (h_i x_j' - h_j x_i'); the stage's
+ * input gradient is the transposed rotation of h; dscale_c = -sum G_c x~_c / s_c.
+ * fp32 arithmetic.  d_x: bf16 [M][d] (the forward input); d_grad: fp32 [M][d];
+ * d_dx: fp32 [M][d]; d_dtheta: fp32 [K][d/2] (may be NULL when K == 0);
+ * d_dscale: fp32 [d], required when d_scale is given (else ignored).  The
+ * stage inputs are recovered from the outputs by the inverse rotation, so
+ * nothing is stored per stage; the per-block partial sums of dtheta and
+ * dscale go to d_workspace (paro_rotate_backward_workspace_bytes(M, d, K,
+ * d_scale != NULL) bytes, 16-byte aligned, caller-owned) and are added in a
+ * fixed order, so repeated calls give identical bits.  Needs d <= 28672
+ * (PARO_ERR_UNSUPPORTED beyond); pair indices >= d are skipped and reported
+ * through paro_get_device_status().
+ */
+PARO_API size_t paro_rotate_backward_workspace_bytes(int M, int d, int K, int with_scale);
+PARO_API paro_status paro_rotate_backward(const uint16_t* d_x, const float* d_grad, int M, int d, int K,
+                                          const uint16_t* d_pairs, const float* d_cos, const float* d_sin,
+                                          const float* d_scale, float* d_dx, float* d_dtheta, float* d_dscale,
+                                          void* d_workspace, size_t workspace_bytes, paro_stream_t stream);
+
+/*
  * Group-wise INT4 weight-only linear y = x W^T with w^ = (q - zero) * scale
  * (page "ParoQuant: pairwise rotations that survive deployment", section
  * "From fake quantization to a real TensorRT engine": the group-wise INT4 GEMM

@@ -19,6 +19,7 @@ __all__ = [
     "paro_pack_weights", "paro_rotate", "paro_w4_linear", "paro_rotate_w4_linear",
     "paro_rotate_w4_linear_noalloc", "paro_get_device_status", "EXPORTED", "ParoLinear", "paro_linear",
     "paro_batched_workspace_bytes", "paro_rotate_w4_linear_batched", "paro_plan_pair_order",
+    "paro_rotate_backward_workspace_bytes", "paro_rotate_backward",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libparo.so")
@@ -39,6 +40,8 @@ EXPORTED = {
     "paro_rotate_w4_linear_batched": (_I, [_P, _I, _I, _P, _S, _P]),
     "paro_plan_pair_order": (_I, [_P, _P, _P, _I, _I, _P, _P, _P]),
     "paro_get_device_status": (_I, [_P]),
+    "paro_rotate_backward_workspace_bytes": (_S, [_I, _I, _I, _I]),
+    "paro_rotate_backward": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
 }
 
 
@@ -147,6 +150,28 @@ def paro_rotate(x: torch.Tensor, pairs=None, cos_t=None, sin_t=None, scale=None,
                          _ptr(scale), _stream(stream))
     _check(st, "paro_rotate")
     return out
+
+
+def paro_rotate_backward(x: torch.Tensor, grad: torch.Tensor, pairs=None, cos_t=None, sin_t=None, scale=None, *,
+                         workspace=None, stream=None):
+    """Gradients of x~ = diag(1/s) R_K ... R_1 x for bf16 x [M, d] and fp32 grad = dL/dx~ [M, d].
+
+    Returns (dx fp32 [M, d], dtheta fp32 [K, d/2] or None when K == 0, dscale fp32 [d] or None
+    without a scale) and the workspace used (reusable).
+    """
+    M, d = x.shape
+    K = _K(pairs)
+    dx = torch.empty(M, d, dtype=torch.float32, device=x.device)
+    dtheta = torch.empty(K, d // 2, dtype=torch.float32, device=x.device) if K else None
+    dscale = torch.empty(d, dtype=torch.float32, device=x.device) if scale is not None else None
+    need = lib.paro_rotate_backward_workspace_bytes(M, d, K, 1 if scale is not None else 0)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    st = lib.paro_rotate_backward(_ptr(_u16(x)), _ptr(grad), M, d, K, _ptr(pairs), _ptr(cos_t), _ptr(sin_t),
+                                  _ptr(scale), _ptr(dx), _ptr(dtheta), _ptr(dscale), _ptr(workspace),
+                                  workspace.numel(), _stream(stream))
+    _check(st, "paro_rotate_backward")
+    return (dx, dtheta, dscale), workspace
 
 
 def paro_w4_linear(x: torch.Tensor, qweight, scales, zeros, *, out=None, group_size: int = 128, stream=None):

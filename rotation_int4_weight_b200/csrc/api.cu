@@ -250,6 +250,42 @@ paro_status paro_rotate(const uint16_t* d_x, uint16_t* d_x_rot, int M, int d, in
   return from_cuda(e, "rotate launch");
 }
 
+size_t paro_rotate_backward_workspace_bytes(int M, int d, int K, int with_scale) {
+  if (M <= 0 || d < 2 || (d & 1) || K < 0 || K > paro::kMaxStages) return 0;
+  return paro::rot_bwd_workspace_bytes(M, d, K, with_scale != 0);
+}
+
+paro_status paro_rotate_backward(const uint16_t* d_x, const float* d_grad, int M, int d, int K,
+                                 const uint16_t* d_pairs, const float* d_cos, const float* d_sin,
+                                 const float* d_scale, float* d_dx, float* d_dtheta, float* d_dscale,
+                                 void* d_workspace, size_t workspace_bytes, paro_stream_t stream) {
+  paro_status st;
+  if (M < 0) return fail(PARO_ERR_INVALID_ARG, "M = %d is negative", M);
+  if ((st = check_width(d)) != PARO_OK) return st;
+  if ((st = check_tables(K, d, d_pairs, d_cos, d_sin, d_scale)) != PARO_OK) return st;
+  if (paro::rot_bwd_rows(d) == 0) return fail(PARO_ERR_UNSUPPORTED, "d = %d is too wide for the backward kernel", d);
+  if (M == 0) return ok();
+  if (!d_x || !d_grad || !d_dx) return fail(PARO_ERR_INVALID_ARG, "null x, grad or dx pointer");
+  if (K > 0 && !d_dtheta) return fail(PARO_ERR_INVALID_ARG, "K > 0 needs a dtheta output");
+  if (d_scale && !d_dscale) return fail(PARO_ERR_INVALID_ARG, "a scale needs a dscale output");
+  if (!aligned(d_x, 4) || !aligned(d_grad, 4) || !aligned(d_dx, 4) || (d_dtheta && !aligned(d_dtheta, 4)) ||
+      (d_dscale && !aligned(d_dscale, 4)))
+    return fail(PARO_ERR_INVALID_ARG, "x, grad, dx, dtheta and dscale must be 4-byte aligned");
+  const size_t need = paro::rot_bwd_workspace_bytes(M, d, K, d_scale != nullptr);
+  if (need && (!d_workspace || workspace_bytes < need || !aligned(d_workspace, 16)))
+    return fail(PARO_ERR_INVALID_ARG, "workspace must be 16-byte aligned and hold %zu bytes", need);
+  const size_t gb = (size_t)M * d * 4;
+  if (overlap(d_dx, gb, d_grad, gb) || overlap(d_dx, gb, d_x, (size_t)M * d * 2) ||
+      (need && (overlap(d_workspace, need, d_dx, gb) || overlap(d_workspace, need, d_grad, gb))))
+    return fail(PARO_ERR_INVALID_ARG, "dx or the workspace overlaps an input");
+  int* status = status_ptr();
+  if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
+  cudaError_t e = paro::launch_rot_backward(d_x, d_grad, M, d, K, reinterpret_cast<const uint32_t*>(d_pairs), d_cos,
+                                            d_sin, d_scale, d_dx, d_dtheta, d_dscale, d_workspace, status,
+                                            reinterpret_cast<cudaStream_t>(stream));
+  return from_cuda(e, "rotate backward launch");
+}
+
 paro_status paro_w4_linear(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
                            const uint16_t* d_zeros, uint16_t* d_y, int M, int d_in, int d_out,
                            int group_size, paro_stream_t stream) {

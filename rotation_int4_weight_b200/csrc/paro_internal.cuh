@@ -29,6 +29,14 @@ paro_status record_error(paro_status s, const char* fmt, ...);
 // All return a cudaError_t from the launch (cudaSuccess when nothing failed).
 
 // Activation transform, bf16 -> bf16 (mode 0) or bf16 -> fp16 (mode 1).
+// Gradients of the activation transform (rotate_backward.cu): token rows per
+// block for width d (0 when d is too wide), the workspace of the per-block
+// partial sums, and the two launches (blocks, then the ordered reduction).
+int rot_bwd_rows(int d);
+size_t rot_bwd_workspace_bytes(int M, int d, int K, bool with_scale);
+cudaError_t launch_rot_backward(const uint16_t* x, const float* grad, int M, int d, int K, const uint32_t* pairs,
+                                const float* cos_t, const float* sin_t, const float* scale, float* dx, float* dtheta,
+                                float* dscale, void* ws, int* status, cudaStream_t stream);
 cudaError_t launch_rotate_act(const uint16_t* x, void* out, int out_is_f16, int M, int d, int K,
                               const uint16_t* pairs, const float* cos_t, const float* sin_t,
                               const float* scale, int* status, cudaStream_t stream, bool pdl_trigger);

@@ -120,6 +120,34 @@ def test_pack_validation(kwargs, expect):
     assert pack(**kwargs) == expect
 
 
+@pytest.mark.parametrize("args,expect", [
+    # (M, d, K, pairs, cos, sin, scale, dtheta, dscale, workspace bytes)
+    ((-1, 512, 8, A, B, C, D, E, E, 1 << 30), INVALID),     # negative M
+    ((4, 511, 8, A, B, C, D, E, E, 1 << 30), INVALID),      # odd width
+    ((4, 30000, 2, A, B, C, D, E, E, 1 << 30), UNSUPPORTED),  # wider than the kernel's shared memory
+    ((4, 512, 17, A, B, C, D, E, E, 1 << 30), UNSUPPORTED),   # more than 16 stages
+    ((4, 512, 8, None, B, C, D, E, E, 1 << 30), INVALID),   # K > 0 without pairs
+    ((4, 512, 8, A, B, C, D, None, E, 1 << 30), INVALID),   # K > 0 without a dtheta output
+    ((4, 512, 8, A, B, C, D, E, None, 1 << 30), INVALID),   # a scale without a dscale output
+    ((4, 512, 8, A, B, C, D, E, E, 16), INVALID),           # workspace too small
+    ((0, 512, 8, A, B, C, D, E, E, 0), OK),                 # no tokens: nothing enqueued
+])
+def test_rotate_backward_validation(args, expect):
+    M, d, K, pr, cs, sn, sc, dth, dsc, wsb = args
+    st = paro.lib.paro_rotate_backward(A, B, M, d, K, pr, cs, sn, sc, W, dth, dsc, C, wsb, None)
+    assert st == expect, paro.lib.paro_last_error()
+
+
+def test_rotate_backward_workspace_bytes():
+    # one partial per block of 4 rows (d <= 7168), 2 rows (d <= 14336) or 1 row
+    assert paro.lib.paro_rotate_backward_workspace_bytes(5, 512, 8, 1) == 2 * (8 * 256 + 512) * 4
+    assert paro.lib.paro_rotate_backward_workspace_bytes(5, 512, 8, 0) == 2 * 8 * 256 * 4
+    assert paro.lib.paro_rotate_backward_workspace_bytes(3, 8960, 2, 1) == 2 * (2 * 4480 + 8960) * 4
+    assert paro.lib.paro_rotate_backward_workspace_bytes(3, 20000, 1, 0) == 3 * 10000 * 4
+    assert paro.lib.paro_rotate_backward_workspace_bytes(0, 512, 8, 1) == 0
+    assert paro.lib.paro_rotate_backward_workspace_bytes(4, 30000, 8, 1) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     pkg = tmp_path / "rotation_int4_weight_b200"
     pkg.mkdir()
