@@ -154,6 +154,18 @@ class Linear:
     def rotate(self, paro):
         paro.paro_rotate(self.x, self.pairs, self.cos, self.sin, self.scale, out=self.xr)
 
+    def rotate_backward(self, paro):
+        # gradients of the transform for a synthetic upstream gradient (the
+        # calibration-time step; buffers made on first use)
+        import torch
+        if getattr(self, "grad", None) is None:
+            g = torch.Generator(device=self.x.device)
+            g.manual_seed(self.d_in * 7 + self.d_out)
+            self.grad = torch.randn(self.x.shape, generator=g, dtype=torch.float32, device=self.x.device)
+            need = paro.lib.paro_rotate_backward_workspace_bytes(self.M, self.d_in, self.pairs.shape[0], 1)
+            self.bws = torch.empty(max(need, 16), dtype=torch.uint8, device=self.x.device)
+        paro.paro_rotate_backward(self.x, self.grad, self.pairs, self.cos, self.sin, self.scale, workspace=self.bws)
+
     def fused_e2e(self, paro):
         self.x.copy_(self.x_host, non_blocking=True)
         self.fused(paro)
@@ -161,7 +173,8 @@ class Linear:
 
 
 # kernels launched per linear of each variant (batched: 2 per call of up to 7 linears)
-LAUNCHES = {"fused": 2, "unfused": 2, "plain": 1, "rotate": 1, "fused_e2e": 2}  # plain: 2 when M > 64
+LAUNCHES = {"fused": 2, "unfused": 2, "plain": 1, "rotate": 1, "fused_e2e": 2,  # plain: 2 when M > 64
+            "rotate_backward": 2}
 BATCH = 7  # linears per batched call (one decoder layer)
 
 
@@ -490,7 +503,7 @@ def main():
     ap.add_argument("--M", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--variants", default="batched,batched_plain,fused,plain,unfused,rotate")
+    ap.add_argument("--variants", default="batched,batched_plain,fused,plain,unfused,rotate,rotate_backward")
     ap.add_argument("--no-plan", action="store_true",
                     help="use the pair tables as drawn instead of the conflict-free order of paro_plan_pair_order")
     ap.add_argument("--profile", action="store_true",
@@ -533,6 +546,14 @@ def main():
             return sum(linear_bytes(l.d_in, l.d_out, M, rotate=False) for l in step_lins)
         if variant == "rotate":
             return sum(4 * M * l.d_in + TABLE_BYTES_PER_CH * l.d_in for l in step_lins)
+        if variant == "rotate_backward":
+            # x (bf16) and the upstream gradient in, dx out (fp32), the tables and
+            # the outputs dtheta, dscale; the per-block partial sums round trip
+            def bwd(l):
+                R = 4 if 8 * 4 * l.d_in <= 226 * 1024 else (2 if 8 * 2 * l.d_in <= 226 * 1024 else 1)
+                n = K_STAGES * l.d_in // 2 + l.d_in
+                return 10 * M * l.d_in + TABLE_BYTES_PER_CH * l.d_in + 4 * n + 2 * 4 * n * -(-M // R)
+            return sum(bwd(l) for l in step_lins)
         return sum(linear_bytes(l.d_in, l.d_out, M, unfused=(variant == "unfused")) for l in step_lins)
 
     variants = [v for v in args.variants.split(",") if v]
@@ -577,6 +598,7 @@ def main():
     w4_launches = units[0].launches("batched_plain") if "batched_plain" in results else len(step_lins)
     traffic = measured_traffic(args.config, args.M)
     rot_gbs = bytes_of("rotate") / (results["rotate"] * 1e-3) / 1e9 if "rotate" in results else None
+    bwd_ms = results.get("rotate_backward")
     prefill = M >= PREFILL_M
 
     out = {
@@ -617,6 +639,12 @@ def main():
         "rotation_overhead_per_linear_fused_pct": (round(100 * (results["fused"] - plain_ms) / plain_ms, 2)
                                                    if plain_ms and "fused" in results else None),
         "rotate_kernel_gbs": round(rot_gbs, 1) if rot_gbs else None,
+        "rotate_backward": ({"ms_per_step": round(bwd_ms, 6),
+                             "gbs": round(bytes_of("rotate_backward") / (bwd_ms * 1e-3) / 1e9, 1),
+                             "what": "dL/dx, dL/dtheta, dL/ds of the step's transforms for a synthetic upstream "
+                                     "gradient (paro_rotate_backward, one call per linear)",
+                             "bound": "shared memory: each stage moves 8 B per element forward and 16 B back "
+                                      "(x and its gradient)"} if bwd_ms else None),
         "tokens_per_s": round(M * world / (ms * 1e-3), 1),
         "tflops": round(flops_step * world / (ms * 1e-3) / 1e12, 3),
         "hbm_frac_of_measured": round(value / hbm, 4),
