@@ -650,9 +650,10 @@ def main():
         "hbm_frac_of_measured": round(value / hbm, 4),
     }
     if prefill:
-        out["roofline"] = {"bound": "tensor", "achieved": round(flops_step / (w4_ms * 1e-3) / 1e12, 2),
+        tf = flops_step / (w4_ms * 1e-3) / 1e12 if w4_ms else None
+        out["roofline"] = {"bound": "tensor", "achieved": round(tf, 2) if tf else None,
                            "peak": bf16, "unit": "TFLOP/s",
-                           "frac": round(flops_step / (w4_ms * 1e-3) / 1e12 / bf16, 4), "traffic": traffic,
+                           "frac": round(tf / bf16, 4) if tf else None, "traffic": traffic,
                            "algorithmic_bytes_per_launch": int(bytes_of("plain") / w4_launches),
                            "kernel": "INT4 linear, 2*M*d_in*d_out / device time",
                            "peak_kind": f"{peak_kind} bf16 dense (f16 operands: same nominal rate)"}
