@@ -25,12 +25,11 @@
 namespace paro {
 namespace {
 
-constexpr int kBwdThreads = 1024;
 constexpr size_t kBwdSmemBudget = 227 * 1024 - 1024;
 
-// shared memory: the rows and their gradients (8 R d bytes), and with STAGED
-// two stage tables (pairs, cos, sin: 6 d bytes each)
-size_t bwd_smem(int d, int R, bool staged) { return (size_t)8 * R * d + (staged ? (size_t)12 * d : 0); }
+// shared memory: the rows and their gradients (8 R d bytes) and NB stage
+// tables (pairs, cos, sin: 6 d bytes each)
+size_t bwd_smem(int d, int R, int NB) { return (size_t)8 * R * d + (size_t)NB * 6 * d; }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
@@ -38,10 +37,6 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
                : "memory");
 }
 
-// STAGED: the tables of the next stage step (forward k = 0 .. K-1, then
-// backward k = K-1 .. 0) are copied into shared memory (cp.async, 16 bytes a
-// thread and copy) while the current step runs; otherwise every pair reads its
-// table entries from global memory.
 template <int R> struct Vec;
 template <> struct Vec<1> { using T = float; };
 template <> struct Vec<2> { using T = float2; };
@@ -50,8 +45,12 @@ __device__ __forceinline__ float& el(float& v, int) { return v; }
 __device__ __forceinline__ float& el(float2& v, int r) { return r == 0 ? v.x : v.y; }
 __device__ __forceinline__ float& el(float4& v, int r) { return r == 0 ? v.x : (r == 1 ? v.y : (r == 2 ? v.z : v.w)); }
 
-template <int R, bool STAGED>
-__global__ void __launch_bounds__(kBwdThreads)
+// NB > 0: the tables of the stage steps (forward k = 0 .. K-1, then backward
+// k = K-1 .. 0) are copied into a ring of NB shared-memory buffers (cp.async,
+// 16 bytes a thread and copy), NB - 1 steps ahead of their use; NB = 0: every
+// pair reads its table entries from global memory.  NTH threads a CTA.
+template <int R, int NB, int NTH>
+__global__ void __launch_bounds__(NTH)
 rot_bwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ grad, int M, int d, int K,
                const uint32_t* __restrict__ pairs, const float* __restrict__ cos_t, const float* __restrict__ sin_t,
                const float* __restrict__ scale, float* __restrict__ dx, float* __restrict__ part, int* status) {
@@ -61,7 +60,8 @@ rot_bwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ grad, i
   // channels of x and of h with four vector loads and four vector stores
   VT* xs = reinterpret_cast<VT*>(sm);                 // [d] x R
   VT* hs = reinterpret_cast<VT*>(sm + (size_t)R * d);  // [d] x R
-  float* tb = sm + (size_t)2 * R * d;  // STAGED: 2 x (pairs [half] | cos [half] | sin [half])
+  float* tb = sm + (size_t)2 * R * d;  // NB x (pairs [half] | cos [half] | sin [half])
+  constexpr bool STAGED = NB > 0;
   const int half = d >> 1, tid = threadIdx.x;
   const int row0 = blockIdx.x * R, nrows = min(R, M - row0);
   // this block's partial sums: dtheta [K][half], then ds [d] (with a scale)
@@ -69,7 +69,7 @@ rot_bwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ grad, i
   float* psc = pth + (size_t)K * half;
 
   // rows (bf16) -> fp32, channel-major; rows past M are zero
-  for (int c = tid; c < d; c += kBwdThreads) {
+  for (int c = tid; c < d; c += NTH) {
     VT v;
 #pragma unroll
     for (int r = 0; r < R; ++r)
@@ -80,13 +80,13 @@ rot_bwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ grad, i
 
   // table step q (0 .. 2K-1) is stage q (forward) or 2K-1-q (backward)
   auto stage_of = [&](int q) { return q < K ? q : 2 * K - 1 - q; };
-  auto stage_copy = [&](int q) {  // STAGED: step q's table into buffer q % 2
+  auto stage_copy = [&](int q) {  // step q's table into buffer q % NB
     if constexpr (STAGED) {
       if (q < 2 * K) {
         const int k = stage_of(q);
-        float* dst = tb + (size_t)(q & 1) * 3 * half;
+        float* dst = tb + (size_t)(q % (NB > 0 ? NB : 1)) * 3 * half;
         const int chunks = half / 4;  // 16-byte pieces of each of the three arrays
-        for (int u = tid; u < 3 * chunks; u += kBwdThreads) {
+        for (int u = tid; u < 3 * chunks; u += NTH) {
           const int a = u / chunks, o = (u - a * chunks) * 4;
           const void* src = a == 0 ? (const void*)(pairs + (size_t)k * half + o)
                                    : (a == 1 ? (const void*)(cos_t + (size_t)k * half + o)
@@ -97,15 +97,15 @@ rot_bwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ grad, i
       asm volatile("cp.async.commit_group;\n" ::: "memory");
     }
   };
-  auto stage_ready = [&]() {  // STAGED: the current step's copies have landed, for every thread
-    if constexpr (STAGED) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+  auto stage_ready = [&]() {  // the current step's copies have landed, for every thread
+    if constexpr (STAGED) asm volatile("cp.async.wait_group %0;\n" ::"n"(NB > 0 ? NB - 1 : 0) : "memory");
     __syncthreads();
   };
   // the pair and angle of pair t in table step q
   auto pair_of = [&](int q, int t, int& i, int& j, float& c, float& s) -> bool {
     uint32_t pr;
     if constexpr (STAGED) {
-      const float* b = tb + (size_t)(q & 1) * 3 * half;
+      const float* b = tb + (size_t)(q % (NB > 0 ? NB : 1)) * 3 * half;
       pr = __float_as_uint(b[t]);
       c = b[half + t];
       s = b[2 * half + t];
@@ -121,13 +121,14 @@ rot_bwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ grad, i
     report_status(status, kStatusBadIndex);
     return false;
   };
-  stage_copy(0);
+#pragma unroll
+  for (int q = 0; q + 1 < NB; ++q) stage_copy(q);
   // forward: x' = R_K ... R_1 x
 #pragma unroll 1
   for (int k = 0; k < K; ++k) {
-    stage_copy(k + 1);
+    stage_copy(k + NB - 1);
     stage_ready();
-    for (int t = tid; t < half; t += kBwdThreads) {
+    for (int t = tid; t < half; t += NTH) {
       int i, j;
       float c, s;
       if (!pair_of(k, t, i, j, c, s)) continue;
@@ -143,7 +144,7 @@ rot_bwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ grad, i
     __syncthreads();
   }
   // scale step: h = G / s, ds partial = -sum_r G (x'/s) / s
-  for (int c = tid; c < d; c += kBwdThreads) {
+  for (int c = tid; c < d; c += NTH) {
     const float sc = scale ? __ldg(scale + c) : 1.f;
     const VT xv = xs[c];
     VT hv;
@@ -167,9 +168,9 @@ rot_bwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ grad, i
 #pragma unroll 1
   for (int k = K - 1; k >= 0; --k) {
     const int q = 2 * K - 1 - k;  // table step
-    stage_copy(q + 1);
+    stage_copy(q + NB - 1);
     stage_ready();
-    for (int t = tid; t < half; t += kBwdThreads) {
+    for (int t = tid; t < half; t += NTH) {
       int i, j;
       float dt = 0.f, c, s;
       if (pair_of(q, t, i, j, c, s)) {
@@ -192,7 +193,7 @@ rot_bwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ grad, i
     __syncthreads();
   }
   // dL/dx of the block's rows
-  for (int c = tid; c < d; c += kBwdThreads) {
+  for (int c = tid; c < d; c += NTH) {
     VT hv = hs[c];
 #pragma unroll
     for (int r = 0; r < R; ++r)
@@ -238,15 +239,29 @@ rot_bwd_reduce_kernel(const float* __restrict__ part, int blocks, int K, int hal
 
 }  // namespace
 
-int rot_bwd_rows(int d) {
+namespace {
+// Launch shape for width d: rows a CTA, table buffers, threads.  Two CTAs of
+// 512 threads an SM when their rows and two tables fit in half the shared
+// memory (each covers the other's table latency); else one CTA of 1024 threads
+// with up to four rows and as many table buffers as fit (three: the copies run
+// two steps ahead); the widest rows read their tables from global memory.
+struct BwdPlan {
+  int R, NB, NTH;
+};
+BwdPlan bwd_plan(int d) {
+  const bool al = d % 8 == 0;
   for (int R = 4; R >= 1; R >>= 1)
-    if (bwd_smem(d, R, false) <= kBwdSmemBudget) return R;
-  return 0;
+    if (al && 2 * bwd_smem(d, R, 2) + 2048 <= kBwdSmemBudget) return {R, 2, 512};
+  for (int R = 4; R >= 1; R >>= 1) {
+    if (al && bwd_smem(d, R, 3) <= kBwdSmemBudget) return {R, 3, 1024};
+    if (al && bwd_smem(d, R, 2) <= kBwdSmemBudget) return {R, 2, 1024};
+    if (bwd_smem(d, R, 0) <= kBwdSmemBudget) return {R, 0, 1024};
+  }
+  return {0, 0, 0};
 }
+}  // namespace
 
-// the tables are staged when both buffers fit next to the rows and every stage's
-// arrays start on a 16-byte boundary
-bool rot_bwd_staged(int d, int R) { return d % 8 == 0 && bwd_smem(d, R, true) <= kBwdSmemBudget; }
+int rot_bwd_rows(int d) { return bwd_plan(d).R; }
 
 size_t rot_bwd_workspace_bytes(int M, int d, int K, bool with_scale) {
   const int R = rot_bwd_rows(d);
@@ -258,28 +273,39 @@ size_t rot_bwd_workspace_bytes(int M, int d, int K, bool with_scale) {
 cudaError_t launch_rot_backward(const uint16_t* x, const float* grad, int M, int d, int K, const uint32_t* pairs,
                                 const float* cos_t, const float* sin_t, const float* scale, float* dx, float* dtheta,
                                 float* dscale, void* ws, int* status, cudaStream_t stream) {
-  const int R = rot_bwd_rows(d);
-  if (R == 0) return cudaErrorInvalidValue;
-  const int blocks = (M + R - 1) / R;
-  const bool staged = rot_bwd_staged(d, R) && (reinterpret_cast<uintptr_t>(pairs) & 15) == 0 &&
-                      (reinterpret_cast<uintptr_t>(cos_t) & 15) == 0 && (reinterpret_cast<uintptr_t>(sin_t) & 15) == 0;
-  const size_t smem = bwd_smem(d, R, staged);
+  BwdPlan pl = bwd_plan(d);
+  if (pl.R == 0) return cudaErrorInvalidValue;
+  if (pl.NB > 0 && K > 0 &&
+      ((reinterpret_cast<uintptr_t>(pairs) | reinterpret_cast<uintptr_t>(cos_t) | reinterpret_cast<uintptr_t>(sin_t)) &
+       15) != 0) {
+    pl.NB = 0;  // the tables are copied in 16-byte pieces
+    pl.NTH = 1024;
+  }
+  const int blocks = (M + pl.R - 1) / pl.R;
+  const size_t smem = bwd_smem(d, pl.R, pl.NB);
   float* part = static_cast<float*>(ws);
-  cudaError_t e;
-#define PARO_BWD_LAUNCH(r, st)                                                                              \
-  {                                                                                                         \
-    e = cudaFuncSetAttribute(rot_bwd_kernel<r, st>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-    if (e != cudaSuccess) return e;                                                                         \
-    rot_bwd_kernel<r, st><<<blocks, kBwdThreads, smem, stream>>>(x, grad, M, d, K, pairs, cos_t, sin_t, scale, \
-                                                                 dx, part, status);                        \
+  cudaError_t e = cudaErrorInvalidValue;
+#define PARO_BWD_LAUNCH(r, nb, nth)                                                                             \
+  if (pl.R == r && pl.NB == nb && pl.NTH == nth) {                                                              \
+    e = cudaFuncSetAttribute(rot_bwd_kernel<r, nb, nth>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    if (e != cudaSuccess) return e;                                                                             \
+    rot_bwd_kernel<r, nb, nth><<<blocks, nth, smem, stream>>>(x, grad, M, d, K, pairs, cos_t, sin_t, scale, dx,   \
+                                                              part, status);                                    \
+    e = cudaGetLastError();                                                                                     \
   }
-  if (staged) {
-    if (R == 4) PARO_BWD_LAUNCH(4, true) else if (R == 2) PARO_BWD_LAUNCH(2, true) else PARO_BWD_LAUNCH(1, true)
-  } else {
-    if (R == 4) PARO_BWD_LAUNCH(4, false) else if (R == 2) PARO_BWD_LAUNCH(2, false) else PARO_BWD_LAUNCH(1, false)
-  }
+  PARO_BWD_LAUNCH(4, 2, 512)
+  PARO_BWD_LAUNCH(2, 2, 512)
+  PARO_BWD_LAUNCH(1, 2, 512)
+  PARO_BWD_LAUNCH(4, 3, 1024)
+  PARO_BWD_LAUNCH(2, 3, 1024)
+  PARO_BWD_LAUNCH(1, 3, 1024)
+  PARO_BWD_LAUNCH(4, 2, 1024)
+  PARO_BWD_LAUNCH(2, 2, 1024)
+  PARO_BWD_LAUNCH(1, 2, 1024)
+  PARO_BWD_LAUNCH(4, 0, 1024)
+  PARO_BWD_LAUNCH(2, 0, 1024)
+  PARO_BWD_LAUNCH(1, 0, 1024)
 #undef PARO_BWD_LAUNCH
-  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t n = (size_t)K * (d / 2) + (scale ? d : 0);
   if (n == 0) return cudaSuccess;
