@@ -503,13 +503,30 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
   }
   if (decode_ok && use_stream && paro::fused_supported(rp, n)) {
     // one token per linear: the transforms run in the INT4 kernel's first CTAs
-    // (one per linear) and each linear's arithmetic waits only for its own x~
+    // (one per linear) and each linear's arithmetic waits only for its own x~.
+    // The widest linear (the slowest transform) goes last and to its own CTAs.
+    int widest = 0;
+    for (int i = 1; i < n; ++i)
+      if (rp[i].d > rp[widest].d) widest = i;
+    if (widest != n - 1) {
+      const paro::RotProblem r = rp[widest];
+      const paro::GemvProblem q = gp[widest];
+      for (int i = widest; i + 1 < n; ++i) {
+        rp[i] = rp[i + 1];
+        gp[i] = gp[i + 1];
+      }
+      rp[n - 1] = r;
+      gp[n - 1] = q;
+    }
     paro::RotBatch rb;
     paro::StreamBatch sb;
     int nt = 1;
     e = paro::plan_fused_rot(rp, n, &rb);
     if (e == cudaSuccess) e = plan_stream(true, rb.count, &sb, &nt);
-    if (e == cudaSuccess) e = paro::launch_fused_batch(sb, rb, status, s, true);
+    if (e == cudaSuccess) {
+      paro::set_fused_split(sb);
+      e = paro::launch_fused_batch(sb, rb, status, s, true);
+    }
     return from_cuda(e, "batched fused launch");
   }
   if (decode_ok) {

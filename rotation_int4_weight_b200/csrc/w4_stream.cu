@@ -314,7 +314,15 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
 
   // ---- this CTA's and this warp's units --------------------------------------------
   const long long U = b.total_units, C = b.ctas, cta = (long long)blockIdx.x - T;
-  const long long c0 = part_start(cta, C, U), c1 = part_start(cta + 1, C, U), nC = c1 - c0;
+  // CTA ranges: CTAs 0 .. CA - 1 split units [0, UA) evenly, the others [UA, U)
+  const long long CA = b.ctas_a, UA = b.units_a;
+  auto cta_start = [&](long long c) -> long long {
+    return c <= CA ? part_start(c, CA, UA) : UA + part_start(c - CA, C - CA, U - UA);
+  };
+  auto cta_of = [&](long long x) -> long long {
+    return x < UA ? part_of(x, CA, UA) : CA + part_of(x - UA, C - CA, U - UA);
+  };
+  const long long c0 = cta_start(cta), c1 = cta_start(cta + 1), nC = c1 - c0;
   const long long w0 = c0 + part_start(warp, W, nC), w1 = c0 + part_start(warp + 1, W, nC);
   const int n = (int)(w1 - w0);
   const uint32_t ring = sbase + (uint32_t)(warp * D * SLOT);
@@ -689,11 +697,11 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
       for (int m = 0; m < NT; ++m)
 #pragma unroll
         for (int e = 0; e < 4; ++e) tot[rt][m][e] = 0.f;
-    const long long ca = part_of(Ub, C, U);
+    const long long ca = cta_of(Ub);
 #pragma unroll 1
     for (long long cx = ca; cx < cta; ++cx) {
-      const long long s0 = part_start(cx, C, U);
-      if (part_start(cx + 1, C, U) <= s0) continue;  // a CTA without units
+      const long long s0 = cta_start(cx);
+      if (cta_start(cx + 1) <= s0) continue;  // a CTA without units
       const int e = (Ub <= s0) ? 0 : 1;
       int seen = 1;
       if (lane == 0) seen = wait_flag(b.flags + cx * 2 + e, tag) ? 1 : 0;
@@ -818,6 +826,8 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
   const int avail = sms - reserved_ctas;
   if (avail < 1) return cudaErrorInvalidValue;
   out->ctas = (int)(want < avail ? want : avail);
+  out->ctas_a = out->ctas;
+  out->units_a = units;
   out->flags = static_cast<unsigned long long*>(ws);
   out->partials = reinterpret_cast<float*>(static_cast<char*>(ws) + round256((size_t)sms * 2 * 8));
   out->xflags = reinterpret_cast<unsigned long long*>(
@@ -874,6 +884,25 @@ int fused_u(const RotBatch& rb) {
   return rounds <= 4 ? 4 : (rounds <= 8 ? 8 : (rounds <= 10 ? 10 : 8));
 }
 }  // namespace
+
+void set_fused_split(StreamBatch& b) {
+  b.ctas_a = b.ctas;
+  b.units_a = b.total_units;
+  if (b.count < 2 || b.ctas < 4) return;
+  int other = 0;
+  for (int i = 0; i + 1 < b.count; ++i) other = b.p[i].d_in > other ? b.p[i].d_in : other;
+  const int wide = b.p[b.count - 1].d_in;
+  if (2 * wide < 3 * other) return;
+  // units a CTA of the last linear gets, relative to the others: the later its
+  // x~ comes (the wider it is than the rest), the fewer (fitted to the arrival
+  // times of the transforms on B200 for Qwen2.5-1.5B and Llama-3-8B layers)
+  const double rho = 1.0 - 0.65 * (double)(wide - other) / wide;
+  const long long UA = b.p[b.count - 1].unit_begin, UB = b.total_units - UA;
+  long long CA = (long long)((double)b.ctas / (1.0 + (double)UB / (rho * (double)UA)) + 0.5);
+  CA = CA < 1 ? 1 : (CA > b.ctas - 1 ? b.ctas - 1 : CA);
+  b.ctas_a = (int)CA;
+  b.units_a = UA;
+}
 
 bool fused_supported(const RotProblem* probs, int count) {
   if (count < 1 || count > kMaxBatch) return false;

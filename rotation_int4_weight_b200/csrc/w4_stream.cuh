@@ -31,6 +31,11 @@ struct StreamBatch {
   unsigned long long* flags;     // two per CTA: its partials' publication flags (workspace)
   float* partials;               // two tile partials per CTA (workspace)
   unsigned long long* xflags;    // fused form: one per linear, set when its x~ is written (workspace)
+  // CTAs 0 .. ctas_a - 1 split units [0, units_a) evenly and the others the rest
+  // (the fused form gives the widest linear, whose x~ comes last, fewer units a
+  // CTA); ctas_a = ctas, units_a = total_units is the even split
+  long long units_a;
+  int ctas_a;
   int count;
   int ctas;                      // CTAs of the INT4 linear (after the transform CTAs in the fused form)
 };
@@ -56,6 +61,11 @@ cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* s
 // only for its own transform.  b must come from plan_stream_batch with
 // reserved_ctas = rb.count and x_f16; rb from plan_fused_rot.
 bool fused_supported(const RotProblem* probs, int count);
+// When the last linear is at least 1.5 times wider than any other, its
+// transform finishes last: its units go to a separate group of CTAs with
+// proportionally fewer units each, so that those CTAs, which start late,
+// finish with the others.
+void set_fused_split(StreamBatch& b);
 cudaError_t plan_fused_rot(const RotProblem* probs, int count, RotBatch* out);
 cudaError_t launch_fused_batch(const StreamBatch& b, const RotBatch& rb, int* status, cudaStream_t stream,
                                bool pdl_wait);
