@@ -501,23 +501,27 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     }
     if (all_tc) return from_cuda(paro::launch_w4_tc_batch(tl, n, false, status, s), "batched w4 linear launch");
   }
-  if (decode_ok && use_stream && paro::fused_supported(rp, n)) {
-    // one token per linear: the transforms run in the INT4 kernel's first CTAs
-    // (one per linear) and each linear's arithmetic waits only for its own x~.
-    // The widest linear (the slowest transform) goes last and to its own CTAs.
+  // the widest linear (the slowest transform) last, so that its units go to the
+  // INT4 grid's last CTAs
+  auto widest_last = [&]() {
     int widest = 0;
     for (int i = 1; i < n; ++i)
       if (rp[i].d > rp[widest].d) widest = i;
-    if (widest != n - 1) {
-      const paro::RotProblem r = rp[widest];
-      const paro::GemvProblem q = gp[widest];
-      for (int i = widest; i + 1 < n; ++i) {
-        rp[i] = rp[i + 1];
-        gp[i] = gp[i + 1];
-      }
-      rp[n - 1] = r;
-      gp[n - 1] = q;
+    if (widest == n - 1) return;
+    const paro::RotProblem r = rp[widest];
+    const paro::GemvProblem q = gp[widest];
+    for (int i = widest; i + 1 < n; ++i) {
+      rp[i] = rp[i + 1];
+      gp[i] = gp[i + 1];
     }
+    rp[n - 1] = r;
+    gp[n - 1] = q;
+  };
+  if (decode_ok && use_stream && paro::fused_supported(rp, n)) {
+    // one token per linear: the transforms run in the INT4 kernel's first CTAs
+    // (one per linear) and each linear's arithmetic waits only for its own x~.
+    // The widest linear goes to its own CTAs.
+    widest_last();
     paro::RotBatch rb;
     paro::StreamBatch sb;
     int nt = 1;
@@ -528,6 +532,27 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
       e = paro::launch_fused_batch(sb, rb, status, s, true);
     }
     return from_cuda(e, "batched fused launch");
+  }
+  if (decode_ok && use_stream) {
+    // few tokens: the transform launch publishes a flag per CTA, and the INT4
+    // launch after it requests a linear's x~ once that linear's transform CTAs
+    // have all published, not when the whole transform launch is done
+    widest_last();
+    paro::RotBatch rb;
+    paro::StreamBatch sb;
+    int R = 1, nt = 1;
+    e = paro::plan_rot_batch(rp, n, &rb, &R);
+    if (e == cudaSuccess) e = plan_stream(true, 0, &sb, &nt);
+    if (e != cudaSuccess) return from_cuda(e, "batched decode plan");
+    rb.tagword = sb.tagword;
+    rb.xflags = sb.xflags;
+    for (int i = 0; i < n; ++i) {
+      sb.p[i].xf_begin = rb.p[i].cta_begin;
+      sb.p[i].xf_count = (rb.p[i].M + R - 1) / R;
+    }
+    e = paro::launch_rot_batch(rb, R, true, status, s, true, true);
+    if (e == cudaSuccess) e = paro::launch_stream_flagged(sb, nt, status, s);
+    return from_cuda(e, "batched decode launch");
   }
   if (decode_ok) {
     paro::RotBatch rb;
@@ -557,7 +582,6 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     return from_cuda(e, "batched launch");
   }
   if (e != cudaSuccess) return from_cuda(e, "batched transform launch");
-  if (use_stream) return from_cuda(launch_stream(true, status, true), "batched w4 linear launch");
   paro::GemvBatch gb;
   int nt = 1;
   e = paro::plan_gemv_batch(gp, n, true, &gb, &nt);

@@ -33,14 +33,32 @@ __global__ void __launch_bounds__(kRotThreads)
 rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_trigger, int pdl_wait) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ __align__(8) uint64_t bars[rotdec::kRotMaxRing];
+  unsigned long long gid = 0;
+  if (batch.tagword) {
+    asm volatile("mov.u64 %0, %%gridid;\n" : "=l"(gid));
+    // the INT4 linear launched after this grid reads the word before it lets
+    // its own dependents (the next transform) launch, so it sees this id
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      asm volatile("st.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(batch.tagword), "l"(gid) : "memory");
+      __threadfence();
+    }
+    __syncthreads();
+  }
   if (pdl_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   int pi = 0;
 #pragma unroll 1
   while (pi + 1 < batch.count && (int)blockIdx.x >= batch.p[pi + 1].cta_begin) ++pi;
   const RotProblem& P = batch.p[pi];
   constexpr int U = UP > 0 ? UP : (R == 4 ? 2 : 4);
-  rotdec::rot_decode_cta<R, F16OUT, U, kRotThreads>(P, ((int)blockIdx.x - P.cta_begin) * R, smem, bars, status,
-                                                   pdl_wait != 0);
+  const bool done = rotdec::rot_decode_cta<R, F16OUT, U, kRotThreads>(
+      P, ((int)blockIdx.x - P.cta_begin) * R, smem, bars, status, pdl_wait != 0);
+  if (batch.xflags && done) {
+    // every thread's x~ stores, then this CTA's flag
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0)
+      asm volatile("st.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(batch.xflags + blockIdx.x), "l"(gid) : "memory");
+  }
 }
 
 size_t rot_smem(int d, int R, int ring) { return (size_t)d * R * 4 + (size_t)ring * 6 * d; }

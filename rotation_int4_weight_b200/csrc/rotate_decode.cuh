@@ -23,6 +23,12 @@ struct RotProblem {
 
 struct RotBatch {
   RotProblem p[kMaxBatch];
+  // optional (the INT4 linear that follows then waits per linear, not for the
+  // whole grid): CTA 0 writes this launch's grid id to *tagword before the grid
+  // lets its dependents launch, and every CTA sets xflags[its index] to the
+  // same id once its rows of x~ are written
+  unsigned long long* tagword;
+  unsigned long long* xflags;
   int count;
   int total_ctas;
 };

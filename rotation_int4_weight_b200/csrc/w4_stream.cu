@@ -274,6 +274,10 @@ __device__ bool wait_flag(const unsigned long long* f, unsigned long long v) {
 // activation transform of one linear each, FU pairs per thread and round, and
 // publish a flag holding this launch's grid id once its x~ is written; the
 // INT4 CTAs request a linear's activations only after its flag.
+// FU < 0: the flag form: the transform ran in the launch just before, whose
+// grid id is in *b.tagword and whose CTAs publish flags; the INT4 CTAs request
+// a linear's activations once all its transform CTAs have published (and do
+// not wait for the whole launch).
 template <bool F16, int NT, int FU>
 __global__ void __launch_bounds__(Geo<NT>::W * 32, 1)
 w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ RotBatch rb, int* status,
@@ -284,6 +288,17 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   __shared__ __align__(8) uint64_t bars[W * D];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  // flag form: the preceding transform's grid id, read before this grid lets
+  // the next transform (which rewrites it) launch
+  __shared__ unsigned long long s_xtag;
+  if constexpr (FU < 0) {
+    if (threadIdx.x == 0) {
+      unsigned long long v;
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];\n" : "=l"(v) : "l"(b.tagword) : "memory");
+      s_xtag = v;
+    }
+    __syncthreads();
+  }
   // a programmatic dependent (the next call's transform) may start its table
   // fetches as SMs free up; it waits for this grid before touching its data
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
@@ -351,7 +366,9 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   }
   uint32_t szc[4] = {0u, 0u, 0u, 0u};  // scale and zero bits of the unit being computed
   if (n > 0) load_sz(meta[cc.pi], cc, g, t, szc);
-  if (pdl_wait) asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  // (the flag form orders everything after the transform's flags instead: the
+  // transform waited for the previous launch before it published any)
+  if (FU >= 0 && pdl_wait) asm volatile("griddepcontrol.wait;\n" ::: "memory");
   // the activations of the unit in slot s (with the slot's arrival; its codes
   // were requested without one)
   auto issue_x = [&](const Cur& c, int s) {
@@ -364,17 +381,24 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   // fused form (lane 0): linears whose x~ flag was seen, and slots whose
   // activations are still to be requested
   uint32_t xready = 0u, xpend = 0u;
-  const unsigned long long xtag = grid_tag();
+  unsigned long long xtag = 0;
+  if constexpr (FU > 0) xtag = grid_tag();
+  if constexpr (FU < 0) xtag = s_xtag;
   auto x_ready = [&](int pi, bool block) -> bool {
     if (FU == 0 || ((xready >> pi) & 1u)) return true;
-    bool seen;
-    if (block) {
-      seen = wait_flag(b.xflags + pi, xtag);
-      if (!seen) report_status(status, kStatusTimeout);
-    } else {
-      unsigned long long v;
-      asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];\n" : "=l"(v) : "l"(b.xflags + pi) : "memory");
-      seen = v == xtag;
+    const unsigned long long* f = FU > 0 ? b.xflags + pi : b.xflags + b.p[pi].xf_begin;
+    const int nf = FU > 0 ? 1 : b.p[pi].xf_count;
+    bool seen = true;
+#pragma unroll 1
+    for (int q = 0; q < nf && seen; ++q) {
+      if (block) {
+        seen = wait_flag(f + q, xtag);
+        if (!seen) report_status(status, kStatusTimeout);
+      } else {
+        unsigned long long v;
+        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];\n" : "=l"(v) : "l"(f + q) : "memory");
+        seen = v == xtag;
+      }
     }
     if (!seen) return false;
     // acquire the transform CTA's x~, then order the TMA reads after it
@@ -448,7 +472,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
       cur_next(meta, nx);
       load_sz(meta[nx.pi], nx, g, t, szn);
     }
-    if constexpr (FU > 0) {
+    if constexpr (FU != 0) {
       // the unit's activations were deferred: wait (bounded) for its linear's x~
       if (lane == 0 && ((xpend >> slot) & 1u)) {
         // (on a timeout the slot still gets its arrival, so that its phase
@@ -770,7 +794,7 @@ bool stream_supported(int M, int d_in, int d_out, const void* x, const void* qwe
 size_t stream_workspace_bytes(int max_m) {
   const int NT = max_m <= 8 ? 1 : 2;
   return round256((size_t)device_sm_count() * 2 * 8) + round256((size_t)device_sm_count() * 2 * (4 * NT * 32 * 4) * 4) +
-         round256((size_t)kMaxBatch * 8);
+         round256((size_t)kXFlagWords * 8);
 }
 
 cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* qw, const __half* const* sc,
@@ -833,6 +857,7 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
   out->xflags = reinterpret_cast<unsigned long long*>(
       static_cast<char*>(ws) + round256((size_t)sms * 2 * 8) +
       round256((size_t)sms * 2 * (4 * (maxM <= 8 ? 1 : 2) * 32 * 4) * 4));
+  out->tagword = out->xflags + kMaxBatch * kStreamMaxM;
   *nt_out = maxM <= 8 ? 1 : 2;
   return cudaSuccess;
 }
@@ -866,6 +891,30 @@ cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* s
     if (NT == 1) PARO_STREAM_LAUNCH(false, 1) else PARO_STREAM_LAUNCH(false, 2)
   }
 #undef PARO_STREAM_LAUNCH
+}
+
+cudaError_t launch_stream_flagged(const StreamBatch& b, int NT, int* status, cudaStream_t stream) {
+  const size_t smem = NT == 1 ? Geo<1>::SMEM : Geo<2>::SMEM;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(b.ctas);
+  cfg.blockDim = dim3((NT == 1 ? Geo<1>::W : Geo<2>::W) * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const RotBatch none{};
+  cudaError_t e;
+  if (NT == 1) {
+    e = cudaFuncSetAttribute(w4_stream_kernel<true, 1, -1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, w4_stream_kernel<true, 1, -1>, b, none, status, 1);
+  }
+  e = cudaFuncSetAttribute(w4_stream_kernel<true, 2, -1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, w4_stream_kernel<true, 2, -1>, b, none, status, 1);
 }
 
 // ---- fused form -----------------------------------------------------------------------

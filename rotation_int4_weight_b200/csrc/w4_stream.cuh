@@ -23,6 +23,7 @@ struct StreamProblem {
   long long unit_begin;        // first unit (one 64-row tile x one 128-column group) of this linear
   int M, d_in, d_out, G;       // G = d_in / 128
   int tiles;                   // ceil(d_out / 64)
+  int xf_begin, xf_count;      // flag form: the flags of this linear's transform CTAs
 };
 
 struct StreamBatch {
@@ -30,7 +31,9 @@ struct StreamBatch {
   long long total_units;
   unsigned long long* flags;     // two per CTA: its partials' publication flags (workspace)
   float* partials;               // two tile partials per CTA (workspace)
-  unsigned long long* xflags;    // fused form: one per linear, set when its x~ is written (workspace)
+  unsigned long long* xflags;    // fused form: one per linear, set when its x~ is written (workspace);
+                                 // flag form: one per CTA of the preceding transform launch
+  unsigned long long* tagword;   // flag form: the grid id of the preceding transform launch
   // CTAs 0 .. ctas_a - 1 split units [0, units_a) evenly and the others the rest
   // (the fused form gives the widest linear, whose x~ comes last, fewer units a
   // CTA); ctas_a = ctas, units_a = total_units is the even split
@@ -52,6 +55,14 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
                               int reserved_ctas = 0);
 cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* status, cudaStream_t stream,
                                 bool pdl_wait);
+// The flag form (fp16 x~ written by a transform launched just before with
+// flags, see RotBatch): instead of waiting for the whole transform launch, the
+// INT4 linear requests a linear's activations once all of that linear's
+// transform CTAs have published.  b.tagword, b.xflags and every problem's
+// xf_begin / xf_count must be set.
+cudaError_t launch_stream_flagged(const StreamBatch& b, int NT, int* status, cudaStream_t stream);
+// Workspace words of the flag form: the tag word and one flag per transform CTA.
+constexpr int kXFlagWords = kMaxBatch * kStreamMaxM + 1;
 
 // The fused form for one token per linear: the kernel's first rb.count CTAs
 // each run the activation transform of one linear (writing its fp16 x~, the
