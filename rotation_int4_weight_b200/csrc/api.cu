@@ -537,18 +537,24 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     // few tokens: the transform launch publishes a flag per CTA, and the INT4
     // launch after it requests a linear's x~ once that linear's transform CTAs
     // have all published, not when the whole transform launch is done
+    // The widest linear's units go last in the INT4 launch; its transform
+    // (the slowest) takes the transform launch's first CTAs, which get SMs first.
     widest_last();
+    paro::RotProblem rt[PARO_MAX_BATCH];
+    rt[0] = rp[n - 1];
+    for (int i = 0; i + 1 < n; ++i) rt[i + 1] = rp[i];
     paro::RotBatch rb;
     paro::StreamBatch sb;
     int R = 1, nt = 1;
-    e = paro::plan_rot_batch(rp, n, &rb, &R);
+    e = paro::plan_rot_batch(rt, n, &rb, &R);
     if (e == cudaSuccess) e = plan_stream(true, 0, &sb, &nt);
     if (e != cudaSuccess) return from_cuda(e, "batched decode plan");
     rb.tagword = sb.tagword;
     rb.xflags = sb.xflags;
     for (int i = 0; i < n; ++i) {
-      sb.p[i].xf_begin = rb.p[i].cta_begin;
-      sb.p[i].xf_count = (rb.p[i].M + R - 1) / R;
+      const paro::RotProblem& t = rb.p[i + 1 < n ? i + 1 : 0];
+      sb.p[i].xf_begin = t.cta_begin;
+      sb.p[i].xf_count = (t.M + t.rows - 1) / t.rows;
     }
     e = paro::launch_rot_batch(rb, R, true, status, s, true, true);
     if (e == cudaSuccess) e = paro::launch_stream_flagged(sb, nt, status, s);

@@ -50,8 +50,9 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
   while (pi + 1 < batch.count && (int)blockIdx.x >= batch.p[pi + 1].cta_begin) ++pi;
   const RotProblem& P = batch.p[pi];
   constexpr int U = UP > 0 ? UP : (R == 4 ? 2 : 4);
+  const int rp = P.rows > 0 && P.rows < R ? P.rows : R;
   const bool done = rotdec::rot_decode_cta<R, F16OUT, U, kRotThreads>(
-      P, ((int)blockIdx.x - P.cta_begin) * R, smem, bars, status, pdl_wait != 0);
+      P, ((int)blockIdx.x - P.cta_begin) * rp, smem, bars, status, pdl_wait != 0);
   if (batch.xflags && done) {
     // every thread's x~ stores, then this CTA's flag
     __threadfence();
@@ -74,21 +75,26 @@ cudaError_t plan_rot_batch(const RotProblem* probs, int count, RotBatch* out, in
   if (count < 1 || count > kMaxBatch) return cudaErrorInvalidValue;
   int maxM = 0;
   for (int i = 0; i < count; ++i) maxM = probs[i].M > maxM ? probs[i].M : maxM;
-  int R = maxM >= 4 ? 4 : (maxM >= 2 ? 2 : 1);
-  // the widest problem must still hold its rows and two stages (one copy in
-  // flight while the other is used)
-  for (int i = 0; i < count; ++i)
-    while (R > 1 && rot_smem(probs[i].d, R, probs[i].K > 1 ? 2 : 1) > kRotSmemBudget) R >>= 1;
+  const int R = maxM >= 4 ? 4 : (maxM >= 2 ? 2 : 1);
   *out = RotBatch{};
   int ctas = 0;
   for (int i = 0; i < count; ++i) {
     RotProblem p = probs[i];
+    // rows a CTA for this problem: as many as R while its rows and min(K, 3)
+    // stages of tables fit.  A stage's rotation is shorter than the refill of
+    // a table slot (issued when the slot frees), so a wide problem with a
+    // shallower ring would wait on its tables every stage; it takes fewer rows
+    // (more CTAs) instead.
+    const int want = p.K < 1 ? 1 : (p.K < 3 ? p.K : 3);
+    int rows = R;
+    while (rows > 1 && rot_smem(p.d, rows, want) > kRotSmemBudget) rows >>= 1;
     int ring = p.K < 1 ? 1 : p.K;
     if (ring > 8) ring = 8;
-    while (ring > 1 && rot_smem(p.d, R, ring) > kRotSmemBudget) --ring;
+    while (ring > 1 && rot_smem(p.d, rows, ring) > kRotSmemBudget) --ring;
+    p.rows = rows;
     p.ring = ring;
     p.cta_begin = ctas;
-    ctas += (p.M + R - 1) / R;
+    ctas += (p.M + rows - 1) / rows;
     out->p[i] = p;
   }
   out->count = count;
@@ -101,7 +107,8 @@ cudaError_t launch_rot_batch(const RotBatch& b, int R, bool f16_out, int* status
                              bool pdl_trigger, bool pdl_wait) {
   size_t smem = 0;
   for (int i = 0; i < b.count; ++i) {
-    const size_t s = rot_smem(b.p[i].d, R, b.p[i].ring);
+    const int rows = b.p[i].rows > 0 && b.p[i].rows < R ? b.p[i].rows : R;
+    const size_t s = rot_smem(b.p[i].d, rows, b.p[i].ring);
     smem = s > smem ? s : smem;
   }
   const int trig = pdl_trigger ? 1 : 0, wait = pdl_wait ? 1 : 0;

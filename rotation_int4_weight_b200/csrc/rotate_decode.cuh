@@ -17,6 +17,7 @@ struct RotProblem {
   const float* sin_t;     // [K][d/2]
   const float* scale;     // [d] or null
   // filled by plan_rot_batch
+  int rows;               // token rows a CTA (<= the launch's R; 0 means R)
   int ring;               // stages of tables held in shared memory at once
   int cta_begin;          // first CTA of this problem
 };

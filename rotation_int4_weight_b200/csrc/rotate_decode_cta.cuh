@@ -63,8 +63,9 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 }
 
 
-// Transforms rows row0 .. row0 + R - 1 of problem P with NTHR threads; smem
-// holds d R 4 + ring 6 d bytes (16-byte aligned), bars kRotMaxRing mbarriers.
+// Transforms rows row0 .. row0 + RP - 1 of problem P with NTHR threads, RP =
+// P.rows (at most R; 0 means R); smem holds d RP 4 + ring 6 d bytes (16-byte
+// aligned), bars kRotMaxRing mbarriers.
 // Returns true when the rows were written (uniform over the CTA).
 template <int R, bool F16OUT, int U, int NTHR>
 __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, unsigned char* smem, uint64_t* bars,
@@ -72,13 +73,14 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
   constexpr int kProd = NTHR - 32;  // the table-fetching thread (lane 0 of the last warp)
   constexpr int kComp = NTHR - 32;  // rotating threads
   const int d = P.d, K = P.K, half = d >> 1, ring = P.ring;
-  const int nrows = min(R, P.M - row0);
+  const int RP = P.rows > 0 && P.rows < R ? P.rows : R;  // row planes (uniform)
+  const int nrows = min(RP, P.M - row0);
   const int tid = threadIdx.x;
 
-  // shared memory: xs [R][d] fp32 (one plane per row: channel c in bank c % 32) |
+  // shared memory: xs [RP][d] fp32 (one plane per row: channel c in bank c % 32) |
   // ring [ring][6d] of stage tables
   float* xs = reinterpret_cast<float*>(smem);
-  unsigned char* tab = reinterpret_cast<unsigned char*>(xs + (size_t)d * R);
+  unsigned char* tab = reinterpret_cast<unsigned char*>(xs + (size_t)d * RP);
   const size_t stage_bytes = (size_t)6 * d;  // pairs | cos | sin
   const uint32_t s_tab = static_cast<uint32_t>(__cvta_generic_to_shared(tab));
   const uint32_t s_bar = static_cast<uint32_t>(__cvta_generic_to_shared(bars));
@@ -135,7 +137,7 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
       if (cp < half) {
 #pragma unroll
         for (int r = 0; r < R; ++r)
-          *reinterpret_cast<float2*>(xs + (size_t)r * d + 2 * cp) = __bfloat1622float2(v[q][r]);
+          if (r < RP) *reinterpret_cast<float2*>(xs + (size_t)r * d + 2 * cp) = __bfloat1622float2(v[q][r]);
       }
     }
   }
@@ -177,8 +179,13 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
           if (ii[u] >= 0) {
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-              a[u][r] = xs[(size_t)r * d + ii[u]];
-              b[u][r] = xs[(size_t)r * d + jj[u]];
+              if (r < RP) {
+                a[u][r] = xs[(size_t)r * d + ii[u]];
+                b[u][r] = xs[(size_t)r * d + jj[u]];
+              } else {
+                a[u][r] = 0.f;
+                b[u][r] = 0.f;
+              }
             }
           }
 #pragma unroll
@@ -192,8 +199,10 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
             }
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-              xs[(size_t)r * d + ii[u]] = na[r];
-              xs[(size_t)r * d + jj[u]] = nb[r];
+              if (r < RP) {
+                xs[(size_t)r * d + ii[u]] = na[r];
+                xs[(size_t)r * d + jj[u]] = nb[r];
+              }
             }
           }
       }

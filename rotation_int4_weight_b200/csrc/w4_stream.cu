@@ -972,6 +972,7 @@ cudaError_t plan_fused_rot(const RotProblem* probs, int count, RotBatch* out) {
     RotProblem p = probs[i];
     int ring = p.K < 1 ? 1 : (p.K > rotdec::kRotMaxRing ? rotdec::kRotMaxRing : p.K);
     while (ring > 1 && fused_rot_smem(p.d, ring) > kFusedSmemBudget) --ring;
+    p.rows = 1;
     p.ring = ring;
     p.cta_begin = i;
     out->p[i] = p;
