@@ -54,6 +54,22 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     if (clock64() - t0 > (1LL << 31)) return false;
   return true;
 }
+// plain shared-memory accesses at 32-bit shared-window addresses (volatile:
+// they keep their order with each other; the stage barrier orders them with
+// everything else)
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+  asm volatile("st.shared.f32 [%0], %1;\n" ::"r"(a), "f"(v) : "memory");
+}
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, size_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"((uint32_t)bytes) : "memory");
 }
@@ -152,58 +168,56 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
   int issued = ring < K ? ring : K;    // stages requested so far (producer)
 
   // K stages.  The pairs of a stage are disjoint, so the loads of a batch of
-  // pairs may all be issued before any of its stores.
+  // pairs may all be issued before any of its stores.  Addresses are 32-bit
+  // shared-window offsets worked out once; a channel index outside 0..d-1 is
+  // clamped into range (so every access stays inside the rows) and reported
+  // once (PARO_ERR_INVALID_ARG) after the stages, the result then being void.
+  const uint32_t s_xs = static_cast<uint32_t>(__cvta_generic_to_shared(xs));
+  const uint32_t ud = (uint32_t)d, plane = 4u * ud;
+  uint32_t slot_off = 0;  // this stage's ring slot, bytes from s_tab
+  bool bad = false;
 #pragma unroll 1
   for (int k = 0; k < K && !failed; ++k) {
     if (tid < kComp) {
-      const unsigned char* st = tab + (size_t)(k % ring) * stage_bytes;
-      const uint32_t* pk = reinterpret_cast<const uint32_t*>(st);
-      const float* ck = reinterpret_cast<const float*>(st + 2 * d);
-      const float* sk = reinterpret_cast<const float*>(st + 4 * d);
+      const uint32_t st = s_tab + slot_off;
       for (int t0 = tid; t0 < half; t0 += U * kComp) {
-        int ii[U], jj[U];
+        uint32_t ai[U], aj[U];
         float c[U], sn[U], a[U][R], b[U][R];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int t = t0 + u * kComp;
-          ii[u] = -1;
           if (t < half) {
-            const uint32_t pr = pk[t];
-            const int i = pr & 0xFFFF, j = pr >> 16;
-            if (i < d && j < d) { ii[u] = i; jj[u] = j; c[u] = ck[t]; sn[u] = sk[t]; }
-            else report_status(status, kStatusBadIndex);
+            const uint32_t off = st + 4u * (uint32_t)t;
+            const uint32_t pr = lds_u32(off);
+            c[u] = lds_f32(off + 2u * ud);
+            sn[u] = lds_f32(off + 4u * ud);
+            uint32_t i = pr & 0xFFFFu, j = pr >> 16;
+            bad |= (i >= ud) | (j >= ud);
+            i = min(i, ud - 1u);
+            j = min(j, ud - 1u);
+            ai[u] = s_xs + 4u * i;
+            aj[u] = s_xs + 4u * j;
           }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u)
-          if (ii[u] >= 0) {
+          if (t0 + u * kComp < half) {
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
+            for (int r = 0; r < R; ++r)
               if (r < RP) {
-                a[u][r] = xs[(size_t)r * d + ii[u]];
-                b[u][r] = xs[(size_t)r * d + jj[u]];
-              } else {
-                a[u][r] = 0.f;
-                b[u][r] = 0.f;
+                a[u][r] = lds_f32(ai[u] + r * plane);
+                b[u][r] = lds_f32(aj[u] + r * plane);
               }
-            }
           }
 #pragma unroll
         for (int u = 0; u < U; ++u)
-          if (ii[u] >= 0) {
-            float na[R], nb[R];
+          if (t0 + u * kComp < half) {
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-              na[r] = fmaf(c[u], a[u][r], sn[u] * b[u][r]);
-              nb[r] = fmaf(-sn[u], a[u][r], c[u] * b[u][r]);
-            }
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
+            for (int r = 0; r < R; ++r)
               if (r < RP) {
-                xs[(size_t)r * d + ii[u]] = na[r];
-                xs[(size_t)r * d + jj[u]] = nb[r];
+                sts_f32(ai[u] + r * plane, fmaf(c[u], a[u][r], sn[u] * b[u][r]));
+                sts_f32(aj[u] + r * plane, fmaf(-sn[u], a[u][r], c[u] * b[u][r]));
               }
-            }
           }
       }
     } else if (tid == kProd && ring > 1) {
@@ -215,6 +229,8 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
       if (k + 1 < K) ok = mbar_wait_bounded(s_bar + 8u * ((k + 1) % ring), (uint32_t)(((k + 1) / ring) & 1));
     }
     failed = __syncthreads_or(!ok);
+    slot_off += (uint32_t)stage_bytes;
+    if (slot_off == (uint32_t)(ring * stage_bytes)) slot_off = 0;
     if (ring == 1 && k + 1 < K && !failed) {
       if (tid == kProd) {
         issue_stage(k + 1);
@@ -224,6 +240,7 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
       failed = __syncthreads_or(!ok);
     }
   }
+  if (bad) report_status(status, kStatusBadIndex);
   if (failed) {
     // a stage never arrived: report, let the latest copy of every slot land
     // (each wait bounded again), then leave
