@@ -41,14 +41,14 @@ METRIC = "rot+W4 linear: decode HBM GB/s (% peak), prefill TFLOP/s, rotation ove
 # DRAM bytes (read + write) per launch of the kernel the roofline times, from
 # one ncu capture of `bench.py --profile --variants batched_plain --config N`
 # (metrics dram__bytes_read.sum, dram__bytes_write.sum; the first launch after
-# four skipped; profiles/int4_linear_traffic.md), with the sha256 prefix
+# four skipped), with the sha256 prefix
 # of the kernel's sources at capture time: once the sources change, the figure
 # no longer describes the kernel and the bench reports null.
 TRAFFIC = {
-    1: {"bytes": 24964864, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "eba64dc696a0975c"},
-    2: {"bytes": 131877120 + 3483904, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "eba64dc696a0975c"},
+    1: {"bytes": 24964864, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "9f513bb1fda02648"},
+    2: {"bytes": 132190720 + 3635456, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "9f513bb1fda02648"},
     3: {"bytes": 346587136 + 137527040, "src": ("w4_tc.cu", "w4_tc.cuh"), "sha": "a093d18620409e5a"},
-    4: {"bytes": 25541888, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "eba64dc696a0975c"},
+    4: {"bytes": 25542400, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "9f513bb1fda02648"},
 }
 
 

@@ -31,14 +31,13 @@
 //
 // Partial sums.  A tile wholly inside one warp's units is written by that warp.
 // A tile split between warps of a CTA is summed in shared memory at the end, in
-// warp order.  A tile split between CTAs goes through the workspace: each CTA
-// writes its partial tile, then counts itself in on the tile's arrival counter;
-// the last to arrive sums the partials in CTA order and writes y.  The counter
-// is a 64-bit word holding (grid id, count): a word left by another launch, or
-// never initialised, is read as count 0, and the last arrival puts the count
-// back to 0, so the workspace needs no clearing between calls.  No thread ever
-// waits for another CTA, and every sum has a fixed order (the result does not
-// depend on timing).
+// warp order.  A tile split between CTAs goes through the workspace: every CTA
+// holding part of it but the last writes its partial tile and then a flag
+// holding this launch's grid id (a flag left by another launch, or never
+// written, never matches, so the workspace needs no clearing between calls);
+// the tile's last CTA waits (bounded) for the flags of the earlier CTAs, which
+// were launched no later than it, and sums the partials in CTA order.  Every
+// sum has a fixed order, so the result does not depend on timing.
 #include "paro_internal.cuh"
 #include "w4_stream.cuh"
 #include "rotate_decode_cta.cuh"
