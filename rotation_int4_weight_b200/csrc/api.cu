@@ -528,7 +528,7 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     e = paro::plan_fused_rot(rp, n, &rb);
     if (e == cudaSuccess) e = plan_stream(true, rb.count, &sb, &nt);
     if (e == cudaSuccess) {
-      paro::set_fused_split(sb);
+      paro::set_fused_split(sb, 0.4);
       e = paro::launch_fused_batch(sb, rb, status, s, true);
     }
     return from_cuda(e, "batched fused launch");
@@ -556,6 +556,11 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
       sb.p[i].xf_begin = t.cta_begin;
       sb.p[i].xf_count = (t.M + t.rows - 1) / t.rows;
     }
+    // With a long INT4 share per CTA (at least 96 units: Llama-3-8B's layer
+    // has about 180, Qwen2.5-1.5B's 39), the CTAs of the widest linear, whose
+    // transform ends last, take fewer units (measured at 8 and 16 tokens:
+    // Llama 54.3 -> 50.9 and 86.7 -> 79.5 us; Qwen's stack would lose 0.9 %).
+    if (sb.total_units >= 96LL * sb.ctas) paro::set_fused_split(sb, 0.9);
     e = paro::launch_rot_batch(rb, R, true, status, s, true, true);
     if (e == cudaSuccess) e = paro::launch_stream_flagged(sb, nt, status, s);
     return from_cuda(e, "batched decode launch");

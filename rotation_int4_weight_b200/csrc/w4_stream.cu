@@ -933,7 +933,7 @@ int fused_u(const RotBatch& rb) {
 }
 }  // namespace
 
-void set_fused_split(StreamBatch& b) {
+void set_fused_split(StreamBatch& b, double late) {
   b.ctas_a = b.ctas;
   b.units_a = b.total_units;
   if (b.count < 2 || b.ctas < 4) return;
@@ -944,7 +944,7 @@ void set_fused_split(StreamBatch& b) {
   // units a CTA of the last linear gets, relative to the others: the later its
   // x~ comes (the wider it is than the rest), the fewer (fitted to the arrival
   // times of the transforms on B200 for Qwen2.5-1.5B and Llama-3-8B layers)
-  const double rho = 1.0 - 0.4 * (double)(wide - other) / wide;
+  const double rho = 1.0 - late * (double)(wide - other) / wide;
   const long long UA = b.p[b.count - 1].unit_begin, UB = b.total_units - UA;
   long long CA = (long long)((double)b.ctas / (1.0 + (double)UB / (rho * (double)UA)) + 0.5);
   CA = CA < 1 ? 1 : (CA > b.ctas - 1 ? b.ctas - 1 : CA);

@@ -75,8 +75,9 @@ bool fused_supported(const RotProblem* probs, int count);
 // When the last linear is at least 1.5 times wider than any other, its
 // transform finishes last: its units go to a separate group of CTAs with
 // proportionally fewer units each, so that those CTAs, which start late,
-// finish with the others.
-void set_fused_split(StreamBatch& b);
+// finish with the others.  A CTA of the last linear gets 1 - late (w - o) / w
+// of the others' share (w, o: the widest and the next widest d_in).
+void set_fused_split(StreamBatch& b, double late);
 cudaError_t plan_fused_rot(const RotProblem* probs, int count, RotBatch* out);
 cudaError_t launch_fused_batch(const StreamBatch& b, const RotBatch& rb, int* status, cudaStream_t stream,
                                bool pdl_wait);
