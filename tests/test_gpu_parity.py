@@ -385,6 +385,44 @@ def test_stream_decode_matches_oracle_and_repeats_bit_exactly(shapes_m, rotate):
         assert torch.equal(f.view(torch.int16), d["y"].view(torch.int16))
 
 
+def test_stream_decode_full_size_llama_layer_split():
+    """The seven Llama-3-8B-shaped linears at 8 tokens in one batched call: the
+    two-launch decode path (transform CTAs publish per-CTA flags, the INT4
+    launch waits per linear) with the widest linear's units on CTAs of their
+    own, since the layer gives every CTA a long INT4 share.  Sampled output
+    columns against the oracle, then a repeat that must give the same bits."""
+    M = 8
+    probs, devs = [], []
+    for p in config_problems(2, M=M):
+        tables = dev_tables(p)
+        qw, sc, z = paro.paro_pack_weights(torch.from_numpy(p.W).to(DEV), *tables)
+        p.W = None  # the host weights are not needed again
+        y = torch.full((M, p.d_out), float("nan"), dtype=torch.bfloat16, device=DEV)
+        probs.append(p)
+        devs.append(dict(x=dev_x(p.x), tables=tables, qw=qw, sc=sc, z=z, y=y))
+    layers = [paro.paro_linear(d["x"], *d["tables"], d["qw"], d["sc"], d["z"], d["y"]) for d in devs]
+    ws = paro.paro_rotate_w4_linear_batched(layers)
+    torch.cuda.synchronize()
+    assert paro.paro_get_device_status() == 0
+    first = [d["y"].clone() for d in devs]
+    rng = np.random.default_rng(5)
+    for p, d in zip(probs, devs):
+        got = host(d["y"])
+        assert np.isfinite(got).all(), p.name
+        cols = np.sort(rng.choice(p.d_out, size=128, replace=False))
+        qwn, scn, zn = to_np_pack(d["qw"], d["sc"], d["z"])
+        ref = oracle.linear(oracle.rotate(p.x, p.pairs, p.cos_t, p.sin_t, p.scale),
+                            oracle.dequantize(qwn[cols], scn[cols], zn[cols]))
+        assert_linear_close(got[:, cols], ref)
+    for d in devs:
+        d["y"].fill_(float("nan"))
+    paro.paro_rotate_w4_linear_batched(layers, workspace=ws)
+    torch.cuda.synchronize()
+    assert paro.paro_get_device_status() == 0
+    for f, d in zip(first, devs):
+        assert torch.equal(f.view(torch.int16), d["y"].view(torch.int16))
+
+
 # ---------------------------------------------------------------- fused decode (one token per linear)
 # With every linear at M = 1 the batched call runs the transforms in the INT4
 # kernel's first CTAs (one per linear), which publish x~ with a flag that the
