@@ -220,16 +220,18 @@ typedef struct {
  * transformed activations of every linear (paro_workspace_bytes(M, d_in)
  * each, in order), then, when every M is at most 16, the publication flags
  * and partial sums of the stream-K INT4 linear (2 flags and 2 partial
- * 64-row tiles per SM, and one flag per linear for the fused form below).
+ * 64-row tiles per SM) and the flags of the transform's CTAs (at most 128,
+ * plus a tag word) that the INT4 linear waits on (see below).
  * The second part is optional: given only the first, the call runs the older
  * per-block kernel.
  */
 PARO_API size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int count);
 
 /*
- * Runs paro_rotate_w4_linear for up to PARO_MAX_BATCH independent linears with
- * at most two kernel launches in all (one transform launch, one INT4-linear
- * launch), e.g. the seven linears of one decoder layer; each linear has its own
+ * Runs paro_rotate_w4_linear for up to PARO_MAX_BATCH independent linears,
+ * e.g. the seven linears of one decoder layer, with one transform launch and
+ * one INT4-linear launch up to 64 tokens (one launch in all at one token per
+ * linear; one transform launch per linear beyond 64); each linear has its own
  * transform ("one rotation operator plus one group-wise INT4 GEMM operator for
  * each layer", page "ParoQuant: pairwise rotations that survive deployment",
  * section "From fake quantization to a real TensorRT engine").  h_layers is a
@@ -248,7 +250,10 @@ PARO_API size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int co
  * one token (M == 1) and the full workspace is given, the call is one launch:
  * its first CTAs transform one linear each into the workspace and publish a
  * flag, and the INT4 CTAs request a linear's activations once its flag is set
- * (each linear's arithmetic waits for its own transform only).
+ * (each linear's arithmetic waits for its own transform only).  With 2 to 16
+ * tokens the transform launch's CTAs each publish such a flag, and the INT4
+ * launch after it requests a linear's activations once all of that linear's
+ * transform CTAs have published, not when the whole transform launch is done.
  * The stream-K kernel's publication flags need no clearing: a flag holds the
  * id of the launch that wrote it, so one left by another launch, or never
  * written, is never taken for this launch's.  Two calls that may run at the
