@@ -51,8 +51,16 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
   const RotProblem& P = batch.p[pi];
   constexpr int U = UP > 0 ? UP : (R == 4 ? 2 : 4);
   const int rp = P.rows > 0 && P.rows < R ? P.rows : R;
-  const bool done = rotdec::rot_decode_cta<R, F16OUT, U, kRotThreads>(
-      P, ((int)blockIdx.x - P.cta_begin) * rp, smem, bars, status, pdl_wait != 0);
+  const int row0 = ((int)blockIdx.x - P.cta_begin) * rp;
+  bool done;
+  if (R > 1 && rp == 1) {
+    // a linear too wide for more than one row a CTA (its stage tables need the
+    // room): the one-row body, whose registers allow 7 pairs a thread and
+    // round, so a stage of up to 13888 channels is one round, not several
+    done = rotdec::rot_decode_cta<1, F16OUT, 7, kRotThreads>(P, row0, smem, bars, status, pdl_wait != 0);
+  } else {
+    done = rotdec::rot_decode_cta<R, F16OUT, U, kRotThreads>(P, row0, smem, bars, status, pdl_wait != 0);
+  }
   if (batch.xflags && done) {
     // every thread's x~ stores, then this CTA's flag
     __threadfence();
