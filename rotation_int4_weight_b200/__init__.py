@@ -234,7 +234,8 @@ def paro_batched_workspace_bytes(layers) -> int:
 
 
 def paro_rotate_w4_linear_batched(layers, *, workspace=None, group_size: int = 128, stream=None):
-    """Run a list of ParoLinear descriptions (at most 8) with two kernel launches."""
+    """Run a list of ParoLinear descriptions (at most 8): one launch at one token
+    per linear, a transform launch and an INT4-linear launch up to 64 tokens."""
     arr = (ParoLinear * len(layers))(*layers)
     need = int(lib.paro_batched_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), len(layers)))
     if workspace is None:
