@@ -30,9 +30,11 @@
  *   - Pair tables: uint16_t pairs[K][d/2][2]; stage k = 0 (R_1) is applied
  *     first; each stage must be a set of disjoint pairs covering channels
  *     0..d-1 (a perfect matching).  Kernels check that every index is < d; an
- *     out-of-range index is skipped and reported through
- *     paro_get_device_status().  Repeated channels inside a stage are not
- *     detected and give unspecified (but in-bounds) results.
+ *     out-of-range index never addresses memory (its pair is skipped, or the
+ *     index is clamped into range) and is reported through
+ *     paro_get_device_status(), and that call's results are void.  Repeated
+ *     channels inside a stage are not detected and give unspecified (but
+ *     in-bounds) results.
  *   - cos_t[K][d/2], sin_t[K][d/2] (fp32) hold cos and sin of each pair's
  *     angle; scale[d] (fp32, > 0) is the channel scale s, NULL meaning s = 1.
  *   - Packed weights (layout version 1): qweight uint32 [d_out][d_in/8], the
