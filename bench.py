@@ -425,10 +425,7 @@ def oracle_run(probs, idx, rows=None):
     return time.perf_counter() - t0, linear_bytes(p.d_in, r, p.M)
 
 
-def oracle_sample(config, M, seconds=12.0):
-    """Time the fp64 CPU oracle over whole passes of one unit's linears for about
-    `seconds`; returns (GB/s, threads, description)."""
-    probs, sub_m, M = oracle_problems(config, M)
+def _oracle_passes(probs, seconds):
     tot_t, tot_b, reps = 0.0, 0, 0
     while tot_t < seconds or reps == 0:
         for i in range(len(probs)):
@@ -436,9 +433,26 @@ def oracle_sample(config, M, seconds=12.0):
             tot_t += t
             tot_b += b
         reps += 1
-    sample = (f"{reps} pass(es) over the {len(probs)} linears of one unit at M={sub_m}"
-              + (f" (workload M={M}; bytes counted for M={sub_m})" if sub_m != M else "") + f", {tot_t:.1f} s")
-    return tot_b / tot_t / 1e9, _oracle_threads(), sample
+    return tot_b / tot_t / 1e9, reps, tot_t
+
+
+def oracle_sample(config, M, seconds=12.0, one_core_seconds=None):
+    """Time the fp64 CPU oracle over whole passes of one unit's linears for about
+    `seconds` on all host threads; returns (GB/s, threads, description, one-core
+    figure).  With one_core_seconds, the same passes are timed again with the
+    numeric libraries held to one thread: (GB/s, description), else None."""
+    probs, sub_m, M = oracle_problems(config, M)
+    gbs, reps, tot_t = _oracle_passes(probs, seconds)
+    unit = (f" over the {len(probs)} linears of one unit at M={sub_m}"
+            + (f" (workload M={M}; bytes counted for M={sub_m})" if sub_m != M else ""))
+    sample = f"{reps} pass(es){unit}, {tot_t:.1f} s"
+    one = None
+    if one_core_seconds is not None:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            gbs1, reps1, t1 = _oracle_passes(probs, one_core_seconds)
+        one = (gbs1, f"{reps1} pass(es){unit}, one thread, {t1:.1f} s")
+    return gbs, _oracle_threads(), sample, one
 
 
 def reference_rows(probs, steps, warmup, seconds=60.0):
@@ -658,9 +672,11 @@ def main():
                            "kernel": "INT4 linear, 2*M*d_in*d_out / device time",
                            "peak_kind": f"{peak_kind} bf16 dense (f16 operands: same nominal rate)"}
     if rank == 0 and not args.no_cpu:
-        gbs, cores, sample = oracle_sample(args.config, args.M)
+        gbs, cores, sample, one = oracle_sample(args.config, args.M, one_core_seconds=4.0)
         out["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                               "sample": sample}
+                               "sample": sample,
+                               "one_core": {"value": round(one[0], 4), "unit": "GB/s", "cores": 1,
+                                            "sample": one[1]}}
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
