@@ -668,6 +668,8 @@ def main():
         out["roofline"] = {"bound": "tensor", "achieved": round(tf, 2) if tf else None,
                            "peak": bf16, "unit": "TFLOP/s",
                            "frac": round(tf / bf16, 4) if tf else None, "traffic": traffic,
+                           "peak_sustained": bf16_sus,
+                           "frac_of_sustained": round(tf / bf16_sus, 4) if tf and bf16_sus else None,
                            "algorithmic_bytes_per_launch": int(bytes_of("plain") / w4_launches),
                            "kernel": "INT4 linear, 2*M*d_in*d_out / device time",
                            "peak_kind": f"{peak_kind} bf16 dense (f16 operands: same nominal rate)"}
