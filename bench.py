@@ -10,9 +10,21 @@ every step streams its weights from HBM.
 value     = algorithmic HBM bytes of the step / step time  (GB/s, device clock)
 e2e       = the same with the per-step host->device copy of the inputs (pinned)
             and device->host copy of the outputs inside the timed region
-roofline  = the INT4 linear kernel alone, algorithmic bytes / its time, against
-            the measured HBM copy bandwidth
+roofline  = the step's dominant kernel (at one token per linear the step is a
+            single launch of the fused stream-K kernel), algorithmic bytes per
+            launch / its share of the timed region, against the measured HBM
+            copy bandwidth
+sub_records = the rest of the metric: the Llama-3-8B-shaped layer at 2048
+            tokens (TFLOP/s of the tensor-core INT4 linear, rotation overhead),
+            the 196-linear Qwen2.5-1.5B-shaped stack at 16 tokens, and the
+            Llama-3-8B-shaped layer at one token
 cpu_baseline = the fp64 CPU oracle on a bounded sample of the same workload
+
+Timing: every timed region is exactly --steps steps, replayed as CUDA graphs
+whose calls chain by programmatic dependent launch (all graphs launched once
+beforehand); the region is repeated back to back for at least a second (the
+headline) and the median repetition is reported, with SM clocks sampled over
+all repetitions.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..4] [--impl ours|reference]
 Multi-GPU (torchrun): every rank runs its own layers (weak scaling, no data-path
@@ -230,6 +242,9 @@ class Unit:
             # one token per linear: the transforms run inside the INT4 kernel (one
             # launch per call); otherwise a transform launch and an INT4 launch
             return (1 if all(l.M == 1 for l in self.lins) else 2) * len(self.calls)
+        if variant == "fused":
+            # the single-linear call at one token is the same one-launch form
+            return sum(1 if l.M == 1 else 2 for l in self.lins)
         return LAUNCHES[variant] * len(self.lins)
 
 
@@ -266,67 +281,115 @@ def build_layers(config, M, n_layers, rank, dev, plan=True):
     return layers
 
 
-def capture(torch, paro, units, variant):
-    """CUDA graphs of a variant: one per unit (a unit = the linears of one step)
-    and one that runs every unit once in order (a full cycle), so that the host
-    enqueues many steps per replay and never limits the device."""
+def warm_eager(torch, paro, units, variant):
+    """Run every unit of a variant once outside capture (library-side set-up,
+    first-launch costs), on a side stream, and wait for it."""
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        for unit in units:           # warm the launch path outside capture
+        for unit in units:
             unit.run(paro, variant)
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
-    per_unit = []
-    for unit in units:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+
+
+def capture_units(torch, paro, units, variant):
+    """One CUDA graph running the given units in order (their launches chain by
+    programmatic dependent launch inside the graph)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for unit in units:
             unit.run(paro, variant)
-        per_unit.append(g)
-    cycle = None
-    if len(units) > 1:
-        cycle = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(cycle):
-            for unit in units:
-                unit.run(paro, variant)
-    return per_unit, cycle
+    return g
 
 
-def _replay(graphs, first, count):
-    """Replay `count` steps starting at unit index `first` (mod the number of units)."""
-    per_unit, cycle = graphs
-    n = len(per_unit)
-    i = 0
-    while i < count and (first + i) % n != 0:
-        per_unit[(first + i) % n].replay()
-        i += 1
-    while cycle is not None and count - i >= n:
-        cycle.replay()
-        i += n
-    while i < count:
-        per_unit[(first + i) % n].replay()
-        i += 1
+def chained_plan(torch, paro, units, variant, steps):
+    """Graphs that run `steps` steps in unit order 0, 1, ..., L-1, 0, ... (L
+    units) in as few graph launches as possible: a full-cycle graph replayed
+    steps // L times, then a graph of the first steps % L units.  Returns (the
+    sequence of graph launches, the distinct graphs)."""
+    L = len(units)
+    warm_eager(torch, paro, units, variant)
+    full = capture_units(torch, paro, units, variant) if steps >= L else None
+    r = steps % L
+    rem = capture_units(torch, paro, units[:r], variant) if r else None
+    seq = [full] * (steps // L) + ([rem] if rem is not None else [])
+    return seq, [g for g in (full, rem) if g is not None]
 
 
-def time_graphs(torch, graphs, steps, warmup, dist=None):
-    """Run `warmup` untimed steps, then time exactly `steps` steps on the device
-    (CUDA events on the launching stream, barrier + synchronize on both sides).
-    Returns ms per step, the max over ranks."""
-    _replay(graphs, 0, warmup)
+def isolated_plan(torch, paro, units, variant, steps):
+    """One graph launch per step (no chaining across steps): every step waits
+    for the previous one to finish before its first kernel starts."""
+    warm_eager(torch, paro, units, variant)
+    per_unit = [capture_units(torch, paro, [u], variant) for u in units]
+    return [per_unit[i % len(units)] for i in range(steps)], per_unit
+
+
+def l2_bytes(torch):
+    try:
+        return int(torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size)
+    except Exception:  # pragma: no cover
+        return 126 * 2 ** 20
+
+
+class Timed:
+    """Device time of one variant: exactly `steps` steps per timed region,
+    bracketed by a barrier and a synchronize on both sides, timed with CUDA
+    events on the launching stream.  The region is repeated back to back
+    (the same count on every rank) until it has run for `min_seconds`; each
+    repetition's time is the max over ranks, and the median repetition is the
+    figure.  When `steps` steps move less than twice the L2 size, a buffer
+    larger than L2 is written between repetitions (outside the timing)."""
+
+    def __init__(self, median, lo, hi, reps, warmup_steps, l2):
+        self.ms, self.lo, self.hi, self.reps, self.warmup_steps, self.l2 = median, lo, hi, reps, warmup_steps, l2
+
+    def summary(self):
+        return {"ms_per_step": round(self.ms, 6), "reps": self.reps, "rep_min_ms": round(self.lo, 6),
+                "rep_max_ms": round(self.hi, 6), "l2": self.l2}
+
+
+def time_plan(torch, plan, steps, warmup, dist, step_bytes, min_seconds=0.25, flush=None):
+    seq, distinct = plan
+    for g in distinct:                 # every graph launched once before any timing
+        g.replay()
+    done = 0
+    while done < max(warmup, 1):       # at least `warmup` untimed steps
+        for g in seq:
+            g.replay()
+        done += steps
     torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
+    need_flush = flush is not None and steps * step_bytes < 2 * l2_bytes(torch)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    start.record()
-    _replay(graphs, warmup, steps)
-    end.record()
-    torch.cuda.synchronize()
-    ms = max_over_ranks(torch, dist, start.elapsed_time(end) / steps, "cuda")
+
+    def one():
+        if need_flush:
+            flush.zero_()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        start.record()
+        for g in seq:
+            g.replay()
+        end.record()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        return start.elapsed_time(end)
+
+    first = max_over_ranks(torch, dist, one(), "cuda")
+    n = max(3, min(2000, int(min_seconds * 1e3 / max(first, 1e-3)) + 1))
+    n = int(max_over_ranks(torch, dist, float(n), "cuda"))
+    reps = [one() for _ in range(n)]
     if dist is not None:
-        dist.barrier()
-    return ms
+        t = torch.tensor(reps, dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        reps = t.tolist()
+    per_step = sorted(r / steps for r in reps)
+    l2 = ("L2 flushed between repetitions (a 256 MB write)" if need_flush
+          else "each timed region streams more than twice the L2 size")
+    return Timed(statistics.median(per_step), per_step[0], per_step[-1], n, done, l2)
 
 
 class ClockSampler:
@@ -507,27 +570,120 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- main
+def bytes_of(step_lins, M, variant):
+    """Algorithmic bytes of one step of a variant (each table read once per call)."""
+    if variant in ("plain", "batched_plain"):
+        return sum(linear_bytes(l.d_in, l.d_out, M, rotate=False) for l in step_lins)
+    if variant == "rotate":
+        return sum(4 * M * l.d_in + TABLE_BYTES_PER_CH * l.d_in for l in step_lins)
+    if variant == "rotate_backward":
+        # x (bf16) and the upstream gradient in, dx out (fp32), the tables and
+        # the outputs dtheta, dscale; the per-block partial sums round trip
+        def bwd(l):
+            R = 4 if 8 * 4 * l.d_in <= 226 * 1024 else (2 if 8 * 2 * l.d_in <= 226 * 1024 else 1)
+            n = K_STAGES * l.d_in // 2 + l.d_in
+            return 10 * M * l.d_in + TABLE_BYTES_PER_CH * l.d_in + 4 * n + 2 * 4 * n * -(-M // R)
+        return sum(bwd(l) for l in step_lins)
+    return sum(linear_bytes(l.d_in, l.d_out, M, unfused=(variant == "unfused")) for l in step_lins)
+
+
+def run_workload(torch, paro, args, config, M_arg, variants, dist, rank, dev, flush, clock_variant=None,
+                 isolated=False, e2e=False, min_seconds=0.25):
+    """Build one workload, time its variants; returns a dict of results."""
+    name, shapes, M, n_layers, stack = workload(config, M_arg)
+    layers = build_layers(config, M, n_layers, rank, dev, plan=not args.no_plan)
+    torch.cuda.synchronize()
+    units = [Unit(sum(layers, []), paro)] if stack else [Unit(l, paro) for l in layers]
+    del layers
+    step_lins = units[0].lins
+    out = {"name": name, "M": M, "units": units, "step_lins": step_lins, "timed": {}, "clocks": None}
+    for v in variants:
+        plan = chained_plan(torch, paro, units, v, args.steps)
+        sb = bytes_of(step_lins, M, v)
+        if v == clock_variant:
+            with ClockSampler(_smi_id(torch)) as cs:
+                t = time_plan(torch, plan, args.steps, args.warmup, dist, sb, min_seconds=1.0, flush=flush)
+            out["clocks"] = cs.summary()
+        else:
+            t = time_plan(torch, plan, args.steps, args.warmup, dist, sb, min_seconds=min_seconds, flush=flush)
+        out["timed"][v] = t
+        del plan
+    if isolated:
+        plan = isolated_plan(torch, paro, units, "batched", args.steps)
+        out["isolated"] = time_plan(torch, plan, args.steps, args.warmup, dist, bytes_of(step_lins, M, "batched"),
+                                    min_seconds=min_seconds, flush=flush)
+        del plan
+    if e2e:
+        plan = chained_plan(torch, paro, units, "batched_e2e", args.steps)
+        out["e2e"] = time_plan(torch, plan, args.steps, args.warmup, dist, bytes_of(step_lins, M, "batched"),
+                               min_seconds=min_seconds, flush=flush)
+        del plan
+    return out
+
+
+def overhead(t, a, b):
+    return round(100 * (t[a].ms - t[b].ms) / t[b].ms, 2) if a in t and b in t else None
+
+
+def sub_record(r, world, hbm, bf16, bf16_sus):
+    """One workload's figures for the JSON line (value in its metric's unit)."""
+    t, M, lins = r["timed"], r["M"], r["step_lins"]
+    ms = t["batched"].ms
+    flops = sum(2 * M * l.d_in * l.d_out for l in lins)
+    prefill = M >= PREFILL_M
+    rec = {"workload": f"{r['name']}: fused rotate + INT4 linear, M={M}, K={K_STAGES}, group={GROUP}",
+           "linears_per_step": len(lins), "distinct_units_cycled": len(r["units"]),
+           "ms_per_step": round(ms, 6), "reps": t["batched"].reps, "l2": t["batched"].l2,
+           "rotation_overhead_pct": overhead(t, "batched", "batched_plain")}
+    if prefill:
+        tf = whole_job_rate(flops, world, ms) / 1e12
+        rec.update(value=round(tf, 2), unit="TFLOP/s", frac_of_bf16=round(tf / bf16, 4))
+        if "batched_plain" in t:
+            tp = flops / (t["batched_plain"].ms * 1e-3) / 1e12
+            rec["roofline"] = {"bound": "tensor", "kernel": "w4_tc_kernel (tcgen05; one launch per step, plain "
+                                                            "weights, bf16 inputs rounded to fp16 in the kernel)",
+                               "achieved": round(tp, 2), "peak": bf16, "unit": "TFLOP/s", "frac": round(tp / bf16, 4),
+                               "peak_sustained": bf16_sus,
+                               "frac_of_sustained": round(tp / bf16_sus, 4) if bf16_sus else None,
+                               "traffic": None}
+        if "rotate" in t:
+            gb = bytes_of(lins, M, "rotate") / (t["rotate"].ms * 1e-3) / 1e9
+            rec["rotate_kernel"] = {"gbs": round(gb, 1), "frac_of_hbm": round(gb / hbm, 4),
+                                    "ms_per_step": round(t["rotate"].ms, 6),
+                                    "what": "paro_rotate alone, one call per linear (bf16 in and out)"}
+    else:
+        gb = whole_job_rate(bytes_of(lins, M, "batched"), world, ms) / 1e9
+        rec.update(value=round(gb, 1), unit="GB/s", frac_of_hbm=round(gb / hbm, 4),
+                   tokens_per_s=round(M * world / (ms * 1e-3), 1))
+        if "batched_plain" in t:
+            gp = bytes_of(lins, M, "batched_plain") / (t["batched_plain"].ms * 1e-3) / 1e9
+            rec["int4_alone"] = {"gbs": round(gp, 1), "frac_of_hbm": round(gp / hbm, 4),
+                                 "ms_per_step": round(t["batched_plain"].ms, 6),
+                                 "what": "the same step on plain INT4 weights (no transform)"}
+    return rec
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=None,
-                    help="timed steps (default: enough for about half a second of device time)")
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20, help="steps per timed region")
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--M", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-sub", action="store_true", help="skip the prefill, stack and Llama decode sub-records")
     ap.add_argument("--variants", default="batched,batched_plain,fused,plain,unfused,rotate,rotate_backward")
     ap.add_argument("--no-plan", action="store_true",
                     help="use the pair tables as drawn instead of the conflict-free order of paro_plan_pair_order")
     ap.add_argument("--profile", action="store_true",
-                    help="run only the listed variants (no end-to-end leg, no CPU baseline): a fixed, short "
-                         "launch sequence for ncu; its numbers are not bench values")
+                    help="run only the listed variants once each (no repetitions, no end-to-end leg, no "
+                         "sub-records, no CPU baseline): a short launch sequence for ncu; not bench values")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.steps is None:
-        args.steps = {0: 20000, 1: 56000, 2: 8000, 3: 200, 4: 128}.get(args.config, 1000)
+    if args.steps < 1:
+        raise SystemExit("--steps must be >= 1")
     if args.impl == "reference":
         return run_reference(args)
 
@@ -548,131 +704,137 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     hbm, bf16, bf16_sus, peak_kind = peaks()
 
-    name, shapes, M, n_layers, stack = workload(args.config, args.M)
-    layers = build_layers(args.config, M, n_layers, rank, dev, plan=not args.no_plan)
-    torch.cuda.synchronize()
-    units = [Unit(sum(layers, []), paro)] if stack else [Unit(l, paro) for l in layers]
-    step_lins = units[0].lins
-    flops_step = sum(2 * M * l.d_in * l.d_out for l in step_lins)
-
-    def bytes_of(variant):
-        if variant == "plain":
-            return sum(linear_bytes(l.d_in, l.d_out, M, rotate=False) for l in step_lins)
-        if variant == "rotate":
-            return sum(4 * M * l.d_in + TABLE_BYTES_PER_CH * l.d_in for l in step_lins)
-        if variant == "rotate_backward":
-            # x (bf16) and the upstream gradient in, dx out (fp32), the tables and
-            # the outputs dtheta, dscale; the per-block partial sums round trip
-            def bwd(l):
-                R = 4 if 8 * 4 * l.d_in <= 226 * 1024 else (2 if 8 * 2 * l.d_in <= 226 * 1024 else 1)
-                n = K_STAGES * l.d_in // 2 + l.d_in
-                return 10 * M * l.d_in + TABLE_BYTES_PER_CH * l.d_in + 4 * n + 2 * 4 * n * -(-M // R)
-            return sum(bwd(l) for l in step_lins)
-        return sum(linear_bytes(l.d_in, l.d_out, M, unfused=(variant == "unfused")) for l in step_lins)
-
-    variants = [v for v in args.variants.split(",") if v]
-    if "batched" not in variants and not args.profile:
-        variants.insert(0, "batched")
-    results = {}
-    clocks = None
-    for v in variants:
-        graphs = capture(torch, paro, units, v)
-        if v == "batched" and not args.profile:
-            with ClockSampler(_smi_id(torch)) as cs:
-                ms = time_graphs(torch, graphs, args.steps, args.warmup, dist)
-            clocks = cs.summary()
-        else:
-            ms = time_graphs(torch, graphs, args.steps, args.warmup, dist)
-        results[v] = ms
-        del graphs
     if args.profile:
+        # a fixed, short launch sequence: each listed variant's chained graphs,
+        # warmed and then replayed once
+        name, shapes, M, n_layers, stack = workload(args.config, args.M)
+        layers = build_layers(args.config, M, n_layers, rank, dev, plan=not args.no_plan)
+        units = [Unit(sum(layers, []), paro)] if stack else [Unit(l, paro) for l in layers]
+        res = {}
+        for v in [v for v in args.variants.split(",") if v]:
+            seq, distinct = chained_plan(torch, paro, units, v, args.steps)
+            for _ in range(args.warmup):
+                for g in distinct:
+                    g.replay()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for g in seq:
+                g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            res[v] = a.elapsed_time(b) / args.steps
+            del seq, distinct
         if rank == 0:
-            print(json.dumps({"profile_run": True, "variants_ms_per_step": results}), flush=True)
+            print(json.dumps({"profile_run": True, "variants_ms_per_step": res}), flush=True)
         if dist is not None:
             dist.destroy_process_group()
         return
-    # end to end: per step the inputs come from pinned host memory and outputs go back
-    graphs = capture(torch, paro, units, "batched_e2e")
-    ms_e2e = time_graphs(torch, graphs, args.steps, args.warmup, dist)
-    del graphs
+
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    variants = [v for v in args.variants.split(",") if v]
+    if "batched" not in variants:
+        variants.insert(0, "batched")
+    head = run_workload(torch, paro, args, args.config, args.M, variants, dist, rank, dev, flush,
+                        clock_variant="batched", isolated=True, e2e=True)
+    t, M, step_lins, units = head["timed"], head["M"], head["step_lins"], head["units"]
+    ms = t["batched"].ms
+    step_bytes = bytes_of(step_lins, M, "batched")
+    flops_step = sum(2 * M * l.d_in * l.d_out for l in step_lins)
+    prefill = M >= PREFILL_M
+    value = (whole_job_rate(flops_step, world, ms) / 1e12 if prefill
+             else whole_job_rate(step_bytes, world, ms) / 1e9)
     h2d = units[0].x_all.numel() * 2
     d2h = units[0].y_all.numel() * 2
-
-    ms = results["batched"]
-    step_bytes = bytes_of("fused")
-    value = whole_job_rate(step_bytes, world, ms) / 1e9
-    e2e_value = whole_job_rate(step_bytes + h2d + d2h, world, ms_e2e) / 1e9
-    plain_ms = results.get("plain")
-    # dominant kernel: the INT4 linear, timed alone (plain weights, no transform:
-    # one launch per batched call when that variant ran, else one per linear)
-    w4_ms = results.get("batched_plain", plain_ms)
-    w4_gbs = bytes_of("plain") / (w4_ms * 1e-3) / 1e9 if w4_ms else None
-    # launches of the timed kernel per step (one per batched call), for the
-    # per-launch figures next to the captured traffic
-    w4_launches = units[0].launches("batched_plain") if "batched_plain" in results else len(step_lins)
-    traffic = measured_traffic(args.config, args.M)
-    rot_gbs = bytes_of("rotate") / (results["rotate"] * 1e-3) / 1e9 if "rotate" in results else None
-    bwd_ms = results.get("rotate_backward")
-    prefill = M >= PREFILL_M
-
+    ms_e2e = head["e2e"].ms
+    e2e_value = (whole_job_rate(flops_step, world, ms_e2e) / 1e12 if prefill
+                 else whole_job_rate(step_bytes + h2d + d2h, world, ms_e2e) / 1e9)
+    launches = units[0].launches("batched")
+    # the dominant kernel: at one token per linear the whole step is one launch
+    # of the stream-K kernel in its fused form (transform CTAs + INT4 CTAs);
+    # otherwise the INT4 launch, timed alone on plain weights
+    one_launch = launches == len(units[0].calls) and not prefill
+    if prefill:
+        kt = t.get("batched_plain", t["batched"])
+        ach = flops_step / (kt.ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 2), "peak": bf16, "unit": "TFLOP/s",
+                "frac": round(ach / bf16, 4), "traffic": measured_traffic(args.config, args.M),
+                "peak_sustained": bf16_sus, "frac_of_sustained": round(ach / bf16_sus, 4) if bf16_sus else None,
+                "kernel": "w4_tc_kernel, 2*M*d_in*d_out per launch / (timed region / launches)",
+                "peak_kind": f"{peak_kind} bf16 dense (f16 operands: same nominal rate)"}
+    else:
+        kv = "batched" if one_launch else "batched_plain"
+        kt = t.get(kv, t["batched"])
+        per_launch_bytes = bytes_of(step_lins, M, kv) / units[0].launches(kv)
+        per_launch_ms = kt.ms / units[0].launches(kv)
+        ach = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
+                "traffic": measured_traffic(args.config, args.M),
+                "algorithmic_bytes_per_launch": int(per_launch_bytes),
+                "kernel": ("w4_stream_kernel, fused form (one launch per step: transform CTAs and INT4 CTAs)"
+                           if one_launch else "w4_stream_kernel (INT4 linear, plain weights, one launch per "
+                                              "batched call)")
+                          + "; algorithmic bytes per launch / (timed region / launches)",
+                "peak_kind": f"{peak_kind} HBM copy bandwidth"}
+    plain_ms = t["plain"].ms if "plain" in t else None
+    iso = head["isolated"]
     out = {
         "metric": METRIC,
-        "value": round(value if not prefill else whole_job_rate(flops_step, world, ms) / 1e12, 3),
-        "unit": "GB/s" if not prefill else "TFLOP/s",
+        "value": round(value, 3),
+        "unit": "TFLOP/s" if prefill else "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {
-            "workload": f"{name}: fused rotate + INT4 linear (one batched C-ABI call per {BATCH} linears), "
+            "workload": f"{head['name']}: fused rotate + INT4 linear (one batched C-ABI call per {BATCH} linears), "
                         f"M={M}, K={K_STAGES}, group={GROUP}, asymmetric INT4, bf16 activations",
             "linears_per_step": len(step_lins), "distinct_units_cycled": len(units),
-            "l2": ("inputs larger than L2: each step streams a different layer's weights "
-                   f"({len(units)} units, {sum(bytes_of('fused') for _ in units) / 1e9:.2f} GB)") if len(units) > 1
-                  else "inputs larger than L2 per step" if step_bytes > 126e6 else "L2-resident (single unit)",
-            "graphs": "each step is one CUDA-graph replay of the step's C-ABI calls",
+            "timing": (f"each timed region is exactly {args.steps} steps, replayed as CUDA graphs of up to "
+                       f"{len(units)} steps whose calls chain by programmatic dependent launch; every graph is "
+                       f"launched before timing; the region is repeated {t['batched'].reps} times back to back "
+                       "(barrier + synchronize around each) and the median repetition is reported"),
+            "l2": t["batched"].l2,
             "pair_order": "as drawn" if args.no_plan else "paro_plan_pair_order (conflict-free; same transform)",
         },
-        "roofline": {
-            "bound": "hbm", "achieved": round(w4_gbs, 1) if w4_gbs else None, "peak": hbm, "unit": "GB/s",
-            "frac": round(w4_gbs / hbm, 4) if w4_gbs else None, "traffic": traffic,
-            "algorithmic_bytes_per_launch": int(bytes_of("plain") / w4_launches),
-            "kernel": ("w4_stream_kernel" if M <= 16 else "w4_gemv_kernel")
-                      + " (INT4 linear; one launch per batched call of a step's linears, timed alone "
-                        "with plain weights), algorithmic bytes / device time",
-            "peak_kind": f"{peak_kind} HBM copy bandwidth",
-        },
-        "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(ms_e2e, 6)},
-        "gpu_launches": units[0].launches("batched") * args.steps,
-        "clocks": clocks,
-        "variants_ms_per_step": {k: round(v, 6) for k, v in results.items()},
-        "rotation_overhead_pct": (round(100 * (ms - results["batched_plain"]) / results["batched_plain"], 2)
-                                  if "batched_plain" in results else None),
-        "rotation_overhead_vs_per_linear_plain_pct": round(100 * (ms - plain_ms) / plain_ms, 2) if plain_ms else None,
-        "rotation_overhead_unfused_pct": (round(100 * (results["unfused"] - plain_ms) / plain_ms, 2)
-                                          if plain_ms and "unfused" in results else None),
-        "rotation_overhead_per_linear_fused_pct": (round(100 * (results["fused"] - plain_ms) / plain_ms, 2)
-                                                   if plain_ms and "fused" in results else None),
-        "rotate_kernel_gbs": round(rot_gbs, 1) if rot_gbs else None,
-        "rotate_backward": ({"ms_per_step": round(bwd_ms, 6),
-                             "gbs": round(bytes_of("rotate_backward") / (bwd_ms * 1e-3) / 1e9, 1),
+        "roofline": roof,
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s" if prefill else "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 6),
+                "what": "per step: host->device copy of the step's inputs from pinned memory, the C-ABI call, "
+                        "device->host copy of its outputs, all inside the timed region"},
+        "gpu_launches": launches * args.steps,
+        "clocks": head["clocks"],
+        "timed_region": t["batched"].summary(),
+        "isolated_step": {"ms_per_step": round(iso.ms, 6),
+                          "value": round((flops_step / 1e12 if prefill else step_bytes / 1e9) / (iso.ms * 1e-3), 3),
+                          "what": "one graph launch per step, so no step overlaps the previous one"},
+        "variants_ms_per_step": {k: round(v.ms, 6) for k, v in t.items()},
+        "rotation_overhead_pct": overhead(t, "batched", "batched_plain"),
+        "rotation_overhead_unfused_pct": overhead(t, "unfused", "plain"),
+        "rotation_overhead_per_linear_fused_pct": overhead(t, "fused", "plain"),
+        "rotate_kernel_gbs": (round(bytes_of(step_lins, M, "rotate") / (t["rotate"].ms * 1e-3) / 1e9, 1)
+                              if "rotate" in t else None),
+        "rotate_backward": ({"ms_per_step": round(t["rotate_backward"].ms, 6),
+                             "gbs": round(bytes_of(step_lins, M, "rotate_backward")
+                                          / (t["rotate_backward"].ms * 1e-3) / 1e9, 1),
                              "what": "dL/dx, dL/dtheta, dL/ds of the step's transforms for a synthetic upstream "
-                                     "gradient (paro_rotate_backward, one call per linear)",
-                             "bound": "shared memory: each stage moves 8 B per element forward and 16 B back "
-                                      "(x and its gradient)"} if bwd_ms else None),
+                                     "gradient (paro_rotate_backward, one call per linear)"}
+                            if "rotate_backward" in t else None),
         "tokens_per_s": round(M * world / (ms * 1e-3), 1),
-        "tflops": round(flops_step * world / (ms * 1e-3) / 1e12, 3),
-        "hbm_frac_of_measured": round(value / hbm, 4),
+        "hbm_frac_of_measured": None if prefill else round(value / hbm, 4),
     }
-    if prefill:
-        tf = flops_step / (w4_ms * 1e-3) / 1e12 if w4_ms else None
-        out["roofline"] = {"bound": "tensor", "achieved": round(tf, 2) if tf else None,
-                           "peak": bf16, "unit": "TFLOP/s",
-                           "frac": round(tf / bf16, 4) if tf else None, "traffic": traffic,
-                           "peak_sustained": bf16_sus,
-                           "frac_of_sustained": round(tf / bf16_sus, 4) if tf and bf16_sus else None,
-                           "algorithmic_bytes_per_launch": int(bytes_of("plain") / w4_launches),
-                           "kernel": "INT4 linear, 2*M*d_in*d_out / device time",
-                           "peak_kind": f"{peak_kind} bf16 dense (f16 operands: same nominal rate)"}
+    del head, units, step_lins, t
+    torch.cuda.empty_cache()
+    if not args.no_sub and args.config == 1 and args.M is None:
+        subs = {}
+        for key, cfg, m, vs in [("prefill_llama_m2048", 3, None, "batched,batched_plain,rotate"),
+                                ("stack_qwen_196_linears_m16", 4, None, "batched,batched_plain"),
+                                ("decode_llama_m1", 2, 1, "batched,batched_plain")]:
+            r = run_workload(torch, paro, args, cfg, m, vs.split(","), dist, rank, dev, flush, min_seconds=0.5)
+            subs[key] = sub_record(r, world, hbm, bf16, bf16_sus)
+            if cfg == 4:
+                subs[key]["tokens_per_s_note"] = "one step = all 196 linears at 16 tokens"
+            del r
+            torch.cuda.empty_cache()
+        out["sub_records"] = subs
     if rank == 0 and not args.no_cpu:
         gbs, cores, sample, one = oracle_sample(args.config, args.M, one_core_seconds=4.0)
         out["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",

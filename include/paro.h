@@ -45,7 +45,8 @@
  *     d_in % 128 == 0 and group_size == 128 for the INT4 calls; d_out % 16 == 0;
  *     0 <= K <= 16; M >= 0 (M == 0 enqueues nothing and returns PARO_OK).
  *   - No exception crosses this boundary.  Calls are thread-safe; the only
- *     library state is one device status word per GPU.
+ *     library state is one device status word per GPU and the scratch array of
+ *     paro_rotate_w4_linear_noalloc.
  */
 #ifndef PARO_H
 #define PARO_H
@@ -176,7 +177,12 @@ PARO_API paro_status paro_w4_linear(const uint16_t* d_x, const uint32_t* d_qweig
 PARO_API paro_status paro_plan_pair_order(const uint16_t* h_pairs, const float* h_cos, const float* h_sin, int K,
                                           int d, uint16_t* h_pairs_out, float* h_cos_out, float* h_sin_out);
 
-/* Bytes of device workspace paro_rotate_w4_linear needs for M tokens of width d_in. */
+/*
+ * Bytes of device workspace paro_rotate_w4_linear takes for M tokens of width
+ * d_in: the fp16 transformed activations (2 M d_in rounded up to 256 bytes)
+ * and, for M <= 16, the flags and partial tiles of the stream-K INT4 kernel
+ * (about 8.2 KB per SM at 9-16 tokens, half that up to 8).
+ */
 PARO_API size_t paro_workspace_bytes(int M, int d_in);
 
 /*
@@ -187,7 +193,11 @@ PARO_API size_t paro_workspace_bytes(int M, int d_in);
  * activations never leave the GPU as bf16: they are handed to the linear in
  * fp16 through d_workspace (paro_workspace_bytes(M, d_in) bytes, 256-byte
  * aligned, caller-owned, contents undefined between calls; two calls that run
- * at the same time need two workspaces).
+ * at the same time need two workspaces).  Up to 16 tokens with that full
+ * workspace the call runs as paro_rotate_w4_linear_batched does for one
+ * linear (one launch at one token: its first CTA transforms while the others
+ * stream the weights); given only the activations' 2 M d_in bytes (rounded
+ * up to 256), it runs the transform and then the INT4 linear.
  * d_x: bf16 [M][d_in]; d_y: bf16 [M][d_out], not overlapping any input.
  */
 PARO_API paro_status paro_rotate_w4_linear(const uint16_t* d_x, int K, const uint16_t* d_pairs,
@@ -265,20 +275,27 @@ PARO_API paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, 
                                                   void* d_workspace, size_t workspace_bytes,
                                                   paro_stream_t stream);
 
+/* Bytes of the scratch array built into the library for the call below. */
+#define PARO_NOALLOC_SCRATCH_BYTES (2u << 20)
+
 /*
  * The same computation as paro_rotate_w4_linear for callers that cannot
  * allocate device memory (the paper has no counterpart: this is an interface
  * convenience of this library).  Instead of a caller-provided workspace, the
- * transformed activations go to a scratch array built into the library: every
- * GPU that loads libparo holds 512 KiB for it until the process exits, and
- * M * d_in may not exceed 262144 (PARO_ERR_UNSUPPORTED, nothing enqueued).
- * The call allocates nothing.  Its first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture.  All calls on a device
- * share the one array: calls that may overlap on the GPU (different streams,
- * or other work between them that is not ordered) race on it and must be
- * serialised by the caller.  Arguments, layouts and results are those of
- * paro_rotate_w4_linear.
+ * call uses a scratch array built into the library: every GPU that loads
+ * libparo holds PARO_NOALLOC_SCRATCH_BYTES (2 MiB) for it until the process
+ * exits.  M * d_in may not exceed 262144 (PARO_ERR_UNSUPPORTED, nothing
+ * enqueued).  The call allocates nothing and runs the same kernels as
+ * paro_rotate_w4_linear given a workspace of PARO_NOALLOC_SCRATCH_BYTES, so
+ * its results are bit-identical to that call's.  Its first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) with that device
+ * current and keeps it for the life of the process; make that first call
+ * before any stream capture, and do not call cudaDeviceReset on that device
+ * afterwards (the kept address would no longer be mapped).  All calls on a
+ * device share the one array: calls that may overlap on the GPU (different
+ * streams, or other work between them that is not ordered) race on it and
+ * must be serialised by the caller.  Arguments, layouts and results are those
+ * of paro_rotate_w4_linear.
  */
 PARO_API paro_status paro_rotate_w4_linear_noalloc(const uint16_t* d_x, int K, const uint16_t* d_pairs,
                                   const float* d_cos, const float* d_sin, const float* d_scale,
@@ -289,7 +306,11 @@ PARO_API paro_status paro_rotate_w4_linear_noalloc(const uint16_t* d_x, int K, c
 /*
  * Synchronises `stream`, then returns and clears the device status word of
  * the current GPU: PARO_OK, PARO_ERR_INVALID_ARG (a kernel met a pair index
- * >= d and skipped it) or PARO_ERR_TIMEOUT (a bounded wait gave up).
+ * >= d and skipped or clamped it: that call's results are void) or
+ * PARO_ERR_TIMEOUT (a bounded wait gave up: that call's results are void).
+ * The word's device address is looked up on the first call of the library on
+ * each device and kept for the life of the process, so cudaDeviceReset on a
+ * device after the library has used it is not supported.
  */
 PARO_API paro_status paro_get_device_status(paro_stream_t stream);
 

@@ -116,6 +116,20 @@ cudaError_t launch_linear(const uint16_t* x, bool x_f16, const uint32_t* qweight
     return paro::launch_w4_tc(x, x_f16, qweight, reinterpret_cast<const __half*>(scales),
                               reinterpret_cast<const __half*>(zeros), reinterpret_cast<__nv_bfloat16*>(y), M, d_in,
                               d_out, status, s);
+  if (M <= paro::kStreamMaxM && paro::stream_supported(M, d_in, d_out, x, qweight)) {
+    // few tokens: the TMA stream-K kernel, each CTA on whole 64-row tiles so
+    // that no partial sum crosses CTAs (this call has no workspace for them)
+    const uint16_t* xs[1] = {x};
+    const uint32_t* qs[1] = {qweight};
+    const __half* ss[1] = {reinterpret_cast<const __half*>(scales)};
+    const __half* zs[1] = {reinterpret_cast<const __half*>(zeros)};
+    __nv_bfloat16* ys[1] = {reinterpret_cast<__nv_bfloat16*>(y)};
+    paro::StreamBatch sb;
+    int nt = 1;
+    cudaError_t e = paro::plan_stream_batch(xs, qs, ss, zs, ys, &M, &d_in, &d_out, 1, x_f16, nullptr, &sb, &nt);
+    if (e != cudaSuccess) return e;
+    return paro::launch_stream_batch(sb, nt, x_f16, status, s, pdl_wait);
+  }
   paro::GemvProblem p = {};
   p.x = x;
   p.qw = qweight;
@@ -307,10 +321,19 @@ paro_status paro_w4_linear(const uint16_t* d_x, const uint32_t* d_qweight, const
   return from_cuda(e, "w4 linear launch");
 }
 
+namespace {
+// fp16 transformed activations of M tokens of width d_in, rounded up to 256 bytes
+size_t xt_bytes(int M, int d_in) {
+  if (M <= 0 || d_in <= 0) return 0;
+  const size_t b = (size_t)M * d_in * 2;
+  return (b + 255) & ~(size_t)255;
+}
+}  // namespace
+
 size_t paro_workspace_bytes(int M, int d_in) {
   if (M <= 0 || d_in <= 0) return 0;
-  const size_t b = (size_t)M * d_in * 2;  // fp16 transformed activations
-  return (b + 255) & ~(size_t)255;
+  // up to 16 tokens, also the stream-K kernel's flags and partial tiles
+  return xt_bytes(M, d_in) + (M <= paro::kStreamMaxM ? paro::stream_workspace_bytes(M) : 0);
 }
 
 paro_status paro_rotate_w4_linear(const uint16_t* d_x, int K, const uint16_t* d_pairs,
@@ -327,16 +350,39 @@ paro_status paro_rotate_w4_linear(const uint16_t* d_x, int K, const uint16_t* d_
   if ((st = check_weights(d_qweight, d_scales, d_zeros)) != PARO_OK) return st;
   if (!d_x || !d_y) return fail(PARO_ERR_INVALID_ARG, "null activation pointer");
   if (!aligned(d_x, 16) || !aligned(d_y, 16)) return fail(PARO_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
-  const size_t need = paro_workspace_bytes(M, d_in);
+  // the transformed activations are required; up to 16 tokens, the stream-K
+  // kernel's flags and partial tiles behind them are optional
+  const size_t need = xt_bytes(M, d_in), full = paro_workspace_bytes(M, d_in);
   if (!d_workspace || workspace_bytes < need || !aligned(d_workspace, 256))
-    return fail(PARO_ERR_INVALID_ARG, "workspace must be 256-byte aligned and hold %zu bytes", need);
+    return fail(PARO_ERR_INVALID_ARG, "workspace must be 256-byte aligned and hold %zu bytes", full);
+  const size_t used = workspace_bytes < full ? need : full;
   const size_t yb = (size_t)M * d_out * 2;
-  if (overlap(d_y, yb, d_x, (size_t)M * d_in * 2) || overlap(d_y, yb, d_workspace, need) ||
-      overlap(d_workspace, need, d_x, (size_t)M * d_in * 2) ||
+  if (overlap(d_y, yb, d_x, (size_t)M * d_in * 2) || overlap(d_y, yb, d_workspace, used) ||
+      overlap(d_workspace, used, d_x, (size_t)M * d_in * 2) ||
       overlap(d_y, yb, d_qweight, (size_t)d_out * d_in / 2))
     return fail(PARO_ERR_INVALID_ARG, "y, x and workspace must not overlap");
   int* status = status_ptr();
   if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
+  if (M <= paro::kStreamMaxM && used == full) {
+    // few tokens with the full workspace: the batched call's decode forms for
+    // this one linear (at one token a single launch whose first CTA runs the
+    // transform while the others stream the weights)
+    paro_linear L = {};
+    L.d_x = d_x;
+    L.d_y = d_y;
+    L.M = M;
+    L.d_in = d_in;
+    L.d_out = d_out;
+    L.K = K;
+    L.d_pairs = d_pairs;
+    L.d_cos = d_cos;
+    L.d_sin = d_sin;
+    L.d_scale = d_scale;
+    L.d_qweight = d_qweight;
+    L.d_scales = d_scales;
+    L.d_zeros = d_zeros;
+    return paro_rotate_w4_linear_batched(&L, 1, group_size, d_workspace, full, stream);
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = launch_transform(d_x, d_workspace, true, M, d_in, K, d_pairs, d_cos, d_sin, d_scale, status, s,
                                    true);
@@ -361,7 +407,7 @@ size_t batched_stream_bytes(const paro_linear* h_layers, int count) {
 size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int count) {
   if (!h_layers || count <= 0) return 0;
   size_t b = 0;
-  for (int i = 0; i < count; ++i) b += paro_workspace_bytes(h_layers[i].M, h_layers[i].d_in);
+  for (int i = 0; i < count; ++i) b += xt_bytes(h_layers[i].M, h_layers[i].d_in);
   return b + batched_stream_bytes(h_layers, count);
 }
 
@@ -404,7 +450,7 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
       decode_ok = false;
     if (L.K > 0 || L.d_scale) any_transform = true;
     uint16_t* xt = reinterpret_cast<uint16_t*>(static_cast<char*>(d_workspace) + off);
-    off += paro_workspace_bytes(L.M, L.d_in);
+    off += xt_bytes(L.M, L.d_in);
     rp[n] = paro::RotProblem{};
     rp[n].x = L.d_x;
     rp[n].out = xt;
@@ -442,7 +488,7 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
   // the stream-K kernel takes the INT4 linears when every linear has at most 16
   // tokens and the workspace holds its flags and partial tiles (behind the
   // transformed activations)
-  const size_t xt_bytes = xt_need;
+  const size_t xt_total = xt_need;
   bool use_stream = decode_ok && batched_stream_bytes(h_layers, count) > 0 && d_workspace &&
                     workspace_bytes >= need && aligned(d_workspace, 256);
   for (int i = 0; i < n && use_stream; ++i)
@@ -465,7 +511,7 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
       dos[i] = gp[i].d_out;
     }
     return paro::plan_stream_batch(xs, qs, ss, zs, ys, Ms, dis, dos, n, x_f16,
-                                   static_cast<char*>(d_workspace) + xt_bytes, sb, nt, reserved);
+                                   static_cast<char*>(d_workspace) + xt_total, sb, nt, reserved);
   };
   auto launch_stream = [&](bool x_f16, int* st, bool pdl) -> cudaError_t {
     paro::StreamBatch sb;

@@ -7,12 +7,13 @@
 // that must not take the implicit device synchronisation cudaFree can cause,
 // or a program that reserves all of its memory at start-up and forbids any
 // allocation afterwards.  Those callers still own their inputs and outputs;
-// only the fused call's scratch (the transformed activations in fp16) is
-// provided here, by a fixed device array that the library carries.
+// only the fused call's scratch is provided here, by a fixed device array
+// that the library carries: the transformed activations in fp16 and, up to 16
+// tokens, the stream-K INT4 kernel's publication flags and partial tiles.
 //
 // The array is a file-scope __device__ variable: every GPU that loads this
-// library holds kNoAllocMaxElems fp16 values (512 KiB) until the process
-// exits.  Host code cannot use the array's name as a device address (it is a
+// library holds PARO_NOALLOC_SCRATCH_BYTES (2 MiB) until the process exits.
+// Host code cannot use the array's name as a device address (it is a
 // host-side stand-in), so the entry point looks the address up once per
 // device with cudaGetSymbolAddress, with that device current, and passes it
 // to the kernels as their workspace.
@@ -23,10 +24,15 @@
 namespace {
 
 // M * d_in of one call may not exceed this many fp16 elements (e.g. M = 16
-// tokens of width 16384, or one token of width 49152).
+// tokens of width 16384, or one token of width 49152); the rest of the array
+// holds the stream-K kernel's flags and partial tiles, which need about
+// 8.2 KB per SM (the call runs the older per-block kernels on a GPU with so
+// many SMs that they do not fit)
 constexpr size_t kNoAllocMaxElems = size_t(1) << 18;
+constexpr size_t kScratchBytes = PARO_NOALLOC_SCRATCH_BYTES;
+static_assert(kScratchBytes >= kNoAllocMaxElems * sizeof(__half), "scratch holds the transformed activations");
 
-static __device__ __align__(256) __half g_noalloc_scratch[kNoAllocMaxElems];
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::atomic<void*> g_scratch_addr[kMaxDevices];
@@ -68,9 +74,10 @@ extern "C" paro_status paro_rotate_w4_linear_noalloc(const uint16_t* d_x, int K,
       return paro::record_error(PARO_ERR_CUDA, "paro_rotate_w4_linear_noalloc: scratch address lookup: %s",
                                 cudaGetErrorString(e));
   }
-  // Same validation and kernels as the workspace-taking call; nothing here
-  // needs to start at zero because the transform overwrites every scratch
-  // value it hands to the linear.
+  // Same validation and kernels as the workspace-taking call given a workspace
+  // of kScratchBytes.  Nothing here needs to start at zero: the transform
+  // overwrites every activation it hands to the linear, and a stream-K flag
+  // only counts when it holds the id of the launch that reads it.
   return paro_rotate_w4_linear(d_x, K, d_pairs, d_cos, d_sin, d_scale, d_qweight, d_scales, d_zeros, d_y, M,
-                               d_in, d_out, group_size, scratch, kNoAllocMaxElems * sizeof(__half), stream);
+                               d_in, d_out, group_size, scratch, kScratchBytes, stream);
 }

@@ -191,7 +191,7 @@ struct Meta {
   const unsigned short* sc;
   const unsigned short* z;
   __nv_bfloat16* y;
-  int M, d_out, G, tiles;
+  int M, d_out, G, tiles, tile_begin;
 };
 __device__ __forceinline__ void cur_at(const Meta* mp, int count, long long u, Cur& c) {
   int pi = 0;
@@ -320,7 +320,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   __shared__ Meta meta[kMaxBatch];
   if (threadIdx.x < b.count) {
     const StreamProblem& P = b.p[threadIdx.x];
-    meta[threadIdx.x] = Meta{P.unit_begin, P.sc, P.z, P.y, P.M, P.d_out, P.G, P.tiles};
+    meta[threadIdx.x] = Meta{P.unit_begin, P.sc, P.z, P.y, P.M, P.d_out, P.G, P.tiles, P.tile_begin};
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&P.qmap)) : "memory");
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&P.xmap)) : "memory");
   }
@@ -331,6 +331,15 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   // CTA ranges: CTAs 0 .. CA - 1 split units [0, UA) evenly, the others [UA, U)
   const long long CA = b.ctas_a, UA = b.units_a;
   auto cta_start = [&](long long c) -> long long {
+    if (b.tile_split) {
+      // whole tiles: the first unit of tile c T / C of the launch
+      const int tt = (int)part_start(c, C, b.total_tiles);
+      int pi = 0;
+#pragma unroll 1
+      while (pi + 1 < b.count && tt >= meta[pi + 1].tile_begin) ++pi;
+      return tt >= b.total_tiles ? U
+                                 : meta[pi].unit_begin + (long long)(tt - meta[pi].tile_begin) * meta[pi].G;
+    }
     return c <= CA ? part_start(c, CA, UA) : UA + part_start(c - CA, C - CA, U - UA);
   };
   auto cta_of = [&](long long x) -> long long {
@@ -800,11 +809,11 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
                               const __half* const* z, __nv_bfloat16* const* y, const int* M, const int* d_in,
                               const int* d_out, int count, bool x_f16, void* ws, StreamBatch* out, int* nt_out,
                               int reserved_ctas) {
-  if (count < 1 || count > kMaxBatch || !ws) return cudaErrorInvalidValue;
+  if (count < 1 || count > kMaxBatch) return cudaErrorInvalidValue;
   EncodeTiled enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   *out = StreamBatch{};
-  int maxM = 0;
+  int maxM = 0, tiles = 0;
   long long units = 0;
   for (int i = 0; i < count; ++i) {
     if (!stream_supported(M[i], d_in[i], d_out[i], x[i], qw[i])) return cudaErrorInvalidValue;
@@ -819,7 +828,9 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
     p.G = d_in[i] / kGroup;
     p.tiles = (d_out[i] + kStreamRows - 1) / kStreamRows;
     p.unit_begin = units;
+    p.tile_begin = tiles;
     units += (long long)p.tiles * p.G;
+    tiles += p.tiles;
     const cuuint32_t unit_strides[2] = {1, 1};
     {  // codes: uint32 [d_out][d_in / 8], one box = 16 words x 64 rows
       const cuuint64_t dims[2] = {(cuuint64_t)(d_in[i] / 8), (cuuint64_t)d_out[i]};
@@ -843,6 +854,7 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
   }
   out->count = count;
   out->total_units = units;
+  out->total_tiles = tiles;
   const int W = maxM <= 8 ? Geo<1>::W : Geo<2>::W;
   const long long want = (units + W - 1) / W;
   const int sms = device_sm_count();
@@ -851,13 +863,21 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
   out->ctas = (int)(want < avail ? want : avail);
   out->ctas_a = out->ctas;
   out->units_a = units;
+  *nt_out = maxM <= 8 ? 1 : 2;
+  if (!ws) {
+    // no workspace: whole tiles per CTA, so no partial sum crosses a CTA
+    if (reserved_ctas) return cudaErrorInvalidValue;
+    out->tile_split = 1;
+    if (out->ctas > tiles) out->ctas = tiles;
+    out->ctas_a = out->ctas;
+    return cudaSuccess;
+  }
   out->flags = static_cast<unsigned long long*>(ws);
   out->partials = reinterpret_cast<float*>(static_cast<char*>(ws) + round256((size_t)sms * 2 * 8));
   out->xflags = reinterpret_cast<unsigned long long*>(
       static_cast<char*>(ws) + round256((size_t)sms * 2 * 8) +
       round256((size_t)sms * 2 * (4 * (maxM <= 8 ? 1 : 2) * 32 * 4) * 4));
   out->tagword = out->xflags + kMaxBatch * kStreamMaxM;
-  *nt_out = maxM <= 8 ? 1 : 2;
   return cudaSuccess;
 }
 

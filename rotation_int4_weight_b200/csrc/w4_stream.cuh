@@ -21,6 +21,7 @@ struct StreamProblem {
   const unsigned short* z;     // fp16 bits [d_out][d_in/128]
   __nv_bfloat16* y;            // [M][d_out]
   long long unit_begin;        // first unit (one 64-row tile x one 128-column group) of this linear
+  int tile_begin;              // first tile of this linear among the tiles of the launch
   int M, d_in, d_out, G;       // G = d_in / 128
   int tiles;                   // ceil(d_out / 64)
   int xf_begin, xf_count;      // flag form: the flags of this linear's transform CTAs
@@ -39,6 +40,11 @@ struct StreamBatch {
   // CTA); ctas_a = ctas, units_a = total_units is the even split
   long long units_a;
   int ctas_a;
+  // tile_split != 0: CTA c takes the whole tiles [c T / C, (c + 1) T / C) of the
+  // T tiles of the launch, so no tile crosses a CTA boundary and the
+  // cross-CTA flags and partials (flags, partials) are never used
+  int tile_split;
+  int total_tiles;
   int count;
   int ctas;                      // CTAs of the INT4 linear (after the transform CTAs in the fused form)
 };
@@ -49,6 +55,7 @@ bool stream_supported(int M, int d_in, int d_out, const void* x, const void* qwe
 size_t stream_workspace_bytes(int max_m);
 // Builds the launch descriptor: tensor maps, unit and tile offsets, the CTA count.
 // x_f16 selects fp16 (else bf16) activations; ws points at stream_workspace_bytes().
+// ws == nullptr plans the tile-split form (no cross-CTA partial sums).
 cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* qw, const __half* const* sc,
                               const __half* const* z, __nv_bfloat16* const* y, const int* M, const int* d_in,
                               const int* d_out, int count, bool x_f16, void* ws, StreamBatch* out, int* nt_out,

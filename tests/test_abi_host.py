@@ -52,10 +52,23 @@ def test_status_strings_and_version():
 
 
 def test_workspace_bytes():
+    """The fp16 transformed activations (2 M d_in bytes, rounded up to 256), plus,
+    up to 16 tokens, the stream-K kernel's flags and partial tiles: the same
+    bytes as the batched call takes for that one linear."""
+    def xt(M, d):
+        return (2 * M * d + 255) // 256 * 256
     assert paro.paro_workspace_bytes(0, 512) == 0
-    assert paro.paro_workspace_bytes(1, 512) == 1024
-    assert paro.paro_workspace_bytes(3, 1536) == 9216
-    assert paro.paro_workspace_bytes(1, 128) % 256 == 0
+    assert paro.paro_workspace_bytes(17, 512) == xt(17, 512)
+    assert paro.paro_workspace_bytes(2048, 4096) == xt(2048, 4096)
+    extra8 = paro.paro_workspace_bytes(1, 512) - xt(1, 512)
+    extra16 = paro.paro_workspace_bytes(16, 512) - xt(16, 512)
+    assert extra8 > 0 and extra8 % 256 == 0 and extra16 > extra8
+    for M, d in [(1, 512), (3, 1536), (8, 8960), (9, 128), (16, 4096)]:
+        w = paro.paro_workspace_bytes(M, d)
+        assert w % 256 == 0
+        assert w - xt(M, d) == (extra8 if M <= 8 else extra16)
+        one = [paro.ParoLinear(1 << 20, 2 << 20, M, d, 512, 8, 1, 2, 3, 4, 1 << 22, 5, 6)]
+        assert paro.paro_batched_workspace_bytes(one) == w
 
 
 def rot(x=A, y=B, M=4, d=512, K=8, pairs=C, c=D, s=E, scale=W):

@@ -2,7 +2,9 @@
 
 Bit-exact: packing, unpacking, pair indexing.  Within the criteria of
 tests/tolerances.py: the rotation and the linear.  Sizes span several tiles
-and ragged tails; the full-size layers are checked on sampled output rows.
+and ragged tails.  Every decode case (up to 16 tokens) is compared on every
+token and every output column; with more tokens, on sampled token rows that
+include one of every 256-token tile, and every output column.
 """
 import numpy as np
 import pytest
@@ -48,6 +50,16 @@ def gpu_pack(W32, tables=None):
 
 def to_np_pack(qw, sc, z):
     return (qw.cpu().numpy().view(np.uint32), sc.cpu().numpy(), z.cpu().numpy())
+
+
+def oracle_all_columns(xt, qwn, scn, zn, chunk=2048):
+    """The oracle's linear over every output column, dequantising `chunk` weight
+    rows at a time (bounded host memory at the full layer sizes)."""
+    out = np.empty((xt.shape[0], qwn.shape[0]), dtype=np.float64)
+    for r0 in range(0, qwn.shape[0], chunk):
+        r1 = min(r0 + chunk, qwn.shape[0])
+        out[:, r0:r1] = oracle.linear(xt, oracle.dequantize(qwn[r0:r1], scn[r0:r1], zn[r0:r1]))
+    return out
 
 
 # ---------------------------------------------------------------- packing
@@ -214,19 +226,17 @@ def test_empty_batch_is_a_noop():
 
 
 # ---------------------------------------------------------------- full-size layers, sampled rows
-def _sampled_check(p, M_rows, n_cols=256, seed=0):
-    """Full-size fused call; compare sampled tokens x sampled output columns with the oracle."""
+def _full_size_check(p, M_rows, seed=0):
+    """Full-size fused call against the oracle on every output column; every
+    token up to 16 tokens, beyond that M_rows tokens with at least one in every
+    256-token tile of the tensor-core kernel."""
     qw, sc, z = _packed(p)
     y = host(paro.paro_rotate_w4_linear(dev_x(p.x), *dev_tables(p), qw, sc, z))
-    rng = np.random.default_rng(seed)
-    rows = np.sort(rng.choice(p.M, size=min(M_rows, p.M), replace=False))
-    cols = np.sort(rng.choice(p.d_out, size=min(n_cols, p.d_out), replace=False))
-    qwn, scn, zn = to_np_pack(qw, sc, z)
+    rows = np.arange(p.M) if p.M <= 16 else _sampled_rows(p.M, M_rows, seed)
     xt = oracle.rotate(p.x[rows], p.pairs, p.cos_t, p.sin_t, p.scale)
-    w_hat = oracle.dequantize(qwn[cols], scn[cols], zn[cols])
-    ref = oracle.linear(xt, w_hat)
-    got = y[rows][:, cols]
-    # the rms in the criterion is the full output row's, estimated from the sample
+    ref = oracle_all_columns(xt, *to_np_pack(qw, sc, z))
+    got = y[rows]
+    assert np.isfinite(got).all(), p.name
     metric, literal = linear_errors(got, ref)
     assert metric <= 1e-2, (p.name, metric, literal)
 
@@ -234,12 +244,12 @@ def _sampled_check(p, M_rows, n_cols=256, seed=0):
 @pytest.mark.parametrize("cfg", [1, 2])
 def test_full_size_decode_layers(cfg):
     for p in config_problems(cfg, M=1 if cfg == 1 else 16):
-        _sampled_check(p, 16)
+        _full_size_check(p, 16)
 
 
 def test_full_size_prefill_layer_sampled():
     p = next(config_problems(3, only=["k"]))
-    _sampled_check(p, 64, 128)
+    _full_size_check(p, 64)
 
 
 # ---------------------------------------------------------------- batched layer call
@@ -267,15 +277,12 @@ def test_batched_matches_oracle_and_single_calls(shapes_m):
     paro.paro_rotate_w4_linear_batched(layers)
     torch.cuda.synchronize()
     assert paro.paro_get_device_status() == 0
-    rng = np.random.default_rng(0)
     for p, d in zip(probs, devs):
         got = host(d["y"])
         single = host(paro.paro_rotate_w4_linear(d["x"], *d["tables"], d["qw"], d["sc"], d["z"]))
-        cols = np.sort(rng.choice(p.d_out, size=min(256, p.d_out), replace=False))
-        qwn, scn, zn = to_np_pack(d["qw"], d["sc"], d["z"])
-        ref = oracle.linear(oracle.rotate(p.x, p.pairs, p.cos_t, p.sin_t, p.scale),
-                            oracle.dequantize(qwn[cols], scn[cols], zn[cols]))
-        assert_linear_close(got[:, cols], ref)
+        ref = oracle_all_columns(oracle.rotate(p.x, p.pairs, p.cos_t, p.sin_t, p.scale),
+                                 *to_np_pack(d["qw"], d["sc"], d["z"]))
+        assert_linear_close(got, ref)
         assert_linear_close(got, single)
 
 
@@ -291,9 +298,14 @@ def test_batched_rejects_bad_layer_without_launching():
 
 
 # ---------------------------------------------------------------- tensor-core (tcgen05) path, M >= 128
-def _sampled_rows(M, n, seed):
+def _sampled_rows(M, n, seed, tile=256):
+    """n seeded token rows of M, at least one in every `tile`-token tile (the
+    tensor-core kernel's token tile), the rest drawn at random."""
     rng = np.random.default_rng(seed)
-    return np.sort(rng.choice(M, size=min(n, M), replace=False))
+    per_tile = [int(rng.integers(t0, min(t0 + tile, M))) for t0 in range(0, M, tile)]
+    rest = np.setdiff1d(np.arange(M), per_tile)
+    extra = rng.choice(rest, size=max(0, min(n, M) - len(per_tile)), replace=False) if rest.size else []
+    return np.sort(np.concatenate([per_tile, extra]).astype(np.int64))
 
 
 @pytest.mark.parametrize("M,d_in,d_out", [(128, 256, 256), (200, 512, 272), (384, 1536, 1024), (129, 4096, 512)])
@@ -365,15 +377,11 @@ def test_stream_decode_matches_oracle_and_repeats_bit_exactly(shapes_m, rotate):
     torch.cuda.synchronize()
     assert paro.paro_get_device_status() == 0
     first = [d["y"].clone() for d in devs]
-    rng = np.random.default_rng(3)
     for p, d in zip(probs, devs):
         got = host(d["y"])
         assert np.isfinite(got).all(), p.name
-        cols = np.sort(rng.choice(p.d_out, size=min(320, p.d_out), replace=False))
-        qwn, scn, zn = to_np_pack(d["qw"], d["sc"], d["z"])
         xt = oracle.rotate(p.x, p.pairs, p.cos_t, p.sin_t, p.scale) if rotate else p.x
-        ref = oracle.linear(xt, oracle.dequantize(qwn[cols], scn[cols], zn[cols]))
-        assert_linear_close(got[:, cols], ref)
+        assert_linear_close(got, oracle_all_columns(xt, *to_np_pack(d["qw"], d["sc"], d["z"])))
     # the arrival counters left by the first call are reused as they are: the
     # second call must give the same bits (fixed summation order)
     for d in devs:
@@ -405,15 +413,12 @@ def test_stream_decode_full_size_llama_layer_split():
     torch.cuda.synchronize()
     assert paro.paro_get_device_status() == 0
     first = [d["y"].clone() for d in devs]
-    rng = np.random.default_rng(5)
     for p, d in zip(probs, devs):
         got = host(d["y"])
         assert np.isfinite(got).all(), p.name
-        cols = np.sort(rng.choice(p.d_out, size=128, replace=False))
-        qwn, scn, zn = to_np_pack(d["qw"], d["sc"], d["z"])
-        ref = oracle.linear(oracle.rotate(p.x, p.pairs, p.cos_t, p.sin_t, p.scale),
-                            oracle.dequantize(qwn[cols], scn[cols], zn[cols]))
-        assert_linear_close(got[:, cols], ref)
+        ref = oracle_all_columns(oracle.rotate(p.x, p.pairs, p.cos_t, p.sin_t, p.scale),
+                                 *to_np_pack(d["qw"], d["sc"], d["z"]))
+        assert_linear_close(got, ref)
     for d in devs:
         d["y"].fill_(float("nan"))
     paro.paro_rotate_w4_linear_batched(layers, workspace=ws)

@@ -162,6 +162,39 @@ def test_fold_then_transform_reproduces_unquantised_linear():
     assert err < 1e-10
 
 
+def test_pack_weights_scale_only_branch():
+    """K = 0 with a channel scale: the packed weights are those of W diag(s),
+    column c multiplied by s_c (the fold with no stage, page "ParoQuant:
+    pairwise rotations that survive deployment", section "A rotation small
+    enough to execute"), so that W~ (x / s) = W x up to quantisation."""
+    p = linear_problem(98, 0, 256, 32, 3, K=8)
+    W, s = p.W, p.scale
+    # the closed form, one column at a time
+    ws = np.empty(W.shape, dtype=np.float64)
+    for c in range(p.d_in):
+        ws[:, c] = W[:, c].astype(np.float64) * float(s[c])
+    q, sc, z = oracle.quantize_groups(ws.astype(np.float32))
+    qw, scw, zw = oracle.pack_weights(W, None, None, None, s)
+    assert np.array_equal(qw, oracle.pack_nibbles(q))
+    assert np.array_equal(scw.view(np.uint16), sc.view(np.uint16))
+    assert np.array_equal(zw, z.astype(np.float16))
+    # the same as a fold with zero stages, and as pack_weights given empty tables
+    empty = (p.pairs[:0], p.cos_t[:0], p.sin_t[:0])
+    assert np.array_equal(oracle.fold_weights(W, *empty, s), ws)
+    qe, sce, ze = oracle.pack_weights(W, *empty, s)
+    assert np.array_equal(qe, qw) and np.array_equal(sce, scw) and np.array_equal(ze, zw)
+    # a divide (or no scale at all) would give other codes
+    assert not np.array_equal(oracle.pack_weights(W, None, None, None, None)[0], qw)
+    # and the scaled activations undo it: W^ (x / s) stays within the quantisation
+    # bound of W x, row by row
+    xs = p.x.astype(np.float64) / s.astype(np.float64)
+    y = oracle.linear(xs, oracle.dequantize(qw, scw, zw))
+    y_ref = p.x.astype(np.float64) @ W.astype(np.float64).T
+    step = np.repeat(scw.astype(np.float64), 128, axis=1)          # [d_out, d_in]
+    bound = np.abs(xs) @ (step / 2 + 15 * step * 2.0 ** -11).T     # [M, d_out]
+    assert np.all(np.abs(y - y_ref) <= bound + 1e-12)
+
+
 def test_non_disjoint_stage_is_rejected():
     pairs = np.array([[0, 1], [1, 2]], dtype=np.uint16)
     with pytest.raises(ValueError):
