@@ -72,7 +72,8 @@ typedef enum {
   PARO_ERR_INVALID_ARG = 1,
   PARO_ERR_UNSUPPORTED = 2,
   PARO_ERR_CUDA = 3,
-  PARO_ERR_TIMEOUT = 4
+  PARO_ERR_TIMEOUT = 4,
+  PARO_ERR_RANGE = 5
 } paro_status;
 
 /* Layout version of the packed weights described above. */
@@ -305,14 +306,37 @@ PARO_API paro_status paro_rotate_w4_linear_noalloc(const uint16_t* d_x, int K, c
 
 /*
  * Synchronises `stream`, then returns and clears the device status word of
- * the current GPU: PARO_OK, PARO_ERR_INVALID_ARG (a kernel met a pair index
- * >= d and skipped or clamped it: that call's results are void) or
- * PARO_ERR_TIMEOUT (a bounded wait gave up: that call's results are void).
- * The word's device address is looked up on the first call of the library on
- * each device and kept for the life of the process, so cudaDeviceReset on a
- * device after the library has used it is not supported.
+ * the current GPU (the first error a kernel met since the last read):
+ * PARO_OK; PARO_ERR_INVALID_ARG (a kernel met a pair index >= d and skipped or
+ * clamped it); PARO_ERR_TIMEOUT (a bounded wait gave up: a tensor-memory copy
+ * or a hand-over flag between the transform and the INT4 linear did not come
+ * within its limit; the CTAs that waited wrote none of their output tiles);
+ * PARO_ERR_RANGE (a transformed activation handed to the INT4 linear in fp16
+ * was beyond the fp16 range, |x~| >= 65520, and became infinite).  After any
+ * of them that call's results are void.  The word's device address is looked
+ * up on the first call of the library on each device and kept for the life
+ * of the process, so cudaDeviceReset on a device after the library has used
+ * it is not supported.
  */
 PARO_API paro_status paro_get_device_status(paro_stream_t stream);
+
+/*
+ * Test hooks for the failure paths (no counterpart in the pages): they change
+ * how later launches are configured and stay set until called again.
+ * flag_wait_cycles > 0 bounds every wait of the decode INT4 kernel for a
+ * hand-over flag (the transform's "x~ is written" flags, and the partial
+ * sums of a tile split between CTAs) to about that many SM clock cycles
+ * instead of about 2^31 (a second); 0 restores the default.
+ * skip_ready_flags != 0 makes the decode transforms (in the fused one-token
+ * launch and in the transform launch before the INT4 launch at 2-16 tokens)
+ * skip publishing their "x~ is written" flags, so that the INT4 kernel's
+ * waits run out: the call then reports PARO_ERR_TIMEOUT through
+ * paro_get_device_status() and writes none of the output tiles of the linears
+ * it waited for.  Nothing hangs: every wait is bounded.  Not thread-safe with
+ * respect to calls being configured at the same time; PARO_ERR_INVALID_ARG
+ * for a negative cycle count.
+ */
+PARO_API paro_status paro_set_test_hooks(long long flag_wait_cycles, int skip_ready_flags);
 
 #ifdef __cplusplus
 }

@@ -19,7 +19,7 @@ __all__ = [
     "paro_pack_weights", "paro_rotate", "paro_w4_linear", "paro_rotate_w4_linear",
     "paro_rotate_w4_linear_noalloc", "paro_get_device_status", "EXPORTED", "ParoLinear", "paro_linear",
     "paro_batched_workspace_bytes", "paro_rotate_w4_linear_batched", "paro_plan_pair_order",
-    "paro_rotate_backward_workspace_bytes", "paro_rotate_backward",
+    "paro_rotate_backward_workspace_bytes", "paro_rotate_backward", "paro_set_test_hooks",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libparo.so")
@@ -42,6 +42,7 @@ EXPORTED = {
     "paro_get_device_status": (_I, [_P]),
     "paro_rotate_backward_workspace_bytes": (_S, [_I, _I, _I, _I]),
     "paro_rotate_backward": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "paro_set_test_hooks": (_I, [ctypes.c_longlong, _I]),
 }
 
 
@@ -260,6 +261,14 @@ def paro_plan_pair_order(pairs, cos_t, sin_t):
                                   po.ctypes.data, co.ctypes.data, so.ctypes.data)
     _check(st, "paro_plan_pair_order")
     return po, co, so
+
+
+def paro_set_test_hooks(flag_wait_cycles: int = 0, skip_ready_flags: bool = False) -> None:
+    """Test hooks of the failure paths: bound the decode INT4 kernel's hand-over
+    flag waits to `flag_wait_cycles` SM cycles (0: the default, about a second)
+    and make the decode transforms skip publishing their flags.  Affects the
+    calls configured afterwards; (0, False) restores the defaults."""
+    _check(lib.paro_set_test_hooks(int(flag_wait_cycles), 1 if skip_ready_flags else 0), "paro_set_test_hooks")
 
 
 def paro_get_device_status(stream=None) -> int:

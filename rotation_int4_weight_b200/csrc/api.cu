@@ -181,7 +181,18 @@ cudaError_t launch_transform(const uint16_t* x, void* out, bool f16_out, int M, 
 
 }  // namespace
 
+namespace {
+std::atomic<long long> g_hook_flag_wait{0};
+std::atomic<int> g_hook_skip_flags{0};
+}  // namespace
+
 namespace paro {
+long long hook_flag_wait() {
+  const long long v = g_hook_flag_wait.load(std::memory_order_relaxed);
+  return v > 0 ? v : kWaitCycles;
+}
+int hook_skip_ready_flags() { return g_hook_skip_flags.load(std::memory_order_relaxed); }
+
 paro_status record_error(paro_status s, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -202,11 +213,19 @@ const char* paro_status_string(paro_status s) {
     case PARO_ERR_UNSUPPORTED: return "PARO_ERR_UNSUPPORTED";
     case PARO_ERR_CUDA: return "PARO_ERR_CUDA";
     case PARO_ERR_TIMEOUT: return "PARO_ERR_TIMEOUT";
+    case PARO_ERR_RANGE: return "PARO_ERR_RANGE";
   }
   return "PARO_ERR_UNKNOWN";
 }
 
 const char* paro_last_error(void) { return t_last_error; }
+
+paro_status paro_set_test_hooks(long long flag_wait_cycles, int skip_ready_flags) {
+  if (flag_wait_cycles < 0) return fail(PARO_ERR_INVALID_ARG, "flag_wait_cycles = %lld is negative", flag_wait_cycles);
+  g_hook_flag_wait.store(flag_wait_cycles, std::memory_order_relaxed);
+  g_hook_skip_flags.store(skip_ready_flags != 0 ? 1 : 0, std::memory_order_relaxed);
+  return ok();
+}
 
 paro_status paro_pack_weights(const float* d_W, int d_out, int d_in, int group_size, int K,
                               const uint16_t* d_pairs, const float* d_cos, const float* d_sin,
@@ -572,6 +591,7 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     paro::StreamBatch sb;
     int nt = 1;
     e = paro::plan_fused_rot(rp, n, &rb);
+    rb.skip_flags = paro::hook_skip_ready_flags();
     if (e == cudaSuccess) e = plan_stream(true, rb.count, &sb, &nt);
     if (e == cudaSuccess) {
       paro::set_fused_split(sb, 0.4);
@@ -602,6 +622,7 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
                   paro::kXFlagWords - 1);
     rb.tagword = sb.tagword;
     rb.xflags = sb.xflags;
+    rb.skip_flags = paro::hook_skip_ready_flags();
     for (int i = 0; i < n; ++i) {
       const paro::RotProblem& t = rb.p[i + 1 < n ? i + 1 : 0];
       sb.p[i].xf_begin = t.cta_begin;

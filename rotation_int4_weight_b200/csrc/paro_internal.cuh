@@ -13,6 +13,16 @@ namespace paro {
 // Values written into the per-device status word (first error wins).
 constexpr int kStatusBadIndex = PARO_ERR_INVALID_ARG;
 constexpr int kStatusTimeout = PARO_ERR_TIMEOUT;
+constexpr int kStatusRange = PARO_ERR_RANGE;
+
+// Default bound of a bounded wait, in SM clock cycles (about a second).
+constexpr long long kWaitCycles = 1LL << 31;
+
+// True when either half of a packed fp16 pair is infinite (the rounding of a
+// finite value beyond the fp16 range).
+__device__ __forceinline__ bool half2_inf(uint32_t u) {
+  return ((u & 0x7FFFu) == 0x7C00u) | ((u & 0x7FFF0000u) == 0x7C000000u);
+}
 
 constexpr int kGroup = 128;      // quantisation group along d_in
 constexpr int kMaxStages = 16;   // K
@@ -24,6 +34,11 @@ __device__ __forceinline__ void report_status(int* status, int code) {
 
 // Stores a printf-style message for paro_last_error() and returns s.
 paro_status record_error(paro_status s, const char* fmt, ...);
+
+// Test hooks (paro_set_test_hooks): the wait bound for hand-over flags in
+// cycles, and whether the decode transforms skip publishing their flags.
+long long hook_flag_wait();
+int hook_skip_ready_flags();
 
 // ---- launchers implemented in the kernel translation units --------------------
 // All return a cudaError_t from the launch (cudaSuccess when nothing failed).

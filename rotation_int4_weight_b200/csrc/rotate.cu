@@ -238,7 +238,9 @@ givens_cm_kernel(const void* __restrict__ in, void* __restrict__ out, int M, int
 
   if (bad) report_status(status, kStatusBadIndex);
 
-  // ---- channel scale and store -------------------------------------------------
+  // ---- channel scale and store (an fp16 value that rounds to infinity is
+  // reported once: PARO_ERR_RANGE) ------------------------------------------------
+  bool ovf = false;
 #pragma unroll 1
   for (int cp = tid; cp < half; cp += NTH) {
     const int c = 2 * cp;
@@ -259,11 +261,14 @@ givens_cm_kernel(const void* __restrict__ in, void* __restrict__ out, int M, int
         } else if constexpr (MODE == kActBf16) {
           *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(out) + off) = __floats2bfloat162_rn(a, b);
         } else {
-          *reinterpret_cast<__half2*>(static_cast<__half*>(out) + off) = __floats2half2_rn(a, b);
+          const __half2 h = __floats2half2_rn(a, b);
+          ovf |= half2_inf(*reinterpret_cast<const uint32_t*>(&h));
+          *reinterpret_cast<__half2*>(static_cast<__half*>(out) + off) = h;
         }
       }
     }
   }
+  if (ovf) report_status(status, kStatusRange);
 }
 
 // Rows per CTA: the widest channel vector whose rows fit in shared memory

@@ -61,7 +61,7 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
   } else {
     done = rotdec::rot_decode_cta<R, F16OUT, U, kRotThreads>(P, row0, smem, bars, status, pdl_wait != 0);
   }
-  if (batch.xflags && done) {
+  if (batch.xflags && done && !batch.skip_flags) {
     // every thread's x~ stores, then this CTA's flag
     __threadfence();
     __syncthreads();

@@ -30,6 +30,7 @@ struct RotBatch {
   // same id once its rows of x~ are written
   unsigned long long* tagword;
   unsigned long long* xflags;
+  int skip_flags;  // test hook: publish no xflags (the INT4 linear's waits then run out)
   int count;
   int total_ctas;
 };

@@ -254,7 +254,9 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
   }
 
   // channel scale and store: the scales of LB channel pairs are loaded (from
-  // L2, where the prologue put them) before any of them is used
+  // L2, where the prologue put them) before any of them is used.  An fp16
+  // value that rounds to infinity is reported once (PARO_ERR_RANGE).
+  bool ovf = false;
 #pragma unroll 1
   for (int cp0 = tid; cp0 < half; cp0 += LB * NTHR) {
     float2 sc[LB];
@@ -275,15 +277,18 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
         if (r < nrows) {
           const float2 v = *reinterpret_cast<const float2*>(xs + (size_t)r * d + c);
           const size_t off = (size_t)(row0 + r) * d + c;
-          if constexpr (F16OUT)
-            *reinterpret_cast<__half2*>(static_cast<__half*>(P.out) + off) = __floats2half2_rn(v.x * f0, v.y * f1);
-          else
+          if constexpr (F16OUT) {
+            const __half2 h = __floats2half2_rn(v.x * f0, v.y * f1);
+            ovf |= half2_inf(*reinterpret_cast<const uint32_t*>(&h));
+            *reinterpret_cast<__half2*>(static_cast<__half*>(P.out) + off) = h;
+          } else
             *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(P.out) + off) =
                 __floats2bfloat162_rn(v.x * f0, v.y * f1);
         }
       }
     }
   }
+  if (ovf) report_status(status, kStatusRange);
   return true;
 }
 

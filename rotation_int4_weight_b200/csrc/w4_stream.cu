@@ -256,15 +256,16 @@ __device__ __forceinline__ unsigned long long grid_tag() {
 __device__ __forceinline__ void st_flag(unsigned long long* f, unsigned long long v) {
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(f), "l"(v) : "memory");
 }
-// Bounded wait (about a second of SM clock) for a flag to hold v.
-__device__ bool wait_flag(const unsigned long long* f, unsigned long long v) {
+// Bounded wait (at most `limit` SM clock cycles; about a second by default)
+// for a flag to hold v.
+__device__ bool wait_flag(const unsigned long long* f, unsigned long long v, long long limit) {
   const long long t0 = clock64();
 #pragma unroll 1
   while (true) {
     unsigned long long x;
     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];\n" : "=l"(x) : "l"(f) : "memory");
     if (x == v) return true;
-    if (clock64() - t0 > (1LL << 31)) return false;
+    if (clock64() - t0 > limit) return false;
     __nanosleep(64);
   }
 }
@@ -312,7 +313,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
         // the asynchronous proxy after seeing it)
         __threadfence();
         __syncthreads();
-        if (threadIdx.x == 0) st_flag(b.xflags + blockIdx.x, grid_tag());
+        if (threadIdx.x == 0 && !rb.skip_flags) st_flag(b.xflags + blockIdx.x, grid_tag());
       }
       return;
     }
@@ -400,7 +401,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
 #pragma unroll 1
     for (int q = 0; q < nf && seen; ++q) {
       if (block) {
-        seen = wait_flag(f + q, xtag);
+        seen = wait_flag(f + q, xtag, b.flag_wait);
         if (!seen) report_status(status, kStatusTimeout);
       } else {
         unsigned long long v;
@@ -482,14 +483,23 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
     }
     if constexpr (FU != 0) {
       // the unit's activations were deferred: wait (bounded) for its linear's x~
+      int xfail = 0;
       if (lane == 0 && ((xpend >> slot) & 1u)) {
-        // (on a timeout the slot still gets its arrival, so that its phase
-        // completes once the codes have landed; the status says the result is void)
-        if (x_ready(cc.pi, true)) issue_x(cc, slot);
-        else mbar_arrive(bar0 + 8u * slot);
+        // on a timeout the slot still gets its arrival, so that its phase
+        // completes once the codes have landed, and the warp stops: the
+        // status says the result is void and no tile it holds is written
+        if (x_ready(cc.pi, true)) {
+          issue_x(cc, slot);
+        } else {
+          mbar_arrive(bar0 + 8u * slot);
+          xfail = 1;
+        }
         xpend &= ~(1u << slot);
       }
-      __syncwarp();
+      if (__shfl_sync(0xffffffffu, xfail, 0)) {
+        ok = false;
+        break;
+      }
     }
     if (!mbar_wait(bar0 + 8u * slot, phase)) {
       report_status(status, kStatusTimeout);
@@ -613,6 +623,9 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
     __syncwarp();
     for (int j = done; j < n && j < done + D; ++j) mbar_wait(bar0 + 8u * (j % D), (uint32_t)((j / D) & 1));
   }
+  // a warp that gave up voids the CTA's result: none of its remaining tiles is
+  // written and no partial is published (a CTA waiting for one gives up too)
+  if (__syncthreads_or(!ok)) return;
 
   // ---- the last tile, and the partial tiles in shared memory -------------------------
   // slot 0: the warp's first tile when it began before the warp's units;
@@ -730,16 +743,18 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
 #pragma unroll
         for (int e = 0; e < 4; ++e) tot[rt][m][e] = 0.f;
     const long long ca = cta_of(Ub);
+    bool got = true;  // every earlier CTA's partial arrived
 #pragma unroll 1
     for (long long cx = ca; cx < cta; ++cx) {
       const long long s0 = cta_start(cx);
       if (cta_start(cx + 1) <= s0) continue;  // a CTA without units
       const int e = (Ub <= s0) ? 0 : 1;
       int seen = 1;
-      if (lane == 0) seen = wait_flag(b.flags + cx * 2 + e, tag) ? 1 : 0;
+      if (lane == 0) seen = wait_flag(b.flags + cx * 2 + e, tag, b.flag_wait) ? 1 : 0;
       seen = __shfl_sync(0xffffffffu, seen, 0);
       if (!seen) {
         if (lane == 0) report_status(status, kStatusTimeout);
+        got = false;
         break;
       }
       __threadfence();
@@ -752,6 +767,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
           tot[rt][m][0] += v.x; tot[rt][m][1] += v.y; tot[rt][m][2] += v.z; tot[rt][m][3] += v.w;
         }
     }
+    if (!got) continue;  // the tile stays unwritten: the status says the result is void
 #pragma unroll
     for (int rt = 0; rt < 4; ++rt)
 #pragma unroll
@@ -863,6 +879,7 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
   out->ctas = (int)(want < avail ? want : avail);
   out->ctas_a = out->ctas;
   out->units_a = units;
+  out->flag_wait = hook_flag_wait();
   *nt_out = maxM <= 8 ? 1 : 2;
   if (!ws) {
     // no workspace: whole tiles per CTA, so no partial sum crosses a CTA

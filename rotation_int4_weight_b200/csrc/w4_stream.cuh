@@ -39,6 +39,7 @@ struct StreamBatch {
   // (the fused form gives the widest linear, whose x~ comes last, fewer units a
   // CTA); ctas_a = ctas, units_a = total_units is the even split
   long long units_a;
+  long long flag_wait;           // bound of a hand-over flag wait, SM clock cycles
   int ctas_a;
   // tile_split != 0: CTA c takes the whole tiles [c T / C, (c + 1) T / C) of the
   // T tiles of the launch, so no tile crosses a CTA boundary and the

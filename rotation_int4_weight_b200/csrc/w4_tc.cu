@@ -187,6 +187,7 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
   __shared__ __align__(8) uint64_t bars[5 * kStages + 2];
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
+  __shared__ int s_issued, s_committed;  // stages the TMA thread issued / the MMA thread committed
   __shared__ TcMeta meta[kTcMaxBatch];
 
   // the 128-byte swizzle needs every tile at a 1024-byte aligned shared address
@@ -220,6 +221,8 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
     mbar_init(b_acc_full, 1);
     mbar_init(b_acc_empty, kDqWarps * 32);
     abort_flag = 0;
+    s_issued = 0;
+    s_committed = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   if (warp == kWarpTma) {  // tensor memory for the accumulators
@@ -247,7 +250,7 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
     if constexpr (!XF16) {
       const int t = threadIdx.x - kWarpConv * 32;  // 0 .. 255
       int it = 0;
-      bool stop = false;
+      bool stop = false, ovf = false;
 #pragma unroll 1
       for (int j = 0; !stop; ++j) {
         const int T = tile_of(j, total);
@@ -273,6 +276,7 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
               const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v[q][e]));
               const __half2 h = __floats2half2_rn(f.x, f.y);
               v[q][e] = *reinterpret_cast<const uint32_t*>(&h);
+              ovf |= half2_inf(v[q][e]);
             }
             const uint32_t a = a0 + (uint32_t)((t + q * BM) * 16);
             asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(a), "r"(v[q][0]), "r"(v[q][1]), "r"(v[q][2]),
@@ -283,6 +287,9 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
           mbar_arrive(b_full_a + 8 * s);
         }
       }
+      // a bf16 input beyond the fp16 range became infinite (the rows past M are
+      // zero-filled by the copy, so this is always a real input)
+      if (ovf) report_status(status, kStatusRange);
     }
   } else if (warp == kWarpTma) {
     // ---------------- TMA producer: packed codes (both variants), fp16 activations ---
@@ -309,6 +316,7 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
           tma_load_2d(s_base + s * STAGE_BYTES, &P.xmap, k * BK, ti.m0, bar_a);
         }
       }
+      s_issued = it;
     }
   } else if (warp == kWarpMma) {
     // ---------------- MMA issuer ---------------------------------------------------
@@ -344,6 +352,7 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
         }
         if (ok) mma_commit(b_acc_full);  // arrives once every MMA of the tile has completed
       }
+      s_committed = it;
     }
   } else {
     // ---------------- dequantisation (warps 0-15), then each tile's epilogue ----------
@@ -467,15 +476,21 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
   if (abort_flag && threadIdx.x == 0) {
-    // let any copies and MMAs still in flight land before the memory goes away
+    // let the copies and MMAs still in flight land before the memory goes away:
+    // per slot, the phase of the last copy issued into it and of the last MMA
+    // commit that read it (earlier phases have completed before those could be
+    // issued); a wait that gives up again is reported again
+    const uint32_t bar_a = XF16 ? b_full_a : b_full_raw;
+    auto last_of = [](int n, int slot) { return n > slot ? slot + ((n - 1 - slot) / kStages) * kStages : -1; };
     for (int s = 0; s < kStages; ++s) {
-      const uint32_t bar_a = XF16 ? b_full_a : b_full_raw;
-      mbar_wait(bar_a + 8 * s, 0);
-      mbar_wait(bar_a + 8 * s, 1);
-      mbar_wait(b_full_c + 8 * s, 0);
-      mbar_wait(b_full_c + 8 * s, 1);
-      mbar_wait(b_empty + 8 * s, 0);
-      mbar_wait(b_empty + 8 * s, 1);
+      const int jt = last_of(s_issued, s), jm = last_of(s_committed, s);
+      bool landed = true;
+      if (jt >= 0) {
+        const uint32_t par = (uint32_t)((jt / kStages) & 1);
+        landed = mbar_wait(bar_a + 8 * s, par) && mbar_wait(b_full_c + 8 * s, par);
+      }
+      if (jm >= 0) landed = mbar_wait(b_empty + 8 * s, (uint32_t)((jm / kStages) & 1)) && landed;
+      if (!landed) report_status(status, kStatusTimeout);
     }
   }
   __syncthreads();

@@ -47,8 +47,14 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_version():
     assert paro.paro_weight_layout_version() == 1
     for code, name in [(0, "PARO_OK"), (1, "PARO_ERR_INVALID_ARG"), (2, "PARO_ERR_UNSUPPORTED"),
-                       (3, "PARO_ERR_CUDA"), (4, "PARO_ERR_TIMEOUT")]:
+                       (3, "PARO_ERR_CUDA"), (4, "PARO_ERR_TIMEOUT"), (5, "PARO_ERR_RANGE")]:
         assert paro.lib.paro_status_string(code).decode() == name
+
+
+def test_test_hooks_validate_and_reset():
+    assert paro.lib.paro_set_test_hooks(-1, 0) == INVALID
+    assert paro.lib.paro_set_test_hooks(100000, 1) == OK
+    assert paro.lib.paro_set_test_hooks(0, 0) == OK
 
 
 def test_workspace_bytes():
