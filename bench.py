@@ -166,6 +166,18 @@ class Linear:
     def rotate(self, paro):
         paro.paro_rotate(self.x, self.pairs, self.cos, self.sin, self.scale, out=self.xr)
 
+    def dense(self, paro):
+        # the contrast the pages draw: a dense d x d rotation (bf16 matrix
+        # multiply on the tensor cores) before the same INT4 linear
+        if getattr(self, "Q", None) is None:
+            import torch
+            g = torch.Generator(device=self.x.device)
+            g.manual_seed(self.d_in * 131 + self.d_out)
+            self.Q = (torch.randn(self.d_in, self.d_in, generator=g, device=self.x.device)
+                      * self.d_in ** -0.5).to(torch.bfloat16)
+        paro.paro_dense_rotate(self.x, self.Q, out=self.xr)
+        paro.paro_w4_linear(self.xr, self.qw0, self.sc0, self.z0, out=self.y)
+
     def rotate_backward(self, paro):
         # gradients of the transform for a synthetic upstream gradient (the
         # calibration-time step; buffers made on first use)
@@ -186,7 +198,7 @@ class Linear:
 
 # kernels launched per linear of each variant (batched: 2 per call of up to 7 linears)
 LAUNCHES = {"fused": 2, "unfused": 2, "plain": 1, "rotate": 1, "fused_e2e": 2,  # plain: 2 when M > 64
-            "rotate_backward": 2}
+            "rotate_backward": 2, "dense": 2}
 BATCH = 7  # linears per batched call (one decoder layer)
 
 
@@ -576,6 +588,10 @@ def bytes_of(step_lins, M, variant):
         return sum(linear_bytes(l.d_in, l.d_out, M, rotate=False) for l in step_lins)
     if variant == "rotate":
         return sum(4 * M * l.d_in + TABLE_BYTES_PER_CH * l.d_in for l in step_lins)
+    if variant == "dense":
+        # the d x d bf16 matrix and the x~ round trip on top of the plain linear
+        return sum(linear_bytes(l.d_in, l.d_out, M, rotate=False) + 2 * l.d_in * l.d_in + 4 * M * l.d_in
+                   for l in step_lins)
     if variant == "rotate_backward":
         # x (bf16) and the upstream gradient in, dx out (fp32), the tables and
         # the outputs dtheta, dscale; the per-block partial sums round trip
@@ -635,6 +651,10 @@ def sub_record(r, world, hbm, bf16, bf16_sus):
            "linears_per_step": len(lins), "distinct_units_cycled": len(r["units"]),
            "ms_per_step": round(ms, 6), "reps": t["batched"].reps, "l2": t["batched"].l2,
            "rotation_overhead_pct": overhead(t, "batched", "batched_plain")}
+    if "dense" in t:
+        rec["per_linear"] = {k: round(t[k].ms, 6) for k in ("plain", "fused", "dense") if k in t}
+        rec["rotation_overhead_per_linear_fused_pct"] = overhead(t, "fused", "plain")
+        rec["dense_rotation_overhead_pct"] = overhead(t, "dense", "plain")
     if prefill:
         tf = whole_job_rate(flops, world, ms) / 1e12
         rec.update(value=round(tf, 2), unit="TFLOP/s", frac_of_bf16=round(tf / bf16, 4))
@@ -673,7 +693,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-sub", action="store_true", help="skip the prefill, stack and Llama decode sub-records")
-    ap.add_argument("--variants", default="batched,batched_plain,fused,plain,unfused,rotate,rotate_backward")
+    ap.add_argument("--variants", default="batched,batched_plain,fused,plain,unfused,rotate,rotate_backward,dense")
     ap.add_argument("--no-plan", action="store_true",
                     help="use the pair tables as drawn instead of the conflict-free order of paro_plan_pair_order")
     ap.add_argument("--profile", action="store_true",
@@ -810,6 +830,10 @@ def main():
         "rotation_overhead_pct": overhead(t, "batched", "batched_plain"),
         "rotation_overhead_unfused_pct": overhead(t, "unfused", "plain"),
         "rotation_overhead_per_linear_fused_pct": overhead(t, "fused", "plain"),
+        "dense_rotation_overhead_pct": overhead(t, "dense", "plain"),
+        "dense_rotation": ("the contrast the pages draw: a dense d x d bf16 rotation (paro_dense_rotate, tensor "
+                           "cores) then the same INT4 linear, per linear; its overhead against the plain per-"
+                           "linear INT4 calls sits beside rotation_overhead_per_linear_fused_pct"),
         "rotate_kernel_gbs": (round(bytes_of(step_lins, M, "rotate") / (t["rotate"].ms * 1e-3) / 1e9, 1)
                               if "rotate" in t else None),
         "rotate_backward": ({"ms_per_step": round(t["rotate_backward"].ms, 6),
@@ -825,7 +849,7 @@ def main():
     torch.cuda.empty_cache()
     if not args.no_sub and args.config == 1 and args.M is None:
         subs = {}
-        for key, cfg, m, vs in [("prefill_llama_m2048", 3, None, "batched,batched_plain,rotate"),
+        for key, cfg, m, vs in [("prefill_llama_m2048", 3, None, "batched,batched_plain,rotate,plain,fused,dense"),
                                 ("stack_qwen_196_linears_m16", 4, None, "batched,batched_plain"),
                                 ("decode_llama_m1", 2, 1, "batched,batched_plain")]:
             r = run_workload(torch, paro, args, cfg, m, vs.split(","), dist, rank, dev, flush, min_seconds=0.5)

@@ -148,6 +148,22 @@ PARO_API paro_status paro_rotate_backward(const uint16_t* d_x, const float* d_gr
                                           void* d_workspace, size_t workspace_bytes, paro_stream_t stream);
 
 /*
+ * The dense learned rotation that the pairwise transform is contrasted with
+ * (page "ParoQuant: pairwise rotations that survive deployment", section "Why
+ * it differs from a dense learned rotation": a dense rotation puts a large
+ * matrix multiply in front of every INT4 GEMM): x~ = x Q^T for a bf16 d x d
+ * matrix Q, i.e. x~[m][n] = sum_k Q[n][k] x[m][k], on the tensor cores (bf16
+ * operands, fp32 accumulation, bf16 out, round to nearest even).  It exists to
+ * measure that cost against the pairwise transform on the same INT4 linears;
+ * the result feeds paro_w4_linear like any transformed activation.
+ * d_x: bf16 [M][d]; d_q: bf16 [d][d] row-major; d_out: bf16 [M][d], not
+ * overlapping d_x or d_q.  Needs d a multiple of 64 (PARO_ERR_UNSUPPORTED
+ * otherwise) and 16-byte aligned pointers.
+ */
+PARO_API paro_status paro_dense_rotate(const uint16_t* d_x, const uint16_t* d_q, uint16_t* d_out, int M, int d,
+                                       paro_stream_t stream);
+
+/*
  * Group-wise INT4 weight-only linear y = x W^T with w^ = (q - zero) * scale
  * (page "ParoQuant: pairwise rotations that survive deployment", section
  * "From fake quantization to a real TensorRT engine": the group-wise INT4 GEMM

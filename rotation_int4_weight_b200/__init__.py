@@ -19,7 +19,7 @@ __all__ = [
     "paro_pack_weights", "paro_rotate", "paro_w4_linear", "paro_rotate_w4_linear",
     "paro_rotate_w4_linear_noalloc", "paro_get_device_status", "EXPORTED", "ParoLinear", "paro_linear",
     "paro_batched_workspace_bytes", "paro_rotate_w4_linear_batched", "paro_plan_pair_order",
-    "paro_rotate_backward_workspace_bytes", "paro_rotate_backward", "paro_set_test_hooks",
+    "paro_rotate_backward_workspace_bytes", "paro_rotate_backward", "paro_set_test_hooks", "paro_dense_rotate",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libparo.so")
@@ -43,6 +43,7 @@ EXPORTED = {
     "paro_rotate_backward_workspace_bytes": (_S, [_I, _I, _I, _I]),
     "paro_rotate_backward": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
     "paro_set_test_hooks": (_I, [ctypes.c_longlong, _I]),
+    "paro_dense_rotate": (_I, [_P, _P, _P, _I, _I, _P]),
 }
 
 
@@ -173,6 +174,16 @@ def paro_rotate_backward(x: torch.Tensor, grad: torch.Tensor, pairs=None, cos_t=
                                   workspace.numel(), _stream(stream))
     _check(st, "paro_rotate_backward")
     return (dx, dtheta, dscale), workspace
+
+
+def paro_dense_rotate(x: torch.Tensor, q: torch.Tensor, *, out=None, stream=None):
+    """The dense-rotation contrast: x~ = x Q^T for bf16 x [M, d] and bf16 Q [d, d]; bf16 [M, d]."""
+    M, d = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    st = lib.paro_dense_rotate(_ptr(_u16(x)), _ptr(_u16(q)), _ptr(_u16(out)), M, d, _stream(stream))
+    _check(st, "paro_dense_rotate")
+    return out
 
 
 def paro_w4_linear(x: torch.Tensor, qweight, scales, zeros, *, out=None, group_size: int = 128, stream=None):

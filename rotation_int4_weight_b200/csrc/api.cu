@@ -283,6 +283,25 @@ paro_status paro_rotate(const uint16_t* d_x, uint16_t* d_x_rot, int M, int d, in
   return from_cuda(e, "rotate launch");
 }
 
+paro_status paro_dense_rotate(const uint16_t* d_x, const uint16_t* d_q, uint16_t* d_out, int M, int d,
+                              paro_stream_t stream) {
+  if (M < 0) return fail(PARO_ERR_INVALID_ARG, "M = %d is negative", M);
+  if (d <= 0) return fail(PARO_ERR_INVALID_ARG, "d = %d must be positive", d);
+  if (d % 64) return fail(PARO_ERR_UNSUPPORTED, "d = %d is not a multiple of 64", d);
+  if (M == 0) return ok();
+  if (!d_x || !d_q || !d_out) return fail(PARO_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(d_x, 16) || !aligned(d_q, 16) || !aligned(d_out, 16))
+    return fail(PARO_ERR_INVALID_ARG, "x, Q and out must be 16-byte aligned");
+  const size_t xb = (size_t)M * d * 2, qb = (size_t)d * d * 2;
+  if (overlap(d_out, xb, d_x, xb) || overlap(d_out, xb, d_q, qb))
+    return fail(PARO_ERR_INVALID_ARG, "out overlaps x or Q");
+  int* status = status_ptr();
+  if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
+  cudaError_t e = paro::launch_dense_tc(d_x, d_q, reinterpret_cast<__nv_bfloat16*>(d_out), M, d, status,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  return from_cuda(e, "dense rotate launch");
+}
+
 size_t paro_rotate_backward_workspace_bytes(int M, int d, int K, int with_scale) {
   if (M <= 0 || d < 2 || (d & 1) || K < 0 || K > paro::kMaxStages) return 0;
   return paro::rot_bwd_workspace_bytes(M, d, K, with_scale != 0);
@@ -609,6 +628,7 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     paro::RotProblem rt[PARO_MAX_BATCH];
     rt[0] = rp[n - 1];
     for (int i = 0; i + 1 < n; ++i) rt[i + 1] = rp[i];
+    for (int i = 0; i < n; ++i) rt[i].perm = 1;  // x~ in the stream-K kernel's operand order
     paro::RotBatch rb;
     paro::StreamBatch sb;
     int R = 1, nt = 1;

@@ -257,6 +257,39 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
   // L2, where the prologue put them) before any of them is used.  An fp16
   // value that rounds to infinity is reported once (PARO_ERR_RANGE).
   bool ovf = false;
+  if constexpr (F16OUT) {
+    if (P.perm) {
+      // operand order of the stream-K INT4 kernel: one 16-byte store per
+      // 8-column block, (x0, x4, x1/16, x5/16, x2, x6, x3/16, x7/16), the odd
+      // columns divided by 16 to match its codes' exponent bias
+#pragma unroll 1
+      for (int b0 = tid; b0 < (d >> 3); b0 += NTHR) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = P.scale ? 1.0f / __ldg(P.scale + 8 * b0 + e) : 1.0f;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          if (r < nrows) {
+            const float4 lo = *reinterpret_cast<const float4*>(xs + (size_t)r * d + 8 * b0);
+            const float4 hi = *reinterpret_cast<const float4*>(xs + (size_t)r * d + 8 * b0 + 4);
+            const __half2 h0 = __floats2half2_rn(lo.x * f[0], hi.x * f[4]);
+            const __half2 h1 = __floats2half2_rn(lo.y * f[1] * 0.0625f, hi.y * f[5] * 0.0625f);
+            const __half2 h2 = __floats2half2_rn(lo.z * f[2], hi.z * f[6]);
+            const __half2 h3 = __floats2half2_rn(lo.w * f[3] * 0.0625f, hi.w * f[7] * 0.0625f);
+            uint4 u;
+            u.x = *reinterpret_cast<const uint32_t*>(&h0);
+            u.y = *reinterpret_cast<const uint32_t*>(&h1);
+            u.z = *reinterpret_cast<const uint32_t*>(&h2);
+            u.w = *reinterpret_cast<const uint32_t*>(&h3);
+            ovf |= half2_inf(u.x) | half2_inf(u.y) | half2_inf(u.z) | half2_inf(u.w);
+            *reinterpret_cast<uint4*>(static_cast<__half*>(P.out) + (size_t)(row0 + r) * d + 8 * b0) = u;
+          }
+        }
+      }
+      if (ovf) report_status(status, kStatusRange);
+      return true;
+    }
+  }
 #pragma unroll 1
   for (int cp0 = tid; cp0 < half; cp0 += LB * NTHR) {
     float2 sc[LB];

@@ -62,6 +62,11 @@ namespace {
 #ifndef PARO_STREAM_D2
 #define PARO_STREAM_D2 3
 #endif
+// CTAs of the one-token-tile kernel resident per SM (their registers and rings
+// must fit together)
+#ifndef PARO_STREAM_CPS1
+#define PARO_STREAM_CPS1 1
+#endif
 constexpr int kUnitBytes = kStreamRows * 64;  // 64 rows x 128 codes
 
 template <int NT>
@@ -72,8 +77,9 @@ struct Geo {
   static constexpr int SLOT = kUnitBytes + 2 * XB;
   static constexpr int PF = 4 * NT * 32 * 4;        // floats of one tile partial (fragment order)
   static constexpr int SMEM = W * D * SLOT + 1024;
+  static constexpr int CPS = NT == 1 ? PARO_STREAM_CPS1 : 1;  // CTAs per SM
   static_assert(2 * PF * 4 <= D * SLOT, "a warp's two partial tiles fit in its ring");
-  static_assert(SMEM <= 227 * 1024, "ring exceeds shared memory");
+  static_assert(SMEM * CPS <= 227 * 1024, "rings exceed shared memory");
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -147,19 +153,26 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 // operand type: P[0] = columns (0,4), P[1] = (1,5), P[2] = (2,6), P[3] = (3,7).
 //   fp16: even nibbles give 1024 + q, odd nibbles (left in bits 4..7) 1024 + 16 q;
 //   bf16: even nibbles give 128 + q, odd nibbles (moved to bits 3..6) 128 + 8 q.
+// (a & mask) | bias as one three-input logic operation
+template <uint32_t MASK, uint32_t BIAS>
+__device__ __forceinline__ uint32_t and_or(uint32_t a) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(d) : "r"(a), "n"(MASK), "n"(BIAS));
+  return d;
+}
 template <bool F16>
 __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t (&P)[4]) {
   if constexpr (F16) {
     const uint32_t w2 = w >> 8;
-    P[0] = (w & 0x000F000Fu) | 0x64006400u;
-    P[1] = (w & 0x00F000F0u) | 0x64006400u;
-    P[2] = (w2 & 0x000F000Fu) | 0x64006400u;
-    P[3] = (w2 & 0x00F000F0u) | 0x64006400u;
+    P[0] = and_or<0x000F000Fu, 0x64006400u>(w);
+    P[1] = and_or<0x00F000F0u, 0x64006400u>(w);
+    P[2] = and_or<0x000F000Fu, 0x64006400u>(w2);
+    P[3] = and_or<0x00F000F0u, 0x64006400u>(w2);
   } else {
-    P[0] = (w & 0x000F000Fu) | 0x43004300u;
-    P[1] = ((w >> 1) & 0x00780078u) | 0x43004300u;
-    P[2] = ((w >> 8) & 0x000F000Fu) | 0x43004300u;
-    P[3] = ((w >> 9) & 0x00780078u) | 0x43004300u;
+    P[0] = and_or<0x000F000Fu, 0x43004300u>(w);
+    P[1] = and_or<0x00780078u, 0x43004300u>(w >> 1);
+    P[2] = and_or<0x000F000Fu, 0x43004300u>(w >> 8);
+    P[3] = and_or<0x00780078u, 0x43004300u>(w >> 9);
   }
 }
 
@@ -197,10 +210,10 @@ __device__ __forceinline__ void cur_at(const Meta* mp, int count, long long u, C
   int pi = 0;
 #pragma unroll 1
   while (pi + 1 < count && u >= mp[pi + 1].unit_begin) ++pi;
-  const long long local = u - mp[pi].unit_begin;
+  const uint32_t local = (uint32_t)(u - mp[pi].unit_begin);
   c.pi = pi;
-  c.tile = (int)(local / mp[pi].G);
-  c.grp = (int)(local - (long long)c.tile * mp[pi].G);
+  c.tile = (int)(local / (uint32_t)mp[pi].G);
+  c.grp = (int)(local - (uint32_t)c.tile * (uint32_t)mp[pi].G);
 }
 __device__ __forceinline__ void cur_next(const Meta* mp, Cur& c) {
   if (++c.grp == mp[c.pi].G) {
@@ -211,10 +224,15 @@ __device__ __forceinline__ void cur_next(const Meta* mp, Cur& c) {
     }
   }
 }
-// first unit of part i when U units are cut into P contiguous parts
-__device__ __forceinline__ long long part_start(long long i, long long P, long long U) { return i * U / P; }
+// first unit of part i when U units are cut into P contiguous parts (32-bit:
+// a launch has fewer than 2^31 / 2^12 units, and i, P are at most a few hundred)
+__device__ __forceinline__ long long part_start(long long i, long long P, long long U) {
+  return (long long)((uint32_t)i * (uint32_t)U / (uint32_t)P);
+}
 // the part holding unit x
-__device__ __forceinline__ long long part_of(long long x, long long P, long long U) { return ((x + 1) * P - 1) / U; }
+__device__ __forceinline__ long long part_of(long long x, long long P, long long U) {
+  return (long long)((((uint32_t)x + 1u) * (uint32_t)P - 1u) / (uint32_t)U);
+}
 
 // lane (g, t) fetches one 16-bit value per row tile: t = 0 scale of row g, t = 1
 // scale of row g + 8, t = 2 zero of row g, t = 3 zero of row g + 8 (rows past
@@ -278,10 +296,15 @@ __device__ bool wait_flag(const unsigned long long* f, unsigned long long v, lon
 // grid id is in *b.tagword and whose CTAs publish flags; the INT4 CTAs request
 // a linear's activations once all its transform CTAs have published (and do
 // not wait for the whole launch).
-template <bool F16, int NT, int FU>
-__global__ void __launch_bounds__(Geo<NT>::W * 32, 1)
+// XPERM: the fp16 activations were written by this library's decode transform
+// in the MMA's operand order (every 8-column block as x0, x4, x1/16, x5/16, x2,
+// x6, x3/16, x7/16), so a 16-byte chunk is a ready B fragment; the fused and
+// flag forms always take them so.
+template <bool F16, int NT, int FU, bool XPERM>
+__global__ void __launch_bounds__(Geo<NT>::W * 32, Geo<NT>::CPS)
 w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ RotBatch rb, int* status,
                  int pdl_wait) {
+  static_assert(!XPERM || F16, "the operand-order layout is fp16");
   using Gm = Geo<NT>;
   constexpr int W = Gm::W, D = Gm::D, SLOT = Gm::SLOT, XB = Gm::XB, PF = Gm::PF;
   extern __shared__ unsigned char smem_raw[];
@@ -521,9 +544,17 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint32_t ch = (uint32_t)(4 * (t & 1) + j) ^ (uint32_t)(tok & 7);
-          pair_act(lds128(row + (ch << 4)), Bf[m][j]);
-          Bf[m][j][1] = mul2<F16>(Bf[m][j][1], kOddScale);
-          Bf[m][j][3] = mul2<F16>(Bf[m][j][3], kOddScale);
+          const uint4 u = lds128(row + (ch << 4));
+          if constexpr (XPERM) {
+            Bf[m][j][0] = u.x;
+            Bf[m][j][1] = u.y;
+            Bf[m][j][2] = u.z;
+            Bf[m][j][3] = u.w;
+          } else {
+            pair_act(u, Bf[m][j]);
+            Bf[m][j][1] = mul2<F16>(Bf[m][j][1], kOddScale);
+            Bf[m][j][3] = mul2<F16>(Bf[m][j][3], kOddScale);
+          }
         }
       } else {
 #pragma unroll
@@ -815,10 +846,14 @@ bool stream_supported(int M, int d_in, int d_out, const void* x, const void* qwe
          (reinterpret_cast<uintptr_t>(x) & 15) == 0 && (reinterpret_cast<uintptr_t>(qweight) & 15) == 0;
 }
 
+// most INT4 CTAs a launch of that token-tile count has (a flag pair and two
+// partial tiles each in the workspace)
+static int max_ctas(int NT) { return device_sm_count() * (NT == 1 ? Geo<1>::CPS : Geo<2>::CPS); }
+
 size_t stream_workspace_bytes(int max_m) {
   const int NT = max_m <= 8 ? 1 : 2;
-  return round256((size_t)device_sm_count() * 2 * 8) + round256((size_t)device_sm_count() * 2 * (4 * NT * 32 * 4) * 4) +
-         round256((size_t)kXFlagWords * 8);
+  const size_t C = (size_t)max_ctas(NT);
+  return round256(C * 2 * 8) + round256(C * 2 * (4 * NT * 32 * 4) * 4) + round256((size_t)kXFlagWords * 8);
 }
 
 cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* qw, const __half* const* sc,
@@ -868,13 +903,15 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
         return cudaErrorInvalidValue;
     }
   }
+  // the kernel's unit arithmetic is 32-bit: units times CTAs stays below 2^32
+  if (units >= (1LL << 23)) return cudaErrorInvalidValue;
   out->count = count;
   out->total_units = units;
   out->total_tiles = tiles;
   const int W = maxM <= 8 ? Geo<1>::W : Geo<2>::W;
   const long long want = (units + W - 1) / W;
   const int sms = device_sm_count();
-  const int avail = sms - reserved_ctas;
+  const int avail = sms * (maxM <= 8 ? Geo<1>::CPS : Geo<2>::CPS) - reserved_ctas;
   if (avail < 1) return cudaErrorInvalidValue;
   out->ctas = (int)(want < avail ? want : avail);
   out->ctas_a = out->ctas;
@@ -890,10 +927,10 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
     return cudaSuccess;
   }
   out->flags = static_cast<unsigned long long*>(ws);
-  out->partials = reinterpret_cast<float*>(static_cast<char*>(ws) + round256((size_t)sms * 2 * 8));
-  out->xflags = reinterpret_cast<unsigned long long*>(
-      static_cast<char*>(ws) + round256((size_t)sms * 2 * 8) +
-      round256((size_t)sms * 2 * (4 * (maxM <= 8 ? 1 : 2) * 32 * 4) * 4));
+  const size_t C = (size_t)max_ctas(maxM <= 8 ? 1 : 2);
+  out->partials = reinterpret_cast<float*>(static_cast<char*>(ws) + round256(C * 2 * 8));
+  out->xflags = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + round256(C * 2 * 8) +
+                                                      round256(C * 2 * (4 * (maxM <= 8 ? 1 : 2) * 32 * 4) * 4));
   out->tagword = out->xflags + kMaxBatch * kStreamMaxM;
   return cudaSuccess;
 }
@@ -916,7 +953,7 @@ cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* s
   const RotBatch none{};
 #define PARO_STREAM_LAUNCH(f16, nt)                                                                       \
   {                                                                                                       \
-    auto k = w4_stream_kernel<f16, nt, 0>;                                                                \
+    auto k = w4_stream_kernel<f16, nt, 0, false>;                                                         \
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                  \
     if (e != cudaSuccess) return e;                                                                       \
     return cudaLaunchKernelEx(&cfg, k, b, none, status, wait);                                            \
@@ -944,13 +981,15 @@ cudaError_t launch_stream_flagged(const StreamBatch& b, int NT, int* status, cud
   const RotBatch none{};
   cudaError_t e;
   if (NT == 1) {
-    e = cudaFuncSetAttribute(w4_stream_kernel<true, 1, -1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(w4_stream_kernel<true, 1, -1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
     if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, w4_stream_kernel<true, 1, -1>, b, none, status, 1);
+    return cudaLaunchKernelEx(&cfg, w4_stream_kernel<true, 1, -1, true>, b, none, status, 1);
   }
-  e = cudaFuncSetAttribute(w4_stream_kernel<true, 2, -1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(w4_stream_kernel<true, 2, -1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
   if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&cfg, w4_stream_kernel<true, 2, -1>, b, none, status, 1);
+  return cudaLaunchKernelEx(&cfg, w4_stream_kernel<true, 2, -1, true>, b, none, status, 1);
 }
 
 // ---- fused form -----------------------------------------------------------------------
@@ -1011,6 +1050,7 @@ cudaError_t plan_fused_rot(const RotProblem* probs, int count, RotBatch* out) {
     p.rows = 1;
     p.ring = ring;
     p.cta_begin = i;
+    p.perm = 1;  // the INT4 CTAs read x~ in their operand order
     out->p[i] = p;
   }
   out->count = count;
@@ -1041,7 +1081,7 @@ cudaError_t launch_fused_batch(const StreamBatch& b, const RotBatch& rb, int* st
   cudaError_t e;
 #define PARO_FUSED_LAUNCH(fu)                                                                             \
   {                                                                                                       \
-    auto k = w4_stream_kernel<true, 1, fu>;                                                               \
+    auto k = w4_stream_kernel<true, 1, fu, true>;                                                         \
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                  \
     if (e != cudaSuccess) return e;                                                                       \
     return cudaLaunchKernelEx(&cfg, k, b, rb, status, wait);                                              \

@@ -64,7 +64,8 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
 cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* status, cudaStream_t stream,
                                 bool pdl_wait);
 // The flag form (fp16 x~ written by a transform launched just before with
-// flags, see RotBatch): instead of waiting for the whole transform launch, the
+// flags and, per problem, perm set: x~ in the kernel's operand order, see
+// RotProblem): instead of waiting for the whole transform launch, the
 // INT4 linear requests a linear's activations once all of that linear's
 // transform CTAs have published.  b.tagword, b.xflags and every problem's
 // xf_begin / xf_count must be set.

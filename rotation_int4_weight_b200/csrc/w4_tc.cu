@@ -104,9 +104,11 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
   return d;
 }
 
-__host__ __device__ constexpr uint32_t instr_desc() {
-  // fp32 accumulate, A and B fp16, both K-major, N = BN = 256, M = 128
-  return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(MH >> 4) << 24);
+// fp32 accumulate, A and B both fp16 (bf16 = false) or both bf16, both K-major,
+// N = BN = 256, M = 128
+__host__ __device__ constexpr uint32_t instr_desc(bool bf16 = false) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((uint32_t)(BN >> 3) << 17) |
+         ((uint32_t)(MH >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -179,10 +181,15 @@ __device__ __forceinline__ TileInfo tile_info(const TcMeta* mt, int count, int t
   return TileInfo{pi, mtile * BM, ntile * BN, mt[pi].d_in / BK};
 }
 
-template <bool XF16>
+// DENSE: the dense-rotation contrast (a d x d bf16 matrix instead of INT4
+// weights): the TMA producer also loads the B tile (256 rows x 64 columns of
+// the matrix, 128-byte swizzle) straight into the tensor core's layout, A is
+// bf16 as given, and warps 0-15 only run the epilogue.
+template <bool XF16, bool DENSE = false>
 __global__ void __launch_bounds__(XF16 ? kThreadsTma : kThreadsConv, 1)
 w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
-  constexpr bool F16 = true;  // tensor-core operands are fp16 in both variants
+  static_assert(XF16 || !DENSE, "the dense form takes its A tile as given");
+  constexpr bool F16 = true;  // tensor-core operands are fp16 in both INT4 variants
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t bars[5 * kStages + 2];
   __shared__ uint32_t tmem_base_slot;
@@ -213,7 +220,7 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(b_full_a + 8 * s, XF16 ? 1 : BM);
-      mbar_init(b_full_b + 8 * s, kDqWarps * 32);
+      mbar_init(b_full_b + 8 * s, DENSE ? 1 : kDqWarps * 32);
       mbar_init(b_empty + 8 * s, 1);
       mbar_init(b_full_c + 8 * s, 1);
       mbar_init(b_full_raw + 8 * s, 1);
@@ -307,8 +314,15 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
           const int s = it % kStages;
           if (it >= kStages && !mbar_wait(b_empty + 8 * s, ((it / kStages) - 1) & 1)) { fail(); stop = true; break; }
           if (aborted()) { stop = true; break; }
-          mbar_expect_tx(b_full_c + 8 * s, C_BYTES);
-          tma_load_2d(s_base + s * STAGE_BYTES + A_BYTES + B_BYTES, &P.qmap, k * (BK / 8), ti.n0, b_full_c + 8 * s);
+          if constexpr (DENSE) {
+            // the matrix tile goes straight into the B slot
+            mbar_expect_tx(b_full_b + 8 * s, B_BYTES);
+            tma_load_2d(s_base + s * STAGE_BYTES + A_BYTES, &P.qmap, k * BK, ti.n0, b_full_b + 8 * s);
+          } else {
+            mbar_expect_tx(b_full_c + 8 * s, C_BYTES);
+            tma_load_2d(s_base + s * STAGE_BYTES + A_BYTES + B_BYTES, &P.qmap, k * (BK / 8), ti.n0,
+                        b_full_c + 8 * s);
+          }
           // fp16 activations complete the stage's A tile; bf16 ones land first and
           // are converted in place by the conversion warps
           const uint32_t bar_a = XF16 ? b_full_a + 8 * s : b_full_raw + 8 * s;
@@ -321,7 +335,7 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
   } else if (warp == kWarpMma) {
     // ---------------- MMA issuer ---------------------------------------------------
     if (lane == 0) {
-      constexpr uint32_t idesc = instr_desc();
+      constexpr uint32_t idesc = instr_desc(DENSE);
       int it = 0;
       bool ok = true;
 #pragma unroll 1
@@ -371,6 +385,7 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
       if (T < 0) break;
       const TileInfo ti = tile_info(meta, count, T);
       const TcMeta& P = meta[ti.pi];
+      if constexpr (!DENSE) {
       const int G = P.d_in / kGroup;
       const int rA = ti.n0 + t;
       const bool okA = rA < P.d_out;
@@ -424,6 +439,7 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
           ++it;
         }
       }
+      }  // !DENSE
       if (stop) break;
 
       // ---------------- epilogue of this tile --------------------------------------
@@ -481,13 +497,14 @@ w4_tc_kernel(const __grid_constant__ TcBatch b, int* status) {
     // commit that read it (earlier phases have completed before those could be
     // issued); a wait that gives up again is reported again
     const uint32_t bar_a = XF16 ? b_full_a : b_full_raw;
+    const uint32_t bar_w = DENSE ? b_full_b : b_full_c;  // the weight tile's copy
     auto last_of = [](int n, int slot) { return n > slot ? slot + ((n - 1 - slot) / kStages) * kStages : -1; };
     for (int s = 0; s < kStages; ++s) {
       const int jt = last_of(s_issued, s), jm = last_of(s_committed, s);
       bool landed = true;
       if (jt >= 0) {
         const uint32_t par = (uint32_t)((jt / kStages) & 1);
-        landed = mbar_wait(bar_a + 8 * s, par) && mbar_wait(b_full_c + 8 * s, par);
+        landed = mbar_wait(bar_a + 8 * s, par) && mbar_wait(bar_w + 8 * s, par);
       }
       if (jm >= 0) landed = mbar_wait(b_empty + 8 * s, (uint32_t)((jm / kStages) & 1)) && landed;
       if (!landed) report_status(status, kStatusTimeout);
@@ -588,6 +605,55 @@ cudaError_t launch_w4_tc_batch(const TcLinear* lins, int count, bool x_f16, int*
     if (e != cudaSuccess) return e;
     w4_tc_kernel<false><<<grid, kThreadsConv, SMEM_BYTES, stream>>>(b, status);
   }
+  return cudaPeekAtLastError();
+}
+
+bool dense_supported(int M, int d, const void* x, const void* q) {
+  return M >= 1 && d >= BK && d % BK == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(q) & 15) == 0;
+}
+
+cudaError_t launch_dense_tc(const uint16_t* x, const uint16_t* q, __nv_bfloat16* y, int M, int d, int* status,
+                            cudaStream_t stream) {
+  if (!dense_supported(M, d, x, q)) return cudaErrorInvalidValue;
+  EncodeTiled enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  TcBatch b{};
+  TcProblem& P = b.p[0];
+  const cuuint32_t elem[2] = {1, 1};
+  {  // bf16 activations [M][d]: box 64 columns x 256 tokens, 128-byte swizzle
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    const cuuint32_t box[2] = {BK, BM};
+    if (enc(&P.xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, elem,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {  // bf16 matrix [d][d] (row n = output channel n): box 64 columns x 256 rows, 128-byte swizzle
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)d};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    const cuuint32_t box[2] = {BK, BN};
+    if (enc(&P.qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(q), dims, strides, box, elem,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  P.xraw = x;
+  P.y = y;
+  P.M = M;
+  P.d_in = d;
+  P.d_out = d;
+  P.n_tiles = (d + BN - 1) / BN;
+  P.tile_begin = 0;
+  b.count = 1;
+  b.total_tiles = ((M + BM - 1) / BM) * P.n_tiles;
+  const int sms = device_sm_count();
+  const int grid = b.total_tiles < sms ? b.total_tiles : sms;
+  cudaError_t e = cudaFuncSetAttribute(w4_tc_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  w4_tc_kernel<true, true><<<grid, kThreadsTma, SMEM_BYTES, stream>>>(b, status);
   return cudaPeekAtLastError();
 }
 

@@ -48,6 +48,13 @@ bool tc_supported(int M, int d_in, int d_out, const void* x);
 // 256 x 256 output tiles of all of them, the linears with the longest K first.
 cudaError_t launch_w4_tc_batch(const TcLinear* lins, int count, bool x_f16, int* status, cudaStream_t stream);
 
+// The dense-rotation contrast: y = x Q^T for bf16 x [M][d] and a bf16 d x d
+// matrix Q (row n = output channel n), on the same tensor-core pipeline with
+// the matrix tiles copied by TMA instead of dequantised; bf16 out.
+bool dense_supported(int M, int d, const void* x, const void* q);
+cudaError_t launch_dense_tc(const uint16_t* x, const uint16_t* q, __nv_bfloat16* y, int M, int d, int* status,
+                            cudaStream_t stream);
+
 cudaError_t launch_w4_tc(const uint16_t* x, bool x_f16, const uint32_t* qweight, const __half* scales,
                          const __half* zeros, __nv_bfloat16* y, int M, int d_in, int d_out, int* status,
                          cudaStream_t stream);

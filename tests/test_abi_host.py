@@ -57,6 +57,15 @@ def test_test_hooks_validate_and_reset():
     assert paro.lib.paro_set_test_hooks(0, 0) == OK
 
 
+@pytest.mark.parametrize("args,expect", [
+    ((A, B, C, 4, 96), UNSUPPORTED), ((A, B, C, -1, 512), INVALID), ((A, B, C, 4, 0), INVALID),
+    ((None, B, C, 4, 512), INVALID), ((MIS, B, C, 4, 512), INVALID), ((A, B, A, 4, 512), INVALID),
+    ((A, B, C, 0, 512), OK),
+])
+def test_dense_rotate_validation(args, expect):
+    assert paro.lib.paro_dense_rotate(*args, None) == expect
+
+
 def test_workspace_bytes():
     """The fp16 transformed activations (2 M d_in bytes, rounded up to 256), plus,
     up to 16 tokens, the stream-K kernel's flags and partial tiles: the same
@@ -68,7 +77,7 @@ def test_workspace_bytes():
     assert paro.paro_workspace_bytes(2048, 4096) == xt(2048, 4096)
     extra8 = paro.paro_workspace_bytes(1, 512) - xt(1, 512)
     extra16 = paro.paro_workspace_bytes(16, 512) - xt(16, 512)
-    assert extra8 > 0 and extra8 % 256 == 0 and extra16 > extra8
+    assert extra8 > 0 and extra8 % 256 == 0 and extra16 > 0 and extra16 % 256 == 0
     for M, d in [(1, 512), (3, 1536), (8, 8960), (9, 128), (16, 4096)]:
         w = paro.paro_workspace_bytes(M, d)
         assert w % 256 == 0
