@@ -139,7 +139,7 @@ class Linear:
         self.x = torch.from_numpy(p.x).to(dev).to(torch.bfloat16)
         self.xr = torch.empty_like(self.x)
         self.y = torch.empty(p.M, p.d_out, dtype=torch.bfloat16, device=dev)
-        self.ws = torch.empty(max(paro.paro_workspace_bytes(p.M, p.d_in), 256), dtype=torch.uint8, device=dev)
+        self.ws = torch.zeros(max(paro.paro_workspace_bytes(p.M, p.d_in), 256), dtype=torch.uint8, device=dev)
         self.x_host = torch.empty(self.x.shape, dtype=torch.bfloat16, pin_memory=True)
         self.x_host.copy_(self.x)
         self.y_host = torch.empty(self.y.shape, dtype=torch.bfloat16, pin_memory=True)
@@ -232,7 +232,7 @@ class Unit:
             descs = [paro.paro_linear(l.x, l.pairs, l.cos, l.sin, l.scale, l.qw, l.sc, l.z, l.y) for l in grp]
             plain = [paro.paro_linear(l.x, None, None, None, None, l.qw0, l.sc0, l.z0, l.y) for l in grp]
             need = paro.paro_batched_workspace_bytes(descs)
-            ws = __import__("torch").empty(max(need, 256), dtype=__import__("torch").uint8, device=lins[0].x.device)
+            ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=lins[0].x.device)
             self.calls.append((grp, descs, plain, ws))
 
     def run(self, paro, variant):

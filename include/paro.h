@@ -209,8 +209,9 @@ PARO_API size_t paro_workspace_bytes(int M, int d_in);
  * paragraph).  y = (diag(1/s) R_K ... R_1 x) W~^T.  The transformed
  * activations never leave the GPU as bf16: they are handed to the linear in
  * fp16 through d_workspace (paro_workspace_bytes(M, d_in) bytes, 256-byte
- * aligned, caller-owned, contents undefined between calls; two calls that run
- * at the same time need two workspaces).  Up to 16 tokens with that full
+ * aligned, caller-owned; zero before its first use, as for
+ * paro_rotate_w4_linear_batched, after which the calls keep it valid; two
+ * calls that run at the same time need two workspaces).  Up to 16 tokens with that full
  * workspace the call runs as paro_rotate_w4_linear_batched does for one
  * linear (one launch at one token: its first CTA transforms while the others
  * stream the weights); given only the activations' 2 M d_in bytes (rounded
@@ -249,8 +250,8 @@ typedef struct {
  * transformed activations of every linear (paro_workspace_bytes(M, d_in)
  * each, in order), then, when every M is at most 16, the publication flags
  * and partial sums of the stream-K INT4 linear (2 flags and 2 partial
- * 64-row tiles per SM) and the flags of the transform's CTAs (at most 128,
- * plus a tag word) that the INT4 linear waits on (see below).
+ * 64-row tiles per CTA), the flags of the transform's CTAs (at most 128) that
+ * the INT4 linear waits on, and the workspace's launch epoch (see below).
  * The second part is optional: given only the first, the call runs the older
  * per-block kernel.
  */
@@ -266,7 +267,10 @@ PARO_API size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int co
  * section "From fake quantization to a real TensorRT engine").  h_layers is a
  * HOST array read during the call; d_workspace holds
  * paro_batched_workspace_bytes(h_layers, count) bytes (256-byte aligned,
- * caller-owned, undefined between calls).  Results equal count separate calls
+ * caller-owned; zero before its first use, e.g. by cudaMemsetAsync, after
+ * which the calls keep it valid: they leave it holding their own state, which
+ * later calls rely on, so it must not be written by anything else between
+ * calls).  Results equal count separate calls
  * of paro_rotate_w4_linear.  Every linear is validated before anything is
  * enqueued; the message of paro_last_error() names the failing index.  When no
  * linear has a transform (K == 0 and d_scale == NULL for all) and every M is
@@ -283,10 +287,13 @@ PARO_API size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int co
  * tokens the transform launch's CTAs each publish such a flag, and the INT4
  * launch after it requests a linear's activations once all of that linear's
  * transform CTAs have published, not when the whole transform launch is done.
- * The stream-K kernel's publication flags need no clearing: a flag holds the
- * id of the launch that wrote it, so one left by another launch, or never
- * written, is never taken for this launch's.  Two calls that may run at the
- * same time need two workspaces.
+ * Every flag a launch publishes (the transforms' "x~ is written" flags and
+ * the stream-K kernel's partial-tile flags) holds 2E + 1 for the workspace's
+ * launch epoch E, which every CTA reads once the previous kernel has
+ * completed and which the launch's last CTA advances: a flag left by an
+ * earlier call, or by an earlier replay of the same CUDA graph, is never taken
+ * for this launch's, and calls captured in a graph may be replayed with new
+ * inputs.  Two calls that may run at the same time need two workspaces.
  */
 PARO_API paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count, int group_size,
                                                   void* d_workspace, size_t workspace_bytes,

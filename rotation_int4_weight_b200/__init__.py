@@ -206,8 +206,8 @@ def paro_rotate_w4_linear(x: torch.Tensor, pairs, cos_t, sin_t, scale, qweight, 
     if out is None:
         out = torch.empty(M, d_out, dtype=torch.bfloat16, device=x.device)
     need = paro_workspace_bytes(M, d_in)
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    if workspace is None:  # zero before its first use (the calls keep it valid afterwards)
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=x.device)
     st = lib.paro_rotate_w4_linear(_ptr(_u16(x)), _K(pairs), _ptr(pairs), _ptr(cos_t), _ptr(sin_t), _ptr(scale),
                                    _ptr(qweight), _ptr(_u16(scales)), _ptr(_u16(zeros)), _ptr(_u16(out)),
                                    M, d_in, d_out, group_size, _ptr(workspace), workspace.numel(),
@@ -250,8 +250,8 @@ def paro_rotate_w4_linear_batched(layers, *, workspace=None, group_size: int = 1
     per linear, a transform launch and an INT4-linear launch up to 64 tokens."""
     arr = (ParoLinear * len(layers))(*layers)
     need = int(lib.paro_batched_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), len(layers)))
-    if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+    if workspace is None:  # zero before its first use (the calls keep it valid afterwards)
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device="cuda")
     st = lib.paro_rotate_w4_linear_batched(ctypes.cast(arr, ctypes.c_void_p), len(layers), group_size,
                                            _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "paro_rotate_w4_linear_batched")

@@ -77,7 +77,7 @@ class ColumnParallelLinear:
         import rotation_int4_weight_b200 as paro
         need = paro.paro_workspace_bytes(x.shape[0], x.shape[1])
         if self._ws is None or self._ws.numel() < need:
-            self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+            self._ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=x.device)
         return paro.paro_rotate_w4_linear(x, *self.tables, *shard, workspace=self._ws)
 
     def local(self, x: torch.Tensor) -> torch.Tensor:

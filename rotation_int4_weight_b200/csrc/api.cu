@@ -637,10 +637,10 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     if (e != cudaSuccess) return from_cuda(e, "batched decode plan");
     // at most 16 rows of at most 8 linears, one row or more a CTA: the flag
     // area always suffices; checked so that no CTA could write past it
-    if (rb.total_ctas > paro::kXFlagWords - 1)
+    if (rb.total_ctas > paro::kXFlagWords)
       return fail(PARO_ERR_UNSUPPORTED, "%d transform CTAs exceed the workspace's %d flags", rb.total_ctas,
-                  paro::kXFlagWords - 1);
-    rb.tagword = sb.tagword;
+                  paro::kXFlagWords);
+    rb.ctl = sb.ctl;
     rb.xflags = sb.xflags;
     rb.skip_flags = paro::hook_skip_ready_flags();
     for (int i = 0; i < n; ++i) {

@@ -33,18 +33,12 @@ __global__ void __launch_bounds__(kRotThreads)
 rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_trigger, int pdl_wait) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ __align__(8) uint64_t bars[rotdec::kRotMaxRing];
-  unsigned long long gid = 0;
-  if (batch.tagword) {
-    asm volatile("mov.u64 %0, %%gridid;\n" : "=l"(gid));
-    // the INT4 linear launched after this grid reads the word before it lets
-    // its own dependents (the next transform) launch, so it sees this id
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-      asm volatile("st.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(batch.tagword), "l"(gid) : "memory");
-      __threadfence();
-    }
-    __syncthreads();
-  }
-  if (pdl_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // with flags, the INT4 launch that follows may start only once this grid has
+  // waited for the previous kernel (it takes the launch epoch at its start, which
+  // the previous INT4 launch on the workspace advanced at its end): the CTAs
+  // let it launch right after that wait, inside the transform
+  const bool flagged = batch.xflags != nullptr;
+  if (pdl_trigger && !flagged) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   int pi = 0;
 #pragma unroll 1
   while (pi + 1 < batch.count && (int)blockIdx.x >= batch.p[pi + 1].cta_begin) ++pi;
@@ -53,20 +47,28 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
   const int rp = P.rows > 0 && P.rows < R ? P.rows : R;
   const int row0 = ((int)blockIdx.x - P.cta_begin) * rp;
   bool done;
+  const bool trig_late = pdl_trigger && flagged;
   if (R > 1 && rp == 1) {
     // a linear too wide for more than one row a CTA (its stage tables need the
     // room): the one-row body, whose registers allow 7 pairs a thread and
     // round, so a stage of up to 13888 channels is one round, not several
-    done = rotdec::rot_decode_cta<1, F16OUT, 7, kRotThreads>(P, row0, smem, bars, status, pdl_wait != 0);
+    done = rotdec::rot_decode_cta<1, F16OUT, 7, kRotThreads>(P, row0, smem, bars, status, pdl_wait != 0,
+                                                             trig_late);
   } else {
-    done = rotdec::rot_decode_cta<R, F16OUT, U, kRotThreads>(P, row0, smem, bars, status, pdl_wait != 0);
+    done = rotdec::rot_decode_cta<R, F16OUT, U, kRotThreads>(P, row0, smem, bars, status, pdl_wait != 0,
+                                                             trig_late);
   }
-  if (batch.xflags && done && !batch.skip_flags) {
-    // every thread's x~ stores, then this CTA's flag
+  if (flagged && done && !batch.skip_flags) {
+    // every thread's x~ stores, then this CTA's flag (the tag of the launch
+    // epoch, read after this grid's wait for the previous kernel)
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0)
-      asm volatile("st.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(batch.xflags + blockIdx.x), "l"(gid) : "memory");
+    if (threadIdx.x == 0) {
+      unsigned long long e;
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];\n" : "=l"(e) : "l"(batch.ctl) : "memory");
+      asm volatile("st.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(batch.xflags + blockIdx.x), "l"(2ull * e + 1ull)
+                   : "memory");
+    }
   }
 }
 

@@ -27,10 +27,11 @@ struct RotProblem {
 struct RotBatch {
   RotProblem p[kMaxBatch];
   // optional (the INT4 linear that follows then waits per linear, not for the
-  // whole grid): CTA 0 writes this launch's grid id to *tagword before the grid
-  // lets its dependents launch, and every CTA sets xflags[its index] to the
-  // same id once its rows of x~ are written
-  unsigned long long* tagword;
+  // whole grid): every CTA, once it has waited for the previous kernel, takes
+  // the tag 2E + 1 from the epoch word *ctl (advanced by the last CTA of the
+  // previous INT4 launch on this workspace), lets its dependents launch, and
+  // sets xflags[its index] to the tag once its rows of x~ are written
+  unsigned long long* ctl;
   unsigned long long* xflags;
   int skip_flags;  // test hook: publish no xflags (the INT4 linear's waits then run out)
   int count;

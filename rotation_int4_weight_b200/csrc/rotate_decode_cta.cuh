@@ -83,9 +83,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 // P.rows (at most R; 0 means R); smem holds d RP 4 + ring 6 d bytes (16-byte
 // aligned), bars kRotMaxRing mbarriers.
 // Returns true when the rows were written (uniform over the CTA).
+// trigger_after_wait: let the grid's dependents launch right after the wait
+// for the previous kernel (rather than earlier).
 template <int R, bool F16OUT, int U, int NTHR>
 __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, unsigned char* smem, uint64_t* bars,
-                                               int* status, bool pdl_wait) {
+                                               int* status, bool pdl_wait, bool trigger_after_wait = false) {
   constexpr int kProd = NTHR - 32;  // the table-fetching thread (lane 0 of the last warp)
   constexpr int kComp = NTHR - 32;  // rotating threads
   const int d = P.d, K = P.K, half = d >> 1, ring = P.ring;
@@ -131,6 +133,7 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
   // the previous kernel finishes; the rows (which it may have written) and the
   // output (which it may still read) wait for it to complete
   if (pdl_wait) asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  if (trigger_after_wait) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   // rows -> xs as fp32: each thread two adjacent channels of every row, the
   // loads of LB channel pairs issued before their stores so that their
   // latencies overlap

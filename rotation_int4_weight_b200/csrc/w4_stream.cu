@@ -33,8 +33,10 @@
 // A tile split between warps of a CTA is summed in shared memory at the end, in
 // warp order.  A tile split between CTAs goes through the workspace: every CTA
 // holding part of it but the last writes its partial tile and then a flag
-// holding this launch's grid id (a flag left by another launch, or never
-// written, never matches, so the workspace needs no clearing between calls);
+// holding this launch's tag, 2E + 1 for the workspace's launch epoch E (a flag
+// left by another launch or by an earlier replay of the same CUDA graph, or
+// never written, never matches: the last CTA of every launch advances E, so
+// the workspace needs clearing only once, before its first use);
 // the tile's last CTA waits (bounded) for the flags of the earlier CTAs, which
 // were launched no later than it, and sums the partials in CTA order.  Every
 // sum has a fixed order, so the result does not depend on timing.
@@ -264,12 +266,27 @@ __device__ __forceinline__ void store_tile(const Meta& P, int tile, int g, int t
   }
 }
 
-// This launch's grid id: a flag holding it was written by this launch (a word
-// left by an earlier launch, or never written, holds another value).
-__device__ __forceinline__ unsigned long long grid_tag() {
-  unsigned long long gid;
-  asm volatile("mov.u64 %0, %%gridid;\n" : "=l"(gid));
-  return gid;
+// This launch's tag, 2E + 1 for the workspace's launch epoch E read after the
+// launch's dependency point (the previous launch on the workspace has then
+// completed, and no CTA of this launch advances E before every CTA has read
+// it): a flag holding it was written by this launch; a word left by an earlier
+// launch, by an earlier replay of the same graph, or never written (zero)
+// holds another value.
+__device__ __forceinline__ unsigned long long launch_tag(const unsigned long long* ctl) {
+  unsigned long long e;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];\n" : "=l"(e) : "l"(ctl) : "memory");
+  return 2ull * e + 1ull;
+}
+// Every CTA of a launch that has a workspace calls this once, last: the CTA
+// that completes the count advances the epoch (the count wraps back to zero).
+__device__ __forceinline__ void finish_cta(unsigned long long* ctl) {
+  if (!ctl) return;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned old = atomicInc(reinterpret_cast<unsigned*>(ctl + 1), gridDim.x - 1);
+    if (old == gridDim.x - 1) atomicAdd(ctl, 1ull);
+  }
 }
 __device__ __forceinline__ void st_flag(unsigned long long* f, unsigned long long v) {
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(f), "l"(v) : "memory");
@@ -290,12 +307,13 @@ __device__ bool wait_flag(const unsigned long long* f, unsigned long long v, lon
 
 // FU > 0: the fused form (one token per linear): CTAs 0 .. rb.count - 1 run the
 // activation transform of one linear each, FU pairs per thread and round, and
-// publish a flag holding this launch's grid id once its x~ is written; the
-// INT4 CTAs request a linear's activations only after its flag.
-// FU < 0: the flag form: the transform ran in the launch just before, whose
-// grid id is in *b.tagword and whose CTAs publish flags; the INT4 CTAs request
-// a linear's activations once all its transform CTAs have published (and do
-// not wait for the whole launch).
+// publish a flag holding this launch's tag once its x~ is written; the INT4
+// CTAs request a linear's activations only after its flag.
+// FU < 0: the flag form: the transform ran in the launch just before and its
+// CTAs publish flags holding the same launch tag (read from the workspace's
+// epoch after the previous INT4 launch completed); the INT4 CTAs request a
+// linear's activations once all its transform CTAs have published (and do not
+// wait for the whole launch).
 // XPERM: the fp16 activations were written by this library's decode transform
 // in the MMA's operand order (every 8-column block as x0, x4, x1/16, x5/16, x2,
 // x6, x3/16, x7/16), so a 16-byte chunk is a ready B fragment; the fused and
@@ -311,17 +329,10 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   __shared__ __align__(8) uint64_t bars[W * D];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  // flag form: the preceding transform's grid id, read before this grid lets
-  // the next transform (which rewrites it) launch
-  __shared__ unsigned long long s_xtag;
-  if constexpr (FU < 0) {
-    if (threadIdx.x == 0) {
-      unsigned long long v;
-      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];\n" : "=l"(v) : "l"(b.tagword) : "memory");
-      s_xtag = v;
-    }
-    __syncthreads();
-  }
+  // flag form: the preceding transform let this grid launch only after it had
+  // waited for the previous launch, so the epoch is already this launch's
+  unsigned long long ltag = 0;
+  if constexpr (FU < 0) ltag = launch_tag(b.ctl);
   // a programmatic dependent (the next call's transform) may start its table
   // fetches as SMs free up; it waits for this grid before touching its data
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
@@ -336,8 +347,9 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
         // the asynchronous proxy after seeing it)
         __threadfence();
         __syncthreads();
-        if (threadIdx.x == 0 && !rb.skip_flags) st_flag(b.xflags + blockIdx.x, grid_tag());
+        if (threadIdx.x == 0 && !rb.skip_flags) st_flag(b.xflags + blockIdx.x, launch_tag(b.ctl));
       }
+      finish_cta(b.ctl);
       return;
     }
   }
@@ -401,6 +413,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   // (the flag form orders everything after the transform's flags instead: the
   // transform waited for the previous launch before it published any)
   if (FU >= 0 && pdl_wait) asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  if (FU >= 0 && b.ctl) ltag = launch_tag(b.ctl);
   // the activations of the unit in slot s (with the slot's arrival; its codes
   // were requested without one)
   auto issue_x = [&](const Cur& c, int s) {
@@ -413,9 +426,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   // fused form (lane 0): linears whose x~ flag was seen, and slots whose
   // activations are still to be requested
   uint32_t xready = 0u, xpend = 0u;
-  unsigned long long xtag = 0;
-  if constexpr (FU > 0) xtag = grid_tag();
-  if constexpr (FU < 0) xtag = s_xtag;
+  const unsigned long long xtag = ltag;
   auto x_ready = [&](int pi, bool block) -> bool {
     if (FU == 0 || ((xready >> pi) & 1u)) return true;
     const unsigned long long* f = FU > 0 ? b.xflags + pi : b.xflags + b.p[pi].xf_begin;
@@ -656,7 +667,10 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   }
   // a warp that gave up voids the CTA's result: none of its remaining tiles is
   // written and no partial is published (a CTA waiting for one gives up too)
-  if (__syncthreads_or(!ok)) return;
+  if (__syncthreads_or(!ok)) {
+    finish_cta(b.ctl);
+    return;
+  }
 
   // ---- the last tile, and the partial tiles in shared memory -------------------------
   // slot 0: the warp's first tile when it began before the warp's units;
@@ -709,11 +723,11 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   // ---- combine: the warp holding a split tile's first unit in this CTA sums the
   // warps' partials in warp order.  A tile that crosses the CTA's bounds then
   // goes through the workspace: every CTA but the tile's last publishes its
-  // partial and a flag (this launch's grid id) and moves on; the tile's last
+  // partial and a flag (this launch's tag) and moves on; the tile's last
   // CTA waits for the flags of the earlier CTAs, which started no later than
   // it did, and sums the partials in CTA order.  Publishing comes first (the
   // warp's last tile), so no warp waits while holding back a partial. ------------
-  const unsigned long long tag = grid_tag();
+  const unsigned long long tag = ltag;
 #pragma unroll 1
   for (int pass = 0; pass < 2; ++pass) {
     const int which = 1 - pass;
@@ -807,6 +821,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
         for (int e = 0; e < 4; ++e) tot[rt][m][e] += sum[rt][m][e];
     store_tile<NT>(P, tile, g, t, tot);
   }
+  finish_cta(b.ctl);
 }
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -853,7 +868,8 @@ static int max_ctas(int NT) { return device_sm_count() * (NT == 1 ? Geo<1>::CPS 
 size_t stream_workspace_bytes(int max_m) {
   const int NT = max_m <= 8 ? 1 : 2;
   const size_t C = (size_t)max_ctas(NT);
-  return round256(C * 2 * 8) + round256(C * 2 * (4 * NT * 32 * 4) * 4) + round256((size_t)kXFlagWords * 8);
+  return round256(C * 2 * 8) + round256(C * 2 * (4 * NT * 32 * 4) * 4) + round256((size_t)kXFlagWords * 8) +
+         256;  // the launch epoch and the finished-CTA count
 }
 
 cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* qw, const __half* const* sc,
@@ -931,7 +947,7 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
   out->partials = reinterpret_cast<float*>(static_cast<char*>(ws) + round256(C * 2 * 8));
   out->xflags = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + round256(C * 2 * 8) +
                                                       round256(C * 2 * (4 * (maxM <= 8 ? 1 : 2) * 32 * 4) * 4));
-  out->tagword = out->xflags + kMaxBatch * kStreamMaxM;
+  out->ctl = out->xflags + round256((size_t)kXFlagWords * 8) / 8;
   return cudaSuccess;
 }
 

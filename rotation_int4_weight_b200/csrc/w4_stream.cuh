@@ -34,7 +34,12 @@ struct StreamBatch {
   float* partials;               // two tile partials per CTA (workspace)
   unsigned long long* xflags;    // fused form: one per linear, set when its x~ is written (workspace);
                                  // flag form: one per CTA of the preceding transform launch
-  unsigned long long* tagword;   // flag form: the grid id of the preceding transform launch
+  // the workspace's launch epoch E (ctl[0]) and a wrapping count of the CTAs
+  // of the current launch that have finished (the low word of ctl[1]): every
+  // flag a launch publishes holds 2E + 1 for the E of that launch, and its last
+  // CTA advances E, so a flag left by an earlier launch (or a replay of the
+  // same CUDA graph) never matches; null in the tile-split form
+  unsigned long long* ctl;
   // CTAs 0 .. ctas_a - 1 split units [0, units_a) evenly and the others the rest
   // (the fused form gives the widest linear, whose x~ comes last, fewer units a
   // CTA); ctas_a = ctas, units_a = total_units is the even split
@@ -67,11 +72,11 @@ cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* s
 // flags and, per problem, perm set: x~ in the kernel's operand order, see
 // RotProblem): instead of waiting for the whole transform launch, the
 // INT4 linear requests a linear's activations once all of that linear's
-// transform CTAs have published.  b.tagword, b.xflags and every problem's
+// transform CTAs have published.  b.ctl, b.xflags and every problem's
 // xf_begin / xf_count must be set.
 cudaError_t launch_stream_flagged(const StreamBatch& b, int NT, int* status, cudaStream_t stream);
-// Workspace words of the flag form: the tag word and one flag per transform CTA.
-constexpr int kXFlagWords = kMaxBatch * kStreamMaxM + 1;
+// Workspace words of the flag form: one flag per transform CTA.
+constexpr int kXFlagWords = kMaxBatch * kStreamMaxM;
 
 // The fused form for one token per linear: the kernel's first rb.count CTAs
 // each run the activation transform of one linear (writing its fp16 x~, the

@@ -57,7 +57,7 @@ def _call_noalloc(a, y, stream):
 def _call_with_workspace(a):
     """The workspace-taking call, given a workspace of the scratch array's size
     (the no-alloc call's kernel choice depends on the bytes it can use)."""
-    ws = torch.empty(SCRATCH_BYTES, dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(SCRATCH_BYTES, dtype=torch.uint8, device=DEV)
     return paro.paro_rotate_w4_linear(a["x"], a["pairs"], a["cos"], a["sin"], a["scale"], a["qw"], a["sc"], a["z"],
                                       workspace=ws)
 
