@@ -72,7 +72,9 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
   }
 }
 
-size_t rot_smem(int d, int R, int ring) { return (size_t)d * R * 4 + (size_t)ring * 6 * d; }
+size_t rot_smem(int d, int R, int ring, bool rcp = false) {
+  return (size_t)d * R * 4 + (size_t)ring * 6 * d + (rcp ? (size_t)d * 4 : 0);
+}
 
 }  // namespace
 
@@ -101,6 +103,8 @@ cudaError_t plan_rot_batch(const RotProblem* probs, int count, RotBatch* out, in
     int ring = p.K < 1 ? 1 : p.K;
     if (ring > 8) ring = 8;
     while (ring > 1 && rot_smem(p.d, rows, ring) > kRotSmemBudget) --ring;
+    // 1/scale in shared memory when it fits beside the same ring
+    p.rcp = rot_smem(p.d, rows, ring, true) <= kRotSmemBudget;
     p.rows = rows;
     p.ring = ring;
     p.cta_begin = ctas;
@@ -118,7 +122,7 @@ cudaError_t launch_rot_batch(const RotBatch& b, int R, bool f16_out, int* status
   size_t smem = 0;
   for (int i = 0; i < b.count; ++i) {
     const int rows = b.p[i].rows > 0 && b.p[i].rows < R ? b.p[i].rows : R;
-    const size_t s = rot_smem(b.p[i].d, rows, b.p[i].ring);
+    const size_t s = rot_smem(b.p[i].d, rows, b.p[i].ring, b.p[i].rcp != 0);
     smem = s > smem ? s : smem;
   }
   const int trig = pdl_trigger ? 1 : 0, wait = pdl_wait ? 1 : 0;

@@ -19,6 +19,8 @@ struct RotProblem {
   // filled by plan_rot_batch
   int perm;               // fp16 out for the stream-K INT4 kernel: every 8-column block stored as
                           // (x0, x4, x1/16, x5/16, x2, x6, x3/16, x7/16), its MMA operand order
+  int rcp;                // 1/scale kept in shared memory after the table ring (computed before
+                          // the wait for the previous kernel), else computed in the final pass
   int rows;               // token rows a CTA (<= the launch's R; 0 means R)
   int ring;               // stages of tables held in shared memory at once
   int cta_begin;          // first CTA of this problem

@@ -80,8 +80,8 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 
 
 // Transforms rows row0 .. row0 + RP - 1 of problem P with NTHR threads, RP =
-// P.rows (at most R; 0 means R); smem holds d RP 4 + ring 6 d bytes (16-byte
-// aligned), bars kRotMaxRing mbarriers.
+// P.rows (at most R; 0 means R); smem holds d RP 4 + ring 6 d (+ 4 d with
+// P.rcp) bytes (16-byte aligned), bars kRotMaxRing mbarriers.
 // Returns true when the rows were written (uniform over the CTA).
 // trigger_after_wait: let the grid's dependents launch right after the wait
 // for the previous kernel (rather than earlier).
@@ -128,6 +128,14 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
       bulk_prefetch_l2(P.sin_t + off, bytes);
     }
     if (P.scale && (reinterpret_cast<uintptr_t>(P.scale) & 15) == 0) bulk_prefetch_l2(P.scale, (size_t)4 * d);
+  }
+  // 1/scale into shared memory while the previous kernel may still run (the
+  // scale is a layer constant, like the tables); the barrier after the rows
+  // are staged orders these stores before the final pass reads them
+  float* rcp = P.rcp ? reinterpret_cast<float*>(tab + (size_t)ring * stage_bytes) : nullptr;
+  if (rcp) {
+#pragma unroll 4
+    for (int c = tid; c < d; c += NTHR) rcp[c] = P.scale ? 1.0f / __ldg(P.scale + c) : 1.0f;
   }
   // launched as a programmatic dependent: the tables above may be fetched while
   // the previous kernel finishes; the rows (which it may have written) and the
@@ -268,8 +276,17 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
 #pragma unroll 1
       for (int b0 = tid; b0 < (d >> 3); b0 += NTHR) {
         float f[8];
+        if (rcp) {
+          const float4 r0 = *reinterpret_cast<const float4*>(rcp + 8 * b0);
+          const float4 r1 = *reinterpret_cast<const float4*>(rcp + 8 * b0 + 4);
+          f[0] = r0.x; f[1] = r0.y; f[2] = r0.z; f[3] = r0.w;
+          f[4] = r1.x; f[5] = r1.y; f[6] = r1.z; f[7] = r1.w;
+        } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = P.scale ? 1.0f / __ldg(P.scale + 8 * b0 + e) : 1.0f;
+          for (int e = 0; e < 8; ++e) f[e] = P.scale ? __ldg(P.scale + 8 * b0 + e) : 1.0f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = 1.0f / f[e];
+        }
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           if (r < nrows) {
@@ -300,14 +317,17 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
     for (int q = 0; q < LB; ++q) {
       const int cp = cp0 + q * NTHR;
       sc[q] = make_float2(1.0f, 1.0f);
-      if (P.scale && cp < half) sc[q] = make_float2(__ldg(P.scale + 2 * cp), __ldg(P.scale + 2 * cp + 1));
+      if (cp < half) {
+        if (rcp) sc[q] = *reinterpret_cast<const float2*>(rcp + 2 * cp);
+        else if (P.scale) sc[q] = make_float2(__ldg(P.scale + 2 * cp), __ldg(P.scale + 2 * cp + 1));
+      }
     }
 #pragma unroll
     for (int q = 0; q < LB; ++q) {
       const int cp = cp0 + q * NTHR;
       if (cp >= half) continue;
       const int c = 2 * cp;
-      const float f0 = 1.0f / sc[q].x, f1 = 1.0f / sc[q].y;
+      const float f0 = rcp ? sc[q].x : 1.0f / sc[q].x, f1 = rcp ? sc[q].y : 1.0f / sc[q].y;
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         if (r < nrows) {

@@ -69,13 +69,28 @@ namespace {
 #ifndef PARO_STREAM_CPS1
 #define PARO_STREAM_CPS1 1
 #endif
+// ring slots per warp when every linear of the launch has one token, and
+// whether that geometry is used at all
+#ifndef PARO_STREAM_D0
+#define PARO_STREAM_D0 2
+#endif
+#ifndef PARO_STREAM_ONE
+#define PARO_STREAM_ONE 1
+#endif
 constexpr int kUnitBytes = kStreamRows * 64;  // 64 rows x 128 codes
 
-template <int NT>
+// ONE: every linear has a single token.  Its activations for a unit are then
+// one unswizzled 128-column box of 256 bytes (the 128-byte swizzle only
+// spreads 8 token rows over the banks): one copy instead of two, and a slot of
+// 4352 bytes instead of 6144.  (Three slots a warp were measured slower than
+// two on the Llama-3-8B-shaped layer: 45.7 against 39.2 us.)
+template <int NT, bool ONE = false>
 struct Geo {
+  static_assert(!ONE || NT == 1, "one token is one token tile");
   static constexpr int W = NT == 1 ? PARO_STREAM_W1 : PARO_STREAM_W2;  // warps per CTA
-  static constexpr int D = NT == 1 ? PARO_STREAM_D1 : PARO_STREAM_D2;  // ring slots per warp
-  static constexpr int XB = NT == 1 ? 1024 : 2048;  // bytes per activation box slot (>= 128 M, 1024-aligned)
+  static constexpr int D = ONE ? PARO_STREAM_D0 : (NT == 1 ? PARO_STREAM_D1 : PARO_STREAM_D2);  // ring slots
+  // bytes per activation half-box slot (>= 128 M, 1024-aligned under the swizzle)
+  static constexpr int XB = ONE ? 128 : (NT == 1 ? 1024 : 2048);
   static constexpr int SLOT = kUnitBytes + 2 * XB;
   static constexpr int PF = 4 * NT * 32 * 4;        // floats of one tile partial (fragment order)
   static constexpr int SMEM = W * D * SLOT + 1024;
@@ -318,12 +333,12 @@ __device__ bool wait_flag(const unsigned long long* f, unsigned long long v, lon
 // in the MMA's operand order (every 8-column block as x0, x4, x1/16, x5/16, x2,
 // x6, x3/16, x7/16), so a 16-byte chunk is a ready B fragment; the fused and
 // flag forms always take them so.
-template <bool F16, int NT, int FU, bool XPERM>
-__global__ void __launch_bounds__(Geo<NT>::W * 32, Geo<NT>::CPS)
+template <bool F16, int NT, int FU, bool XPERM, bool ONE>
+__global__ void __launch_bounds__(Geo<NT, ONE>::W * 32, Geo<NT, ONE>::CPS)
 w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ RotBatch rb, int* status,
                  int pdl_wait) {
   static_assert(!XPERM || F16, "the operand-order layout is fp16");
-  using Gm = Geo<NT>;
+  using Gm = Geo<NT, ONE>;
   constexpr int W = Gm::W, D = Gm::D, SLOT = Gm::SLOT, XB = Gm::XB, PF = Gm::PF;
   extern __shared__ unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t bars[W * D];
@@ -340,8 +355,20 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   if constexpr (FU > 0) {
     if ((int)blockIdx.x < T) {
       __shared__ __align__(8) uint64_t tbars[rotdec::kRotMaxRing];
-      const bool done = rotdec::rot_decode_cta<1, true, FU, W * 32>(
-          rb.p[blockIdx.x], 0, smem_raw + (sbase - smem_u32(smem_raw)), tbars, status, pdl_wait != 0);
+      // pairs per thread and round: enough that a stage of this linear is one
+      // round of loads and stores where the registers allow (wider ones take two)
+      const RotProblem& Pt = rb.p[blockIdx.x];
+      unsigned char* ts = smem_raw + (sbase - smem_u32(smem_raw));
+      const int rounds = (Pt.d / 2 + W * 32 - 33) / (W * 32 - 32);
+      bool done;
+      if (rounds <= 2)
+        done = rotdec::rot_decode_cta<1, true, 2, W * 32>(Pt, 0, ts, tbars, status, pdl_wait != 0);
+      else if (rounds <= 5)
+        done = rotdec::rot_decode_cta<1, true, 5, W * 32>(Pt, 0, ts, tbars, status, pdl_wait != 0);
+      else if (rounds <= 10)
+        done = rotdec::rot_decode_cta<1, true, 10, W * 32>(Pt, 0, ts, tbars, status, pdl_wait != 0);
+      else
+        done = rotdec::rot_decode_cta<1, true, 8, W * 32>(Pt, 0, ts, tbars, status, pdl_wait != 0);
       if (done) {
         // every thread's x~ stores, then the flag (the INT4 CTAs read x~ through
         // the asynchronous proxy after seeing it)
@@ -421,7 +448,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
     const uint32_t sx = ring + (uint32_t)(s * SLOT + kUnitBytes), bar = bar0 + 8u * s;
     mbar_arrive_expect_tx(bar, (uint32_t)(256 * meta[c.pi].M));
     tma_load_2d(sx, xm, c.grp * 128, 0, bar);
-    tma_load_2d(sx + XB, xm, c.grp * 128 + 64, 0, bar);
+    if constexpr (!ONE) tma_load_2d(sx + XB, xm, c.grp * 128 + 64, 0, bar);
   };
   // fused form (lane 0): linears whose x~ flag was seen, and slots whose
   // activations are still to be requested
@@ -637,7 +664,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
           mbar_arrive_expect_tx(bar, (uint32_t)(kUnitBytes + 256 * meta[ic.pi].M));
           tma_load_2d(sw, &Q.qmap, ic.grp * 16, ic.tile * kStreamRows, bar);
           tma_load_2d(sx, &Q.xmap, ic.grp * 128, 0, bar);
-          tma_load_2d(sx + XB, &Q.xmap, ic.grp * 128 + 64, 0, bar);
+          if constexpr (!ONE) tma_load_2d(sx + XB, &Q.xmap, ic.grp * 128 + 64, 0, bar);
         } else {
           // fused form, x~ not written yet: the codes now, the activations (and
           // the slot's arrival) when the unit comes up
@@ -882,6 +909,8 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
   *out = StreamBatch{};
   int maxM = 0, tiles = 0;
   long long units = 0;
+  bool all_one = PARO_STREAM_ONE != 0;
+  for (int i = 0; i < count; ++i) all_one = all_one && M[i] == 1;
   for (int i = 0; i < count; ++i) {
     if (!stream_supported(M[i], d_in[i], d_out[i], x[i], qw[i])) return cudaErrorInvalidValue;
     maxM = M[i] > maxM ? M[i] : maxM;
@@ -908,13 +937,15 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     }
-    {  // activations [M][d_in], one box = 64 columns x all M tokens, 128-byte swizzle
+    {  // activations [M][d_in]: one box = 64 columns x all M tokens, 128-byte swizzle;
+       // with one token in every linear, one unswizzled box of 128 columns
+      const bool one = all_one;
       const cuuint64_t dims[2] = {(cuuint64_t)d_in[i], (cuuint64_t)M[i]};
       const cuuint64_t strides[1] = {(cuuint64_t)d_in[i] * 2};
-      const cuuint32_t box[2] = {64, (cuuint32_t)M[i]};
+      const cuuint32_t box[2] = {one ? 128u : 64u, (cuuint32_t)M[i]};
       if (enc(&p.xmap, x_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
               const_cast<uint16_t*>(x[i]), dims, strides, box, unit_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              one ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     }
@@ -922,6 +953,7 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
   // the kernel's unit arithmetic is 32-bit: units times CTAs stays below 2^32
   if (units >= (1LL << 23)) return cudaErrorInvalidValue;
   out->count = count;
+  out->one = all_one ? 1 : 0;
   out->total_units = units;
   out->total_tiles = tiles;
   const int W = maxM <= 8 ? Geo<1>::W : Geo<2>::W;
@@ -953,7 +985,8 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
 
 cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* status, cudaStream_t stream,
                                 bool pdl_wait) {
-  const size_t smem = NT == 1 ? Geo<1>::SMEM : Geo<2>::SMEM;
+  const bool one = b.one != 0;
+  const size_t smem = NT == 1 ? (one ? Geo<1, true>::SMEM : Geo<1>::SMEM) : Geo<2>::SMEM;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(b.ctas);
   cfg.blockDim = dim3((NT == 1 ? Geo<1>::W : Geo<2>::W) * 32);
@@ -967,23 +1000,28 @@ cudaError_t launch_stream_batch(const StreamBatch& b, int NT, bool x_f16, int* s
   const int wait = pdl_wait ? 1 : 0;
   cudaError_t e;
   const RotBatch none{};
-#define PARO_STREAM_LAUNCH(f16, nt)                                                                       \
+#define PARO_STREAM_LAUNCH(f16, nt, one)                                                                  \
   {                                                                                                       \
-    auto k = w4_stream_kernel<f16, nt, 0, false>;                                                         \
+    auto k = w4_stream_kernel<f16, nt, 0, false, one>;                                                    \
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                  \
     if (e != cudaSuccess) return e;                                                                       \
     return cudaLaunchKernelEx(&cfg, k, b, none, status, wait);                                            \
   }
   if (x_f16) {
-    if (NT == 1) PARO_STREAM_LAUNCH(true, 1) else PARO_STREAM_LAUNCH(true, 2)
+    if (NT == 1) {
+      if (one) PARO_STREAM_LAUNCH(true, 1, true) else PARO_STREAM_LAUNCH(true, 1, false)
+    } else PARO_STREAM_LAUNCH(true, 2, false)
   } else {
-    if (NT == 1) PARO_STREAM_LAUNCH(false, 1) else PARO_STREAM_LAUNCH(false, 2)
+    if (NT == 1) {
+      if (one) PARO_STREAM_LAUNCH(false, 1, true) else PARO_STREAM_LAUNCH(false, 1, false)
+    } else PARO_STREAM_LAUNCH(false, 2, false)
   }
 #undef PARO_STREAM_LAUNCH
 }
 
 cudaError_t launch_stream_flagged(const StreamBatch& b, int NT, int* status, cudaStream_t stream) {
-  const size_t smem = NT == 1 ? Geo<1>::SMEM : Geo<2>::SMEM;
+  const bool one = b.one != 0 && NT == 1;
+  const size_t smem = NT == 1 ? (one ? Geo<1, true>::SMEM : Geo<1>::SMEM) : Geo<2>::SMEM;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(b.ctas);
   cfg.blockDim = dim3((NT == 1 ? Geo<1>::W : Geo<2>::W) * 32);
@@ -996,16 +1034,22 @@ cudaError_t launch_stream_flagged(const StreamBatch& b, int NT, int* status, cud
   cfg.numAttrs = 1;
   const RotBatch none{};
   cudaError_t e;
-  if (NT == 1) {
-    e = cudaFuncSetAttribute(w4_stream_kernel<true, 1, -1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (NT == 1 && one) {
+    e = cudaFuncSetAttribute(w4_stream_kernel<true, 1, -1, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, w4_stream_kernel<true, 1, -1, true>, b, none, status, 1);
+    return cudaLaunchKernelEx(&cfg, w4_stream_kernel<true, 1, -1, true, true>, b, none, status, 1);
   }
-  e = cudaFuncSetAttribute(w4_stream_kernel<true, 2, -1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (NT == 1) {
+    e = cudaFuncSetAttribute(w4_stream_kernel<true, 1, -1, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, w4_stream_kernel<true, 1, -1, true, false>, b, none, status, 1);
+  }
+  e = cudaFuncSetAttribute(w4_stream_kernel<true, 2, -1, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&cfg, w4_stream_kernel<true, 2, -1, true>, b, none, status, 1);
+  return cudaLaunchKernelEx(&cfg, w4_stream_kernel<true, 2, -1, true, false>, b, none, status, 1);
 }
 
 // ---- fused form -----------------------------------------------------------------------
@@ -1014,14 +1058,8 @@ namespace {
 // transform CTA's row and stage slots after the 1024-byte alignment, whichever
 // is larger, within 227 KB less the kernel's static shared memory
 constexpr size_t kFusedSmemBudget = 227 * 1024 - 2048;
-size_t fused_rot_smem(int d, int ring) { return 1024 + (size_t)d * 4 + (size_t)ring * 6 * d; }
-// pairs per thread and round of the transform CTAs (W1 - 1 rotating warps)
-int fused_u(const RotBatch& rb) {
-  int max_half = 0;
-  for (int i = 0; i < rb.count; ++i) max_half = rb.p[i].d / 2 > max_half ? rb.p[i].d / 2 : max_half;
-  const int comp = Geo<1>::W * 32 - 32;
-  const int rounds = (max_half + comp - 1) / comp;
-  return rounds <= 4 ? 4 : (rounds <= 8 ? 8 : (rounds <= 10 ? 10 : 8));
+size_t fused_rot_smem(int d, int ring, bool rcp = false) {
+  return 1024 + (size_t)d * 4 + (size_t)ring * 6 * d + (rcp ? (size_t)d * 4 : 0);
 }
 }  // namespace
 
@@ -1061,8 +1099,17 @@ cudaError_t plan_fused_rot(const RotProblem* probs, int count, RotBatch* out) {
   *out = RotBatch{};
   for (int i = 0; i < count; ++i) {
     RotProblem p = probs[i];
-    int ring = p.K < 1 ? 1 : (p.K > rotdec::kRotMaxRing ? rotdec::kRotMaxRing : p.K);
-    while (ring > 1 && fused_rot_smem(p.d, ring) > kFusedSmemBudget) --ring;
+    // as many stages of tables as fit, with 1/scale kept in shared memory when
+    // that still leaves at least two stage slots (fewer would make every stage
+    // wait for its table)
+    const int want = p.K < 1 ? 1 : (p.K > rotdec::kRotMaxRing ? rotdec::kRotMaxRing : p.K);
+    int ring = want;
+    while (ring > 1 && fused_rot_smem(p.d, ring, true) > kFusedSmemBudget) --ring;
+    p.rcp = fused_rot_smem(p.d, ring, true) <= kFusedSmemBudget && ring >= (want < 2 ? want : 2);
+    if (!p.rcp) {
+      ring = want;
+      while (ring > 1 && fused_rot_smem(p.d, ring) > kFusedSmemBudget) --ring;
+    }
     p.rows = 1;
     p.ring = ring;
     p.cta_begin = i;
@@ -1077,9 +1124,10 @@ cudaError_t plan_fused_rot(const RotProblem* probs, int count, RotBatch* out) {
 cudaError_t launch_fused_batch(const StreamBatch& b, const RotBatch& rb, int* status, cudaStream_t stream,
                                bool pdl_wait) {
   static_assert(sizeof(StreamBatch) + sizeof(RotBatch) + 16 <= 4096, "kernel parameters");
-  size_t smem = Geo<1>::SMEM;
+
+  size_t smem = b.one ? Geo<1, true>::SMEM : Geo<1>::SMEM;
   for (int i = 0; i < rb.count; ++i) {
-    const size_t s = fused_rot_smem(rb.p[i].d, rb.p[i].ring);
+    const size_t s = fused_rot_smem(rb.p[i].d, rb.p[i].ring, rb.p[i].rcp != 0);
     smem = s > smem ? s : smem;
   }
   cudaLaunchConfig_t cfg = {};
@@ -1093,19 +1141,10 @@ cudaError_t launch_fused_batch(const StreamBatch& b, const RotBatch& rb, int* st
   cfg.attrs = attr;
   cfg.numAttrs = pdl_wait ? 1 : 0;
   const int wait = pdl_wait ? 1 : 0;
-  const int u = fused_u(rb);
-  cudaError_t e;
-#define PARO_FUSED_LAUNCH(fu)                                                                             \
-  {                                                                                                       \
-    auto k = w4_stream_kernel<true, 1, fu, true>;                                                         \
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                  \
-    if (e != cudaSuccess) return e;                                                                       \
-    return cudaLaunchKernelEx(&cfg, k, b, rb, status, wait);                                              \
-  }
-  if (u == 4) PARO_FUSED_LAUNCH(4)
-  else if (u == 10) PARO_FUSED_LAUNCH(10)
-  else PARO_FUSED_LAUNCH(8)
-#undef PARO_FUSED_LAUNCH
+  auto k = b.one ? w4_stream_kernel<true, 1, 1, true, true> : w4_stream_kernel<true, 1, 1, true, false>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, k, b, rb, status, wait);
 }
 
 }  // namespace paro

@@ -51,6 +51,7 @@ struct StreamBatch {
   // cross-CTA flags and partials (flags, partials) are never used
   int tile_split;
   int total_tiles;
+  int one;                       // every linear has one token (its activation geometry, see the kernel)
   int count;
   int ctas;                      // CTAs of the INT4 linear (after the transform CTAs in the fused form)
 };
