@@ -197,8 +197,8 @@ PARO_API paro_status paro_plan_pair_order(const uint16_t* h_pairs, const float* 
 /*
  * Bytes of device workspace paro_rotate_w4_linear takes for M tokens of width
  * d_in: the fp16 transformed activations (2 M d_in rounded up to 256 bytes)
- * and, for M <= 16, the flags and partial tiles of the stream-K INT4 kernel
- * (about 8.2 KB per SM at 9-16 tokens, half that up to 8).
+ * and, for M <= 16, the partial tiles and flags of the stream-K INT4 kernel
+ * (about 16.4 KB per SM at 9-16 tokens, half that up to 8).
  */
 PARO_API size_t paro_workspace_bytes(int M, int d_in);
 
@@ -248,10 +248,11 @@ typedef struct {
 /*
  * Workspace bytes paro_rotate_w4_linear_batched uses for these linears: the
  * transformed activations of every linear (paro_workspace_bytes(M, d_in)
- * each, in order), then, when every M is at most 16, the publication flags
- * and partial sums of the stream-K INT4 linear (2 flags and 2 partial
- * 64-row tiles per CTA), the flags of the transform's CTAs (at most 128) that
- * the INT4 linear waits on, and the workspace's launch epoch (see below).
+ * each, in order), then, when every M is at most 16, the partial sums of
+ * the stream-K INT4 linear (2 partial 64-row tiles per CTA, every fp32 value
+ * in a 64-bit word beside a launch tag), the flags of the transform's CTAs
+ * (at most 128) that the INT4 linear waits on, and the workspace's launch
+ * epoch (see below).
  * The second part is optional: given only the first, the call runs the older
  * per-block kernel.
  */
@@ -287,12 +288,14 @@ PARO_API size_t paro_batched_workspace_bytes(const paro_linear* h_layers, int co
  * tokens the transform launch's CTAs each publish such a flag, and the INT4
  * launch after it requests a linear's activations once all of that linear's
  * transform CTAs have published, not when the whole transform launch is done.
- * Every flag a launch publishes (the transforms' "x~ is written" flags and
- * the stream-K kernel's partial-tile flags) holds 2E + 1 for the workspace's
- * launch epoch E, which every CTA reads once the previous kernel has
- * completed and which the launch's last CTA advances: a flag left by an
- * earlier call, or by an earlier replay of the same CUDA graph, is never taken
- * for this launch's, and calls captured in a graph may be replayed with new
+ * Every flag a launch publishes (the transforms' "x~ is written" flags)
+ * holds 2E + 1 for the workspace's launch epoch E, which every CTA reads once
+ * the previous kernel has completed and which the launch's last CTA advances,
+ * and every value of a partial tile carries the low 32 bits of 2E + 1: a flag
+ * or a value left by an earlier call, or by an earlier replay of the same
+ * CUDA graph, is not taken for this launch's (a partial value left exactly a
+ * multiple of 2^31 launches earlier on the same workspace, and not rewritten
+ * since, would be), and calls captured in a graph may be replayed with new
  * inputs.  Two calls that may run at the same time need two workspaces.
  */
 PARO_API paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count, int group_size,
@@ -300,14 +303,14 @@ PARO_API paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, 
                                                   paro_stream_t stream);
 
 /* Bytes of the scratch array built into the library for the call below. */
-#define PARO_NOALLOC_SCRATCH_BYTES (2u << 20)
+#define PARO_NOALLOC_SCRATCH_BYTES (4u << 20)
 
 /*
  * The same computation as paro_rotate_w4_linear for callers that cannot
  * allocate device memory (the paper has no counterpart: this is an interface
  * convenience of this library).  Instead of a caller-provided workspace, the
  * call uses a scratch array built into the library: every GPU that loads
- * libparo holds PARO_NOALLOC_SCRATCH_BYTES (2 MiB) for it until the process
+ * libparo holds PARO_NOALLOC_SCRATCH_BYTES (4 MiB) for it until the process
  * exits.  M * d_in may not exceed 262144 (PARO_ERR_UNSUPPORTED, nothing
  * enqueued).  The call allocates nothing and runs the same kernels as
  * paro_rotate_w4_linear given a workspace of PARO_NOALLOC_SCRATCH_BYTES, so

@@ -613,7 +613,7 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     rb.skip_flags = paro::hook_skip_ready_flags();
     if (e == cudaSuccess) e = plan_stream(true, rb.count, &sb, &nt);
     if (e == cudaSuccess) {
-      paro::set_fused_split(sb, 0.4);
+      paro::set_fused_split(sb, 0.6);
       e = paro::launch_fused_batch(sb, rb, status, s, true);
     }
     return from_cuda(e, "batched fused launch");

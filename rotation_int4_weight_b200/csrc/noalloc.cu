@@ -12,7 +12,7 @@
 // tokens, the stream-K INT4 kernel's publication flags and partial tiles.
 //
 // The array is a file-scope __device__ variable: every GPU that loads this
-// library holds PARO_NOALLOC_SCRATCH_BYTES (2 MiB) until the process exits.
+// library holds PARO_NOALLOC_SCRATCH_BYTES (4 MiB) until the process exits.
 // Host code cannot use the array's name as a device address (it is a
 // host-side stand-in), so the entry point looks the address up once per
 // device with cudaGetSymbolAddress, with that device current, and passes it
@@ -25,9 +25,10 @@ namespace {
 
 // M * d_in of one call may not exceed this many fp16 elements (e.g. M = 16
 // tokens of width 16384, or one token of width 49152); the rest of the array
-// holds the stream-K kernel's flags and partial tiles, which need about
-// 8.2 KB per SM (the call runs the older per-block kernels on a GPU with so
-// many SMs that they do not fit)
+// holds the stream-K kernel's partial tiles and flags, which need about
+// 16.4 KB per SM at 9-16 tokens (the call runs the stream-K kernel on whole
+// tiles per CTA, without partials, on a GPU with so many SMs that they do not
+// fit)
 constexpr size_t kNoAllocMaxElems = size_t(1) << 18;
 constexpr size_t kScratchBytes = PARO_NOALLOC_SCRATCH_BYTES;
 static_assert(kScratchBytes >= kNoAllocMaxElems * sizeof(__half), "scratch holds the transformed activations");
@@ -75,9 +76,11 @@ extern "C" paro_status paro_rotate_w4_linear_noalloc(const uint16_t* d_x, int K,
                                 cudaGetErrorString(e));
   }
   // Same validation and kernels as the workspace-taking call given a workspace
-  // of kScratchBytes.  Nothing here needs to start at zero: the transform
-  // overwrites every activation it hands to the linear, and a stream-K flag
-  // only counts when it holds the id of the launch that reads it.
+  // of kScratchBytes.  That workspace must be zero before its first use: the
+  // array is, as a __device__ variable without initializer is zero when the
+  // module loads, and every call leaves it in the state the next call expects
+  // (the transform overwrites every activation it hands to the linear; the
+  // stream-K flags hold a launch epoch that each launch advances).
   return paro_rotate_w4_linear(d_x, K, d_pairs, d_cos, d_sin, d_scale, d_qweight, d_scales, d_zeros, d_y, M,
                                d_in, d_out, group_size, scratch, kScratchBytes, stream);
 }

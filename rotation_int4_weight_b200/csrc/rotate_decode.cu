@@ -32,7 +32,7 @@ template <int R, bool F16OUT, int UP>
 __global__ void __launch_bounds__(kRotThreads)
 rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_trigger, int pdl_wait) {
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ __align__(8) uint64_t bars[rotdec::kRotMaxRing];
+  __shared__ __align__(8) uint64_t bars[rotdec::kRotBars];
   // with flags, the INT4 launch that follows may start only once this grid has
   // waited for the previous kernel (it takes the launch epoch at its start, which
   // the previous INT4 launch on the workspace advanced at its end): the CTAs
@@ -72,11 +72,17 @@ rot_decode_kernel(const __grid_constant__ RotBatch batch, int* status, int pdl_t
   }
 }
 
-size_t rot_smem(int d, int R, int ring, bool rcp = false) {
-  return (size_t)d * R * 4 + (size_t)ring * 6 * d + (rcp ? (size_t)d * 4 : 0);
+size_t rot_smem(int d, int R, int ring, bool region = false) {
+  return (size_t)d * R * 4 + (size_t)ring * 6 * d + (region ? (size_t)d * 4 : 0);
 }
 
 }  // namespace
+
+int scale_mode(const RotProblem& p, int ring, bool region_fits) {
+  if (!p.scale || (reinterpret_cast<uintptr_t>(p.scale) & 15) != 0) return 0;
+  if (region_fits) return 1;
+  return ring >= 2 && p.K >= 2 ? 2 : 0;
+}
 
 bool rot_decode_supported(int d, const void* pairs, const void* c, const void* s) {
   auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
@@ -100,11 +106,17 @@ cudaError_t plan_rot_batch(const RotProblem* probs, int count, RotBatch* out, in
     const int want = p.K < 1 ? 1 : (p.K < 3 ? p.K : 3);
     int rows = R;
     while (rows > 1 && rot_smem(p.d, rows, want) > kRotSmemBudget) rows >>= 1;
-    int ring = p.K < 1 ? 1 : p.K;
-    if (ring > 8) ring = 8;
-    while (ring > 1 && rot_smem(p.d, rows, ring) > kRotSmemBudget) --ring;
-    // 1/scale in shared memory when it fits beside the same ring
-    p.rcp = rot_smem(p.d, rows, ring, true) <= kRotSmemBudget;
+    // table slots: as many as fit beside a region for 1/scale while that
+    // leaves two (or all K), else as many as fit without it
+    const int all = p.K < 1 ? 1 : (p.K > 8 ? 8 : p.K);
+    int ring = all;
+    while (ring > 1 && rot_smem(p.d, rows, ring, true) > kRotSmemBudget) --ring;
+    const bool region = rot_smem(p.d, rows, ring, true) <= kRotSmemBudget && ring >= (all < 2 ? all : 2);
+    if (!region) {
+      ring = all;
+      while (ring > 1 && rot_smem(p.d, rows, ring) > kRotSmemBudget) --ring;
+    }
+    p.sscale = scale_mode(p, ring, region);
     p.rows = rows;
     p.ring = ring;
     p.cta_begin = ctas;
@@ -122,7 +134,7 @@ cudaError_t launch_rot_batch(const RotBatch& b, int R, bool f16_out, int* status
   size_t smem = 0;
   for (int i = 0; i < b.count; ++i) {
     const int rows = b.p[i].rows > 0 && b.p[i].rows < R ? b.p[i].rows : R;
-    const size_t s = rot_smem(b.p[i].d, rows, b.p[i].ring, b.p[i].rcp != 0);
+    const size_t s = rot_smem(b.p[i].d, rows, b.p[i].ring, b.p[i].sscale == 1);
     smem = s > smem ? s : smem;
   }
   const int trig = pdl_trigger ? 1 : 0, wait = pdl_wait ? 1 : 0;

@@ -19,8 +19,10 @@ struct RotProblem {
   // filled by plan_rot_batch
   int perm;               // fp16 out for the stream-K INT4 kernel: every 8-column block stored as
                           // (x0, x4, x1/16, x5/16, x2, x6, x3/16, x7/16), its MMA operand order
-  int rcp;                // 1/scale kept in shared memory after the table ring (computed before
-                          // the wait for the previous kernel), else computed in the final pass
+  int sscale;             // the channel scale in shared memory for the final pass, one bulk copy:
+                          // 1 a region after the table ring, requested with the first stages;
+                          // 2 the ring slot the last table refill leaves free, requested then;
+                          // 0 read from global memory by the final pass (also: no scale)
   int rows;               // token rows a CTA (<= the launch's R; 0 means R)
   int ring;               // stages of tables held in shared memory at once
   int cta_begin;          // first CTA of this problem
@@ -44,6 +46,9 @@ struct RotBatch {
 // (d % 8 == 0 and 16-byte aligned tables, since stages are copied in 16-byte pieces).
 bool rot_decode_supported(int d, const void* pairs, const void* cos_t, const void* sin_t);
 cudaError_t plan_rot_batch(const RotProblem* probs, int count, RotBatch* out, int* R_out);
+// RotProblem::sscale for a problem with `ring` table slots: 1 when a region
+// for the scale fits beside them, else 2 when a slot frees before the end.
+int scale_mode(const RotProblem& p, int ring, bool region_fits);
 // pdl_trigger: let the next kernel launch early; pdl_wait: launched as a
 // programmatic dependent, fetches its tables early and waits for the previous
 // kernel before it reads the rows or writes the output.

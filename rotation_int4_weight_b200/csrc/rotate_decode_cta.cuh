@@ -11,8 +11,11 @@
 // stages beyond the ring, and waits for each stage's table before the CTA
 // barrier that starts the stage, so the barrier also tells the other warps that
 // the table has landed; they rotate the pairs, U per thread and round, loads
-// before stores.  Waits are bounded: a stage that never lands is reported as
-// PARO_ERR_TIMEOUT and the CTA returns false without writing.
+// before stores.  The same thread brings the channel scale into shared memory
+// with one more bulk copy (into a region of its own, or into the slot the last
+// table refill leaves free), so the final pass, which divides by it, reads no
+// global memory.  Waits are bounded: a stage or scale that never lands is
+// reported as PARO_ERR_TIMEOUT and the CTA returns false without writing.
 #pragma once
 
 #include "paro_internal.cuh"
@@ -22,6 +25,7 @@ namespace paro {
 namespace rotdec {
 
 constexpr int kRotMaxRing = 8;
+constexpr int kRotBars = kRotMaxRing + 1;  // one mbarrier per ring slot, one for the channel scale
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
@@ -70,18 +74,29 @@ __device__ __forceinline__ float lds_f32(uint32_t a) {
 __device__ __forceinline__ void sts_f32(uint32_t a, float v) {
   asm volatile("st.shared.f32 [%0], %1;\n" ::"r"(a), "f"(v) : "memory");
 }
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, size_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"((uint32_t)bytes) : "memory");
+// An L2 policy that keeps the lines it fetches past lines of normal and
+// evict-first priority: the stage tables and scales are layer constants, read
+// once per call like the weights but a fraction of their size, so they stay in
+// L2 from one token to the next while the weights (fetched evict-first by the
+// INT4 kernels) stream through
+__device__ __forceinline__ uint64_t l2_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(pol));
+  return pol;
 }
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
-               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, size_t bytes, uint64_t pol) {
+  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;\n"
+               ::"l"(src), "r"((uint32_t)bytes), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar, uint64_t pol) {
+  asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;\n"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar), "l"(pol) : "memory");
 }
 
 
 // Transforms rows row0 .. row0 + RP - 1 of problem P with NTHR threads, RP =
 // P.rows (at most R; 0 means R); smem holds d RP 4 + ring 6 d (+ 4 d with
-// P.rcp) bytes (16-byte aligned), bars kRotMaxRing mbarriers.
+// P.sscale == 1) bytes (16-byte aligned), bars kRotBars mbarriers.
 // Returns true when the rows were written (uniform over the CTA).
 // trigger_after_wait: let the grid's dependents launch right after the wait
 // for the previous kernel (rather than earlier).
@@ -102,6 +117,7 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
   const size_t stage_bytes = (size_t)6 * d;  // pairs | cos | sin
   const uint32_t s_tab = static_cast<uint32_t>(__cvta_generic_to_shared(tab));
   const uint32_t s_bar = static_cast<uint32_t>(__cvta_generic_to_shared(bars));
+  const uint64_t pol = tid == kProd ? l2_evict_last() : 0;  // (used by the producer only)
 
   // one thread requests whole stages with bulk copies (three per stage); the
   // stage's mbarrier completes when all 6d bytes have landed
@@ -110,32 +126,51 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
       const int slot = k % ring;
       const uint32_t base = s_tab + (uint32_t)(slot * stage_bytes), bar = s_bar + 8u * slot;
       mbar_expect_tx(bar, (uint32_t)stage_bytes);
-      bulk_g2s(base, P.pairs + (size_t)k * half, 2u * d, bar);
-      bulk_g2s(base + 2u * d, P.cos_t + (size_t)k * half, 2u * d, bar);
-      bulk_g2s(base + 4u * d, P.sin_t + (size_t)k * half, 2u * d, bar);
+      bulk_g2s(base, P.pairs + (size_t)k * half, 2u * d, bar, pol);
+      bulk_g2s(base + 2u * d, P.cos_t + (size_t)k * half, 2u * d, bar, pol);
+      bulk_g2s(base + 4u * d, P.sin_t + (size_t)k * half, 2u * d, bar, pol);
     }
   };
+  // the channel scale in shared memory (fp32, read by the final pass):
+  // sscale 1, a region after the ring, requested with the first stages and
+  // turned into 1/s in place before the wait for the previous kernel; sscale 2,
+  // s in the ring slot that the last refill leaves free, requested once that
+  // slot is free (while the last stages run).  It lands on bars[kRotMaxRing].
+  const uint32_t s_sbar = s_bar + 8u * kRotMaxRing;
+  const int ks = K - ring + 1 > 1 ? K - ring + 1 : 1;  // sscale 2: the stage that requests it
+  const float* ssm = nullptr;
+  if (P.sscale == 1) ssm = reinterpret_cast<const float*>(tab + (size_t)ring * stage_bytes);
+  else if (P.sscale == 2) ssm = reinterpret_cast<const float*>(tab + (size_t)((ks - 1) % ring) * stage_bytes);
+  auto issue_scale = [&]() {
+    mbar_expect_tx(s_sbar, 4u * (uint32_t)d);
+    bulk_g2s(static_cast<uint32_t>(__cvta_generic_to_shared(ssm)), P.scale, 4u * (uint32_t)d, s_sbar, pol);
+  };
   if (tid == kProd) {
-    for (int k = 0; k < kRotMaxRing; ++k) mbar_init(s_bar + 8u * k, 1);
+    for (int k = 0; k < kRotBars; ++k) mbar_init(s_bar + 8u * k, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     for (int k = 0; k < ring; ++k) issue_stage(k);
+    if (P.sscale == 1) issue_scale();
     // then the stages beyond the ring go to L2, so that their copies into the
     // ring later wait for L2 rather than HBM
     if (K > ring) {
       const size_t off = (size_t)ring * half, bytes = (size_t)(K - ring) * 2 * d;
-      bulk_prefetch_l2(P.pairs + off, bytes);
-      bulk_prefetch_l2(P.cos_t + off, bytes);
-      bulk_prefetch_l2(P.sin_t + off, bytes);
+      bulk_prefetch_l2(P.pairs + off, bytes, pol);
+      bulk_prefetch_l2(P.cos_t + off, bytes, pol);
+      bulk_prefetch_l2(P.sin_t + off, bytes, pol);
     }
-    if (P.scale && (reinterpret_cast<uintptr_t>(P.scale) & 15) == 0) bulk_prefetch_l2(P.scale, (size_t)4 * d);
+    if (P.sscale != 1 && P.scale && (reinterpret_cast<uintptr_t>(P.scale) & 15) == 0)
+      bulk_prefetch_l2(P.scale, (size_t)4 * d, pol);
   }
-  // 1/scale into shared memory while the previous kernel may still run (the
-  // scale is a layer constant, like the tables); the barrier after the rows
-  // are staged orders these stores before the final pass reads them
-  float* rcp = P.rcp ? reinterpret_cast<float*>(tab + (size_t)ring * stage_bytes) : nullptr;
-  if (rcp) {
-#pragma unroll 4
-    for (int c = tid; c < d; c += NTHR) rcp[c] = P.scale ? 1.0f / __ldg(P.scale + c) : 1.0f;
+  if (P.sscale == 1) __syncthreads();  // the mbarriers are initialised before anyone waits
+  // sscale 1: 1/s in place, each thread its channels, once the copy has landed
+  // (the scale is a layer constant, so this may overlap the previous kernel;
+  // the barrier after the rows are staged orders it before the final pass)
+  bool ok = true;
+  if (P.sscale == 1) {
+    ok = mbar_wait_bounded(s_sbar, 0u);
+    float* r = const_cast<float*>(ssm);
+    if (ok)
+      for (int c = tid; c < d; c += NTHR) r[c] = 1.0f / r[c];
   }
   // launched as a programmatic dependent: the tables above may be fetched while
   // the previous kernel finishes; the rows (which it may have written) and the
@@ -173,10 +208,10 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
   // the table has landed; it refills a slot as soon as the barrier after its
   // stage has passed.  With one slot the next stage can only be requested once
   // the current one is done, which costs a second barrier per stage.
-  bool ok = true;
-  if (tid == kProd && K > 0) ok = mbar_wait_bounded(s_bar, 0u);
+  if (tid == kProd && K > 0 && ok) ok = mbar_wait_bounded(s_bar, 0u);
   int failed = __syncthreads_or(!ok);  // also: rows staged
   int issued = ring < K ? ring : K;    // stages requested so far (producer)
+  bool scale_issued = P.sscale == 1;   // (producer)
 
   // K stages.  The pairs of a stage are disjoint, so the loads of a batch of
   // pairs may all be issued before any of its stores.  Addresses are 32-bit
@@ -231,13 +266,21 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
               }
           }
       }
-    } else if (tid == kProd && ring > 1) {
-      // stage k - 1's slot is free since the barrier that started this stage
-      if (k >= 1 && k - 1 + ring < K) {
-        issue_stage(k - 1 + ring);
-        ++issued;
+    } else if (tid == kProd) {
+      if (ring > 1) {
+        // stage k - 1's slot is free since the barrier that started this stage:
+        // it takes the next table, or, once none is left, the scale (sscale 2)
+        if (k >= 1 && k - 1 + ring < K) {
+          issue_stage(k - 1 + ring);
+          ++issued;
+        } else if (P.sscale == 2 && k == ks) {
+          issue_scale();
+          scale_issued = true;
+        }
+        if (k + 1 < K) ok = mbar_wait_bounded(s_bar + 8u * ((k + 1) % ring), (uint32_t)(((k + 1) / ring) & 1));
       }
-      if (k + 1 < K) ok = mbar_wait_bounded(s_bar + 8u * ((k + 1) % ring), (uint32_t)(((k + 1) / ring) & 1));
+      // the scale (sscale 2) before the barrier that ends the last stage
+      if (k == K - 1 && P.sscale == 2 && ok) ok = mbar_wait_bounded(s_sbar, 0u);
     }
     failed = __syncthreads_or(!ok);
     slot_off += (uint32_t)stage_bytes;
@@ -259,6 +302,7 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
       report_status(status, kStatusTimeout);
       for (int q = issued > ring ? issued - ring : 0; q < issued; ++q)
         mbar_wait_bounded(s_bar + 8u * (q % ring), (uint32_t)((q / ring) & 1));
+      if (scale_issued) mbar_wait_bounded(s_sbar, 0u);
     }
     __syncthreads();
     return false;
@@ -276,14 +320,16 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
 #pragma unroll 1
       for (int b0 = tid; b0 < (d >> 3); b0 += NTHR) {
         float f[8];
-        if (rcp) {
-          const float4 r0 = *reinterpret_cast<const float4*>(rcp + 8 * b0);
-          const float4 r1 = *reinterpret_cast<const float4*>(rcp + 8 * b0 + 4);
+        if (ssm) {
+          const float4 r0 = *reinterpret_cast<const float4*>(ssm + 8 * b0);
+          const float4 r1 = *reinterpret_cast<const float4*>(ssm + 8 * b0 + 4);
           f[0] = r0.x; f[1] = r0.y; f[2] = r0.z; f[3] = r0.w;
           f[4] = r1.x; f[5] = r1.y; f[6] = r1.z; f[7] = r1.w;
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) f[e] = P.scale ? __ldg(P.scale + 8 * b0 + e) : 1.0f;
+        }
+        if (P.sscale != 1) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) f[e] = 1.0f / f[e];
         }
@@ -318,7 +364,7 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
       const int cp = cp0 + q * NTHR;
       sc[q] = make_float2(1.0f, 1.0f);
       if (cp < half) {
-        if (rcp) sc[q] = *reinterpret_cast<const float2*>(rcp + 2 * cp);
+        if (ssm) sc[q] = *reinterpret_cast<const float2*>(ssm + 2 * cp);
         else if (P.scale) sc[q] = make_float2(__ldg(P.scale + 2 * cp), __ldg(P.scale + 2 * cp + 1));
       }
     }
@@ -327,7 +373,7 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
       const int cp = cp0 + q * NTHR;
       if (cp >= half) continue;
       const int c = 2 * cp;
-      const float f0 = rcp ? sc[q].x : 1.0f / sc[q].x, f1 = rcp ? sc[q].y : 1.0f / sc[q].y;
+      const float f0 = P.sscale == 1 ? sc[q].x : 1.0f / sc[q].x, f1 = P.sscale == 1 ? sc[q].y : 1.0f / sc[q].y;
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         if (r < nrows) {

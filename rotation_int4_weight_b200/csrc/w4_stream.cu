@@ -32,14 +32,20 @@
 // Partial sums.  A tile wholly inside one warp's units is written by that warp.
 // A tile split between warps of a CTA is summed in shared memory at the end, in
 // warp order.  A tile split between CTAs goes through the workspace: every CTA
-// holding part of it but the last writes its partial tile and then a flag
-// holding this launch's tag, 2E + 1 for the workspace's launch epoch E (a flag
-// left by another launch or by an earlier replay of the same CUDA graph, or
-// never written, never matches: the last CTA of every launch advances E, so
-// the workspace needs clearing only once, before its first use);
-// the tile's last CTA waits (bounded) for the flags of the earlier CTAs, which
-// were launched no later than it, and sums the partials in CTA order.  Every
-// sum has a fixed order, so the result does not depend on timing.
+// holding part of it but the last writes its partial tile, each fp32 value in
+// a 64-bit word beside this launch's tag (the low 32 bits of 2E + 1 for the
+// workspace's launch epoch E: a word left by another launch or by an earlier
+// replay of the same CUDA graph, or never written, holds another tag, since
+// the last CTA of every launch advances E; the workspace needs clearing only
+// once, before its first use); the tile's last CTA reads the earlier CTAs'
+// partials, which were launched no later than it, until every word carries
+// the tag (bounded), and sums them in CTA order.  A word is written and read
+// as a whole, so its tag vouches for its value: no flag after the values and
+// no fence between them, which would cost two more round trips to memory at
+// the end of a launch.  (A word left exactly a multiple of 2^31 launches
+// earlier would pass for current; a workspace never sees that many launches
+// between two uses of a slot in practice.)  Every sum has a fixed order, so
+// the result does not depend on timing.
 #include "paro_internal.cuh"
 #include "w4_stream.cuh"
 #include "rotate_decode_cta.cuh"
@@ -135,6 +141,21 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n"
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
       : "memory");
+}
+// the same with an L2 eviction policy (the packed weights: read once per call,
+// fetched evict-first so that they do not push the layer tables out of L2)
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar,
+                                            uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+      "%3}], [%4], %5;\n"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+  return pol;
 }
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -320,6 +341,54 @@ __device__ bool wait_flag(const unsigned long long* f, unsigned long long v, lon
   }
 }
 
+// Two tagged values (a 16-byte store of two 64-bit words, each written as a whole).
+__device__ __forceinline__ void st_tagged(unsigned long long* p, float a, float b, uint32_t tag) {
+  const unsigned long long wa = ((unsigned long long)tag << 32) | __float_as_uint(a);
+  const unsigned long long wb = ((unsigned long long)tag << 32) | __float_as_uint(b);
+  asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};\n" ::"l"(p), "l"(wa), "l"(wb) : "memory");
+}
+// Adds another CTA's tagged partial tile (this lane's 4 NT words of 4 values) to
+// tot once every word of every lane carries `tag`; reads again (bounded by
+// `limit` SM cycles, lane 0's clock deciding for the warp) until then.
+template <int NT>
+__device__ bool add_tagged(const unsigned long long* src, int lane, uint32_t tag, long long limit,
+                           float (&tot)[4][NT][4]) {
+  const long long t0 = clock64();
+#pragma unroll 1
+  while (true) {
+    unsigned long long w[4][NT][4];
+    bool mine = true;
+#pragma unroll
+    for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+      for (int m = 0; m < NT; ++m) {
+        const unsigned long long* q = src + (size_t)(((rt * NT + m) * 32 + lane) * 4);
+        asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];\n"
+                     : "=l"(w[rt][m][0]), "=l"(w[rt][m][1]) : "l"(q) : "memory");
+        asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];\n"
+                     : "=l"(w[rt][m][2]), "=l"(w[rt][m][3]) : "l"(q + 2) : "memory");
+      }
+#pragma unroll
+    for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+      for (int m = 0; m < NT; ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mine = mine && (uint32_t)(w[rt][m][e] >> 32) == tag;
+    if (__all_sync(0xffffffffu, mine)) {
+#pragma unroll
+      for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+        for (int m = 0; m < NT; ++m)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) tot[rt][m][e] += __uint_as_float((uint32_t)w[rt][m][e]);
+      return true;
+    }
+    int late = clock64() - t0 > limit ? 1 : 0;
+    if (__shfl_sync(0xffffffffu, late, 0)) return false;
+    __nanosleep(64);
+  }
+}
+
 // FU > 0: the fused form (one token per linear): CTAs 0 .. rb.count - 1 run the
 // activation transform of one linear each, FU pairs per thread and round, and
 // publish a flag holding this launch's tag once its x~ is written; the INT4
@@ -354,7 +423,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   const int T = FU > 0 ? rb.count : 0;  // transform CTAs
   if constexpr (FU > 0) {
     if ((int)blockIdx.x < T) {
-      __shared__ __align__(8) uint64_t tbars[rotdec::kRotMaxRing];
+      __shared__ __align__(8) uint64_t tbars[rotdec::kRotBars];
       // pairs per thread and round: enough that a stage of this linear is one
       // round of loads and stores where the registers allow (wider ones take two)
       const RotProblem& Pt = rb.p[blockIdx.x];
@@ -431,7 +500,8 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
 #pragma unroll 1
     for (int s = 0; s < D && s < n; ++s) {
       mbar_expect_tx(bar0 + 8u * s, (uint32_t)kUnitBytes);
-      tma_load_2d(ring + (uint32_t)(s * SLOT), &b.p[c.pi].qmap, c.grp * 16, c.tile * kStreamRows, bar0 + 8u * s);
+      tma_load_2d(ring + (uint32_t)(s * SLOT), &b.p[c.pi].qmap, c.grp * 16, c.tile * kStreamRows, bar0 + 8u * s,
+                  l2_evict_first());
       cur_next(meta, c);
     }
   }
@@ -662,14 +732,14 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
         const uint32_t bar = bar0 + 8u * slot;
         if (x_ready(ic.pi, false)) {
           mbar_arrive_expect_tx(bar, (uint32_t)(kUnitBytes + 256 * meta[ic.pi].M));
-          tma_load_2d(sw, &Q.qmap, ic.grp * 16, ic.tile * kStreamRows, bar);
+          tma_load_2d(sw, &Q.qmap, ic.grp * 16, ic.tile * kStreamRows, bar, l2_evict_first());
           tma_load_2d(sx, &Q.xmap, ic.grp * 128, 0, bar);
           if constexpr (!ONE) tma_load_2d(sx + XB, &Q.xmap, ic.grp * 128 + 64, 0, bar);
         } else {
           // fused form, x~ not written yet: the codes now, the activations (and
           // the slot's arrival) when the unit comes up
           mbar_expect_tx(bar, (uint32_t)kUnitBytes);
-          tma_load_2d(sw, &Q.qmap, ic.grp * 16, ic.tile * kStreamRows, bar);
+          tma_load_2d(sw, &Q.qmap, ic.grp * 16, ic.tile * kStreamRows, bar, l2_evict_first());
           xpend |= 1u << slot;
         }
       }
@@ -754,7 +824,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   // CTA waits for the flags of the earlier CTAs, which started no later than
   // it did, and sums the partials in CTA order.  Publishing comes first (the
   // warp's last tile), so no warp waits while holding back a partial. ------------
-  const unsigned long long tag = ltag;
+  const uint32_t tag32 = (uint32_t)ltag;  // the tag's low half, carried by every partial value
 #pragma unroll 1
   for (int pass = 0; pass < 2; ++pass) {
     const int which = 1 - pass;
@@ -792,17 +862,18 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
       continue;
     }
     if (Ue > c1) {
-      // the tile goes on in a later CTA: publish this CTA's partial, then its flag
+      // the tile goes on in a later CTA: publish this CTA's partial, every
+      // value tagged
       const int eC = (Ub <= c0) ? 0 : 1;
-      float4* mine = reinterpret_cast<float4*>(b.partials + ((size_t)cta * 2 + eC) * PF);
+      unsigned long long* mine = b.partials + ((size_t)cta * 2 + eC) * PF;
 #pragma unroll
       for (int rt = 0; rt < 4; ++rt)
 #pragma unroll
-        for (int m = 0; m < NT; ++m)
-          __stcg(mine + (rt * NT + m) * 32 + lane, make_float4(sum[rt][m][0], sum[rt][m][1], sum[rt][m][2], sum[rt][m][3]));
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) st_flag(b.flags + cta * 2 + eC, tag);
+        for (int m = 0; m < NT; ++m) {
+          unsigned long long* q = mine + (size_t)(((rt * NT + m) * 32 + lane) * 4);
+          st_tagged(q, sum[rt][m][0], sum[rt][m][1], tag32);
+          st_tagged(q + 2, sum[rt][m][2], sum[rt][m][3], tag32);
+        }
       continue;
     }
     // the tile began in an earlier CTA and ends here: add the earlier partials
@@ -821,23 +892,11 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
       const long long s0 = cta_start(cx);
       if (cta_start(cx + 1) <= s0) continue;  // a CTA without units
       const int e = (Ub <= s0) ? 0 : 1;
-      int seen = 1;
-      if (lane == 0) seen = wait_flag(b.flags + cx * 2 + e, tag, b.flag_wait) ? 1 : 0;
-      seen = __shfl_sync(0xffffffffu, seen, 0);
-      if (!seen) {
+      if (!add_tagged<NT>(b.partials + ((size_t)cx * 2 + e) * PF, lane, tag32, b.flag_wait, tot)) {
         if (lane == 0) report_status(status, kStatusTimeout);
         got = false;
         break;
       }
-      __threadfence();
-      const float4* src = reinterpret_cast<const float4*>(b.partials + ((size_t)cx * 2 + e) * PF);
-#pragma unroll
-      for (int rt = 0; rt < 4; ++rt)
-#pragma unroll
-        for (int m = 0; m < NT; ++m) {
-          const float4 v = __ldcg(src + (rt * NT + m) * 32 + lane);
-          tot[rt][m][0] += v.x; tot[rt][m][1] += v.y; tot[rt][m][2] += v.z; tot[rt][m][3] += v.w;
-        }
     }
     if (!got) continue;  // the tile stays unwritten: the status says the result is void
 #pragma unroll
@@ -892,11 +951,12 @@ bool stream_supported(int M, int d_in, int d_out, const void* x, const void* qwe
 // partial tiles each in the workspace)
 static int max_ctas(int NT) { return device_sm_count() * (NT == 1 ? Geo<1>::CPS : Geo<2>::CPS); }
 
+// two partial tiles per CTA (a 64-bit tagged word per value), the transforms'
+// flags, the launch epoch and the finished-CTA count
 size_t stream_workspace_bytes(int max_m) {
   const int NT = max_m <= 8 ? 1 : 2;
   const size_t C = (size_t)max_ctas(NT);
-  return round256(C * 2 * 8) + round256(C * 2 * (4 * NT * 32 * 4) * 4) + round256((size_t)kXFlagWords * 8) +
-         256;  // the launch epoch and the finished-CTA count
+  return round256(C * 2 * (4 * NT * 32 * 4) * 8) + round256((size_t)kXFlagWords * 8) + 256;
 }
 
 cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* qw, const __half* const* sc,
@@ -974,11 +1034,10 @@ cudaError_t plan_stream_batch(const uint16_t* const* x, const uint32_t* const* q
     out->ctas_a = out->ctas;
     return cudaSuccess;
   }
-  out->flags = static_cast<unsigned long long*>(ws);
   const size_t C = (size_t)max_ctas(maxM <= 8 ? 1 : 2);
-  out->partials = reinterpret_cast<float*>(static_cast<char*>(ws) + round256(C * 2 * 8));
-  out->xflags = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + round256(C * 2 * 8) +
-                                                      round256(C * 2 * (4 * (maxM <= 8 ? 1 : 2) * 32 * 4) * 4));
+  out->partials = static_cast<unsigned long long*>(ws);
+  out->xflags = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) +
+                                                      round256(C * 2 * (4 * (maxM <= 8 ? 1 : 2) * 32 * 4) * 8));
   out->ctl = out->xflags + round256((size_t)kXFlagWords * 8) / 8;
   return cudaSuccess;
 }
@@ -1058,8 +1117,8 @@ namespace {
 // transform CTA's row and stage slots after the 1024-byte alignment, whichever
 // is larger, within 227 KB less the kernel's static shared memory
 constexpr size_t kFusedSmemBudget = 227 * 1024 - 2048;
-size_t fused_rot_smem(int d, int ring, bool rcp = false) {
-  return 1024 + (size_t)d * 4 + (size_t)ring * 6 * d + (rcp ? (size_t)d * 4 : 0);
+size_t fused_rot_smem(int d, int ring, bool region = false) {
+  return 1024 + (size_t)d * 4 + (size_t)ring * 6 * d + (region ? (size_t)d * 4 : 0);
 }
 }  // namespace
 
@@ -1074,7 +1133,8 @@ void set_fused_split(StreamBatch& b, double late) {
   // units a CTA of the last linear gets, relative to the others: the later its
   // x~ comes (the wider it is than the rest), the fewer (fitted to the arrival
   // times of the transforms on B200 for Qwen2.5-1.5B and Llama-3-8B layers)
-  const double rho = 1.0 - late * (double)(wide - other) / wide;
+  double rho = 1.0 - late * (double)(wide - other) / wide;
+  rho = rho < 0.25 ? 0.25 : rho;  // (a share near zero would leave those CTAs nearly idle)
   const long long UA = b.p[b.count - 1].unit_begin, UB = b.total_units - UA;
   long long CA = (long long)((double)b.ctas / (1.0 + (double)UB / (rho * (double)UA)) + 0.5);
   CA = CA < 1 ? 1 : (CA > b.ctas - 1 ? b.ctas - 1 : CA);
@@ -1099,17 +1159,19 @@ cudaError_t plan_fused_rot(const RotProblem* probs, int count, RotBatch* out) {
   *out = RotBatch{};
   for (int i = 0; i < count; ++i) {
     RotProblem p = probs[i];
-    // as many stages of tables as fit, with 1/scale kept in shared memory when
-    // that still leaves at least two stage slots (fewer would make every stage
-    // wait for its table)
+    // as many stages of tables as fit beside a region for 1/scale, as long as
+    // that leaves at least two slots (a stage's table then lands while the
+    // previous stage is rotated); else as many as fit without it, the scale
+    // then going into the slot that the last refill leaves free
     const int want = p.K < 1 ? 1 : (p.K > rotdec::kRotMaxRing ? rotdec::kRotMaxRing : p.K);
     int ring = want;
     while (ring > 1 && fused_rot_smem(p.d, ring, true) > kFusedSmemBudget) --ring;
-    p.rcp = fused_rot_smem(p.d, ring, true) <= kFusedSmemBudget && ring >= (want < 2 ? want : 2);
-    if (!p.rcp) {
+    const bool region = fused_rot_smem(p.d, ring, true) <= kFusedSmemBudget && ring >= (want < 2 ? want : 2);
+    if (!region) {
       ring = want;
       while (ring > 1 && fused_rot_smem(p.d, ring) > kFusedSmemBudget) --ring;
     }
+    p.sscale = scale_mode(p, ring, region);
     p.rows = 1;
     p.ring = ring;
     p.cta_begin = i;
@@ -1127,7 +1189,7 @@ cudaError_t launch_fused_batch(const StreamBatch& b, const RotBatch& rb, int* st
 
   size_t smem = b.one ? Geo<1, true>::SMEM : Geo<1>::SMEM;
   for (int i = 0; i < rb.count; ++i) {
-    const size_t s = fused_rot_smem(rb.p[i].d, rb.p[i].ring, rb.p[i].rcp != 0);
+    const size_t s = fused_rot_smem(rb.p[i].d, rb.p[i].ring, rb.p[i].sscale == 1);
     smem = s > smem ? s : smem;
   }
   cudaLaunchConfig_t cfg = {};

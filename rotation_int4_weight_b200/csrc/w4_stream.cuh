@@ -30,8 +30,9 @@ struct StreamProblem {
 struct StreamBatch {
   StreamProblem p[kMaxBatch];
   long long total_units;
-  unsigned long long* flags;     // two per CTA: its partials' publication flags (workspace)
-  float* partials;               // two tile partials per CTA (workspace)
+  // two tile partials per CTA (workspace): every 64-bit word one fp32 value in
+  // its low half and the low 32 bits of the publishing launch's tag in its high half
+  unsigned long long* partials;
   unsigned long long* xflags;    // fused form: one per linear, set when its x~ is written (workspace);
                                  // flag form: one per CTA of the preceding transform launch
   // the workspace's launch epoch E (ctl[0]) and a wrapping count of the CTAs

@@ -469,6 +469,32 @@ def test_fused_decode_matches_oracle_and_repeats_bit_exactly(spec):
         assert torch.equal(f.view(torch.int16), d["y"].view(torch.int16))
 
 
+@pytest.mark.parametrize("shapes", [
+    # Llama-3-8B-shaped layer (the widest linear's units on CTAs of their own)
+    [(4096, 4096), (4096, 1024), (4096, 1024), (4096, 4096), (4096, 14336), (4096, 14336), (14336, 4096)],
+    # ragged output tails; the widest linear's tiles split between CTAs
+    [(1024, 1040), (2048, 272), (512, 3088), (6144, 4112)],
+])
+def test_fused_layer_matches_oracle_and_repeats_bit_exactly(shapes):
+    probs, devs = _batch_case([(d_in, d_out, 1) for d_in, d_out in shapes], 64)
+    layers = [paro.paro_linear(d["x"], *d["tables"], d["qw"], d["sc"], d["z"], d["y"]) for d in devs]
+    ws = paro.paro_rotate_w4_linear_batched(layers)
+    torch.cuda.synchronize()
+    assert paro.paro_get_device_status() == 0
+    first = [d["y"].clone() for d in devs]
+    for p, d in zip(probs, devs):
+        ref = oracle_all_columns(oracle.rotate(p.x, p.pairs, p.cos_t, p.sin_t, p.scale),
+                                 *to_np_pack(d["qw"], d["sc"], d["z"]))
+        assert_linear_close(host(d["y"]), ref)
+    for d in devs:
+        d["y"].fill_(float("nan"))
+    paro.paro_rotate_w4_linear_batched(layers, workspace=ws)
+    torch.cuda.synchronize()
+    assert paro.paro_get_device_status() == 0
+    for f, d in zip(first, devs):
+        assert torch.equal(f.view(torch.int16), d["y"].view(torch.int16))
+
+
 # ---------------------------------------------------------------- grouped tensor-core launch (batched, M >= 128)
 @pytest.mark.parametrize("shapes_m", [
     # mixed K, ragged token counts and ragged output tails in one launch

@@ -27,7 +27,7 @@ pytestmark = pytest.mark.gpu
 paro = pytest.importorskip("rotation_int4_weight_b200")
 DEV = "cuda"
 MAX_ELEMS = 1 << 18  # M * d_in limit of the built-in scratch array
-SCRATCH_BYTES = 2 << 20  # the scratch array's size, PARO_NOALLOC_SCRATCH_BYTES in include/paro.h
+SCRATCH_BYTES = 4 << 20  # the scratch array's size, PARO_NOALLOC_SCRATCH_BYTES in include/paro.h
 
 
 def _setup(seed, M, d_in, d_out):
