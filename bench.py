@@ -51,16 +51,19 @@ from synth import LAYER_SHAPES, device_weights, linear_problem  # noqa: E402
 METRIC = "rot+W4 linear: decode HBM GB/s (% peak), prefill TFLOP/s, rotation overhead %"
 
 # DRAM bytes (read + write) per launch of the kernel the roofline times, from
-# one ncu capture of `bench.py --profile --variants batched_plain --config N`
-# (metrics dram__bytes_read.sum, dram__bytes_write.sum; the first launch after
-# four skipped), with the sha256 prefix
-# of the kernel's sources at capture time: once the sources change, the figure
-# no longer describes the kernel and the bench reports null.
+# one ncu capture (metrics dram__bytes_read.sum, dram__bytes_write.sum) of
+#   config 1: `bench.py --profile --variants batched --config 1 --steps 28 --warmup 3 --no-cpu`
+#             (the fused one-launch step; the 21st launch, --set full),
+#   config 3: `... --variants batched_plain --config 3 --steps 4` (the tensor-core launch),
+#   config 4: `... --variants batched_plain --config 4 --steps 8` (the INT4 launch alone;
+#             the first launch after four skipped),
+# with the sha256 prefix of the kernel's sources at capture time: once the
+# sources change, the figure no longer describes the kernel and the bench
+# reports null.  (Config 2's fused step was not captured.)
 TRAFFIC = {
-    1: {"bytes": 24964608, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "2cbfd0012327d0d7"},
-    2: {"bytes": 131985408 + 3412992, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "2cbfd0012327d0d7"},
+    1: {"bytes": 25986560 + 256, "src": ("w4_stream.cu", "w4_stream.cuh", "rotate_decode_cta.cuh"), "sha": "0733fd003a3a3e71"},
     3: {"bytes": 346587136 + 137527040, "src": ("w4_tc.cu", "w4_tc.cuh"), "sha": "a093d18620409e5a"},
-    4: {"bytes": 25542400, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "2cbfd0012327d0d7"},
+    4: {"bytes": 25540608, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "69c1f87283208e9b"},
 }
 
 
