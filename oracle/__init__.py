@@ -19,3 +19,4 @@ from .paro import (  # noqa: F401
     check_stage_disjoint,
 )
 from .backward import rotate_backward  # noqa: F401,E402
+from .w4a4 import dequantize_activations, quantize_activations, rotate_w4a4_linear, w4a4_linear  # noqa: F401,E402
