@@ -193,6 +193,18 @@ class Linear:
             self.bws = torch.empty(max(need, 16), dtype=torch.uint8, device=self.x.device)
         paro.paro_rotate_backward(self.x, self.grad, self.pairs, self.cos, self.sin, self.scale, workspace=self.bws)
 
+    def w4a4(self, paro):
+        # the weight-activation variant on the same packed weights: transform,
+        # per-token INT4 codes of x~, the INT4 x INT4 linear
+        if getattr(self, "ws4", None) is None:
+            import torch
+            need = paro.lib.paro_w4a4_workspace_bytes(self.M, self.d_in, self.d_out, 1)
+            self.ws4 = torch.empty(max(need, 256), dtype=torch.uint8, device=self.x.device)
+            self.w4a4_launches = 3 + (1 if paro.lib.paro_w4a4_workspace_bytes(self.M, self.d_in, self.d_out, 0)
+                                      else 0)
+        paro.paro_rotate_w4a4_linear(self.x, self.pairs, self.cos, self.sin, self.scale, self.qw, self.sc, self.z,
+                                     out=self.y, workspace=self.ws4)
+
     def fused_e2e(self, paro):
         self.x.copy_(self.x_host, non_blocking=True)
         self.fused(paro)
@@ -260,6 +272,10 @@ class Unit:
         if variant == "fused":
             # the single-linear call at one token is the same one-launch form
             return sum(1 if l.M == 1 else 2 for l in self.lins)
+        if variant == "w4a4":
+            # transform, codes, linear, and an ordered reduction when the linear
+            # splits a tile's groups over several CTAs
+            return sum(getattr(l, "w4a4_launches", 4) for l in self.lins)
         return LAUNCHES[variant] * len(self.lins)
 
 
@@ -696,7 +712,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-sub", action="store_true", help="skip the prefill, stack and Llama decode sub-records")
-    ap.add_argument("--variants", default="batched,batched_plain,fused,plain,unfused,rotate,rotate_backward,dense")
+    ap.add_argument("--variants",
+                    default="batched,batched_plain,fused,plain,unfused,rotate,rotate_backward,dense,w4a4")
     ap.add_argument("--no-plan", action="store_true",
                     help="use the pair tables as drawn instead of the conflict-free order of paro_plan_pair_order")
     ap.add_argument("--profile", action="store_true",
@@ -834,6 +851,11 @@ def main():
         "rotation_overhead_unfused_pct": overhead(t, "unfused", "plain"),
         "rotation_overhead_per_linear_fused_pct": overhead(t, "fused", "plain"),
         "dense_rotation_overhead_pct": overhead(t, "dense", "plain"),
+        "w4a4": ({"ms_per_step": round(t["w4a4"].ms, 6),
+                  "vs_w4a16_fused_pct": overhead(t, "w4a4", "fused"),
+                  "what": "the weight-activation variant per linear (paro_rotate_w4a4_linear: transform, per-token "
+                          "INT4 codes, INT4 x INT4 linear on the same packed weights); vs_w4a16_fused_pct: its "
+                          "time against the weight-only fused per-linear calls"} if "w4a4" in t else None),
         "dense_rotation": ("the contrast the pages draw: a dense d x d bf16 rotation (paro_dense_rotate, tensor "
                            "cores) then the same INT4 linear, per linear; its overhead against the plain per-"
                            "linear INT4 calls sits beside rotation_overhead_per_linear_fused_pct"),

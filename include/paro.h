@@ -176,6 +176,59 @@ PARO_API paro_status paro_w4_linear(const uint16_t* d_x, const uint32_t* d_qweig
                            int group_size, paro_stream_t stream);
 
 /*
+ * Weight-activation (W4A4) variant (page "ParoQuant: Pairwise Rotation
+ * Quantization for Efficient Reasoning LLM Inference", section "Abstract
+ * (arXiv)": the method also matches weight-activation quantization methods).
+ * The pages give no detail of that setting; these calls take 4-bit weights
+ * (the packed INT4 weights of the weight-only calls, unchanged) and 4-bit
+ * activations: the transformed activations quantised per token, symmetrically,
+ * to codes in -8..7.
+ *
+ * paro_quantize_activations: s_x[m] = max_k |x[m][k]| / 7 (1 for an all-zero
+ * row) and q[m][k] = clamp(rint(x[m][k] / s_x[m]), -8, 7), in fp32 IEEE
+ * arithmetic with ties to even.  d_x: bf16 [M][d], 16-byte aligned, d % 8 == 0;
+ * d_q: int8 [M][d], one code per byte in column order; d_sx: fp32 [M].  The
+ * outputs must not overlap d_x.
+ */
+PARO_API paro_status paro_quantize_activations(const uint16_t* d_x, int8_t* d_q, float* d_sx, int M, int d,
+                                               paro_stream_t stream);
+
+/*
+ * Bytes of device workspace the W4A4 calls take: fp32 partial sums of the
+ * linear (0 when it needs none), and with with_transform != 0 before them the
+ * bf16 transformed activations, their codes and their scales of
+ * paro_rotate_w4a4_linear (each part rounded up to 256 bytes).
+ */
+PARO_API size_t paro_w4a4_workspace_bytes(int M, int d_in, int d_out, int with_transform);
+
+/*
+ * W4A4 linear: y[m][n] = s_x[m] * sum_g s_w[n][g] * sum_{k in g}
+ * (q_w[n][k] - z[n][g]) * q_x[m][k], the inner sums exact integers, the rest
+ * fp32, bf16 output (round to nearest even).  d_q: int8 [M][d_in] codes in
+ * -8..7, 16-byte aligned; d_sx: fp32 [M]; weights as paro_w4_linear; d_y: bf16
+ * [M][d_out], overlapping no input.  d_workspace: paro_w4a4_workspace_bytes(M,
+ * d_in, d_out, 0) bytes, 256-byte aligned (may be null when that is 0).
+ */
+PARO_API paro_status paro_w4a4_linear(const int8_t* d_q, const float* d_sx, const uint32_t* d_qweight,
+                                      const uint16_t* d_scales, const uint16_t* d_zeros, uint16_t* d_y, int M,
+                                      int d_in, int d_out, int group_size, void* d_workspace,
+                                      size_t workspace_bytes, paro_stream_t stream);
+
+/*
+ * The whole W4A4 path of one linear: the activation transform (as
+ * paro_rotate, bf16 x~ into the workspace), its per-token codes (as
+ * paro_quantize_activations) and the W4A4 linear, three launches on `stream`.
+ * Arguments as paro_rotate_w4_linear; d_workspace: paro_w4a4_workspace_bytes(M,
+ * d_in, d_out, 1) bytes, 256-byte aligned, overlapping nothing else.
+ */
+PARO_API paro_status paro_rotate_w4a4_linear(const uint16_t* d_x, int K, const uint16_t* d_pairs,
+                                             const float* d_cos, const float* d_sin, const float* d_scale,
+                                             const uint32_t* d_qweight, const uint16_t* d_scales,
+                                             const uint16_t* d_zeros, uint16_t* d_y, int M, int d_in, int d_out,
+                                             int group_size, void* d_workspace, size_t workspace_bytes,
+                                             paro_stream_t stream);
+
+/*
  * Host-side, once per layer (no GPU involved): reorders the pairs inside every
  * stage, flipping some (i, j, cos, sin) into the same rotation (j, i, cos, -sin),
  * so that every aligned group of 32 consecutive pairs touches 32 different

@@ -20,6 +20,7 @@ __all__ = [
     "paro_rotate_w4_linear_noalloc", "paro_get_device_status", "EXPORTED", "ParoLinear", "paro_linear",
     "paro_batched_workspace_bytes", "paro_rotate_w4_linear_batched", "paro_plan_pair_order",
     "paro_rotate_backward_workspace_bytes", "paro_rotate_backward", "paro_set_test_hooks", "paro_dense_rotate",
+    "paro_quantize_activations", "paro_w4a4_linear", "paro_rotate_w4a4_linear",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libparo.so")
@@ -44,6 +45,10 @@ EXPORTED = {
     "paro_rotate_backward": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
     "paro_set_test_hooks": (_I, [ctypes.c_longlong, _I]),
     "paro_dense_rotate": (_I, [_P, _P, _P, _I, _I, _P]),
+    "paro_quantize_activations": (_I, [_P, _P, _P, _I, _I, _P]),
+    "paro_w4a4_workspace_bytes": (_S, [_I, _I, _I, _I]),
+    "paro_w4a4_linear": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
+    "paro_rotate_w4a4_linear": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
 }
 
 
@@ -183,6 +188,57 @@ def paro_dense_rotate(x: torch.Tensor, q: torch.Tensor, *, out=None, stream=None
         out = torch.empty_like(x)
     st = lib.paro_dense_rotate(_ptr(_u16(x)), _ptr(_u16(q)), _ptr(_u16(out)), M, d, _stream(stream))
     _check(st, "paro_dense_rotate")
+    return out
+
+
+def paro_quantize_activations(x: torch.Tensor, *, q=None, sx=None, stream=None):
+    """Per-token symmetric INT4 codes of bf16 x [M, d]: (codes int8 [M, d] in -8..7, scales fp32 [M])."""
+    M, d = x.shape
+    if q is None:
+        q = torch.empty(M, d, dtype=torch.int8, device=x.device)
+    if sx is None:
+        sx = torch.empty(M, dtype=torch.float32, device=x.device)
+    st = lib.paro_quantize_activations(_ptr(_u16(x)), _ptr(q), _ptr(sx), M, d, _stream(stream))
+    _check(st, "paro_quantize_activations")
+    return q, sx
+
+
+def _w4a4_ws(M, d_in, d_out, with_transform, workspace, dev):
+    need = int(lib.paro_w4a4_workspace_bytes(M, d_in, d_out, with_transform))
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    return workspace, need
+
+
+def paro_w4a4_linear(q: torch.Tensor, sx: torch.Tensor, qweight, scales, zeros, *, out=None, workspace=None,
+                     group_size: int = 128, stream=None):
+    """The W4A4 linear on activation codes q (int8 [M, d_in]) and scales sx (fp32 [M]); bf16 [M, d_out]."""
+    M, d_in = q.shape
+    d_out = qweight.shape[0]
+    if out is None:
+        out = torch.empty(M, d_out, dtype=torch.bfloat16, device=q.device)
+    workspace, need = _w4a4_ws(M, d_in, d_out, 0, workspace, q.device)
+    st = lib.paro_w4a4_linear(_ptr(q), _ptr(sx), _ptr(qweight), _ptr(_u16(scales)), _ptr(_u16(zeros)),
+                              _ptr(_u16(out)), M, d_in, d_out, group_size, _ptr(workspace) if need else None,
+                              workspace.numel() if need else 0, _stream(stream))
+    _check(st, "paro_w4a4_linear")
+    return out
+
+
+def paro_rotate_w4a4_linear(x: torch.Tensor, pairs, cos_t, sin_t, scale, qweight, scales, zeros, *, out=None,
+                            workspace=None, group_size: int = 128, stream=None):
+    """The W4A4 path of one linear: transform, per-token INT4 codes, W4A4 linear; bf16 [M, d_out].
+    The workspace (returned by paro_w4a4_workspace_bytes(M, d_in, d_out, 1)) holds x~ in bf16
+    first, then its codes and scales."""
+    M, d_in = x.shape
+    d_out = qweight.shape[0]
+    if out is None:
+        out = torch.empty(M, d_out, dtype=torch.bfloat16, device=x.device)
+    workspace, need = _w4a4_ws(M, d_in, d_out, 1, workspace, x.device)
+    st = lib.paro_rotate_w4a4_linear(_ptr(_u16(x)), _K(pairs), _ptr(pairs), _ptr(cos_t), _ptr(sin_t), _ptr(scale),
+                                     _ptr(qweight), _ptr(_u16(scales)), _ptr(_u16(zeros)), _ptr(_u16(out)), M, d_in,
+                                     d_out, group_size, _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "paro_rotate_w4a4_linear")
     return out
 
 

@@ -21,7 +21,7 @@ COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler",
           "-I", os.path.join(ROOT, "include"), "--expt-relaxed-constexpr"]
 # Files whose results must be bit-exact with an IEEE reference compile without FMA contraction.
 PER_FILE = {"pack.cu": ["-fmad=false"]}
-SOURCES = ["api.cu", "rotate.cu", "rotate_decode.cu", "rotate_backward.cu", "pack.cu", "w4_gemv.cu", "w4_tc.cu", "w4_stream.cu", "plan.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "rotate.cu", "rotate_decode.cu", "rotate_backward.cu", "pack.cu", "w4_gemv.cu", "w4_tc.cu", "w4_stream.cu", "plan.cu", "noalloc.cu", "w4a4.cu"]
 
 
 def nvcc() -> str:

@@ -692,6 +692,101 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
   return from_cuda(e, "batched w4 linear launch");
 }
 
+// ---- weight-activation (W4A4) variant ----------------------------------------------
+namespace {
+size_t r256(size_t b) { return (b + 255) & ~(size_t)255; }
+size_t w4a4_front_bytes(int M, int d_in) {
+  return r256((size_t)M * d_in * 2) + r256((size_t)M * d_in) + r256((size_t)M * 4);
+}
+}  // namespace
+
+size_t paro_w4a4_workspace_bytes(int M, int d_in, int d_out, int with_transform) {
+  if (M <= 0 || d_in <= 0 || d_out <= 0) return 0;
+  const size_t part = paro::w4a4_partial_bytes(M, d_in, d_out, paro::device_sm_count());
+  return (with_transform ? w4a4_front_bytes(M, d_in) : 0) + part;
+}
+
+paro_status paro_quantize_activations(const uint16_t* d_x, int8_t* d_q, float* d_sx, int M, int d,
+                                      paro_stream_t stream) {
+  if (M < 0) return fail(PARO_ERR_INVALID_ARG, "M = %d is negative", M);
+  if (d <= 0 || d % 8) return fail(PARO_ERR_INVALID_ARG, "d = %d must be a positive multiple of 8", d);
+  if (M == 0) return ok();
+  if (!d_x || !d_q || !d_sx) return fail(PARO_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(d_x, 16) || !aligned(d_q, 8) || !aligned(d_sx, 4))
+    return fail(PARO_ERR_INVALID_ARG, "x must be 16-byte, q 8-byte and sx 4-byte aligned");
+  const size_t xb = (size_t)M * d * 2;
+  if (overlap(d_q, (size_t)M * d, d_x, xb) || overlap(d_sx, (size_t)M * 4, d_x, xb) ||
+      overlap(d_q, (size_t)M * d, d_sx, (size_t)M * 4))
+    return fail(PARO_ERR_INVALID_ARG, "x, q and sx must not overlap");
+  return from_cuda(paro::launch_quantize_act(d_x, d_q, d_sx, M, d, reinterpret_cast<cudaStream_t>(stream)),
+                   "quantize launch");
+}
+
+paro_status paro_w4a4_linear(const int8_t* d_q, const float* d_sx, const uint32_t* d_qweight,
+                             const uint16_t* d_scales, const uint16_t* d_zeros, uint16_t* d_y, int M, int d_in,
+                             int d_out, int group_size, void* d_workspace, size_t workspace_bytes,
+                             paro_stream_t stream) {
+  paro_status st;
+  if ((st = check_linear_shape(M, d_in, d_out, group_size)) != PARO_OK) return st;
+  if (M == 0) return ok();
+  if ((st = check_weights(d_qweight, d_scales, d_zeros)) != PARO_OK) return st;
+  if (!d_q || !d_sx || !d_y) return fail(PARO_ERR_INVALID_ARG, "null activation pointer");
+  if (!aligned(d_q, 16) || !aligned(d_sx, 4) || !aligned(d_y, 2))
+    return fail(PARO_ERR_INVALID_ARG, "q must be 16-byte aligned, sx 4-byte, y 2-byte");
+  const int sms = paro::device_sm_count();
+  const int shares = paro::w4a4_shares(d_in, d_out, sms);
+  const size_t need = paro::w4a4_partial_bytes(M, d_in, d_out, sms);
+  if (need && (!d_workspace || workspace_bytes < need || !aligned(d_workspace, 256)))
+    return fail(PARO_ERR_INVALID_ARG, "workspace must be 256-byte aligned and hold %zu bytes", need);
+  const size_t yb = (size_t)M * d_out * 2;
+  if (overlap(d_y, yb, d_q, (size_t)M * d_in) || overlap(d_y, yb, d_sx, (size_t)M * 4) ||
+      overlap(d_y, yb, d_qweight, (size_t)d_out * d_in / 2) || (need && overlap(d_y, yb, d_workspace, need)))
+    return fail(PARO_ERR_INVALID_ARG, "y must not overlap an input or the workspace");
+  cudaError_t e = paro::launch_w4a4(d_q, d_sx, d_qweight, d_scales, d_zeros, d_y, M, d_in, d_out,
+                                    static_cast<float*>(need ? d_workspace : nullptr), shares,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  return from_cuda(e, "w4a4 linear launch");
+}
+
+paro_status paro_rotate_w4a4_linear(const uint16_t* d_x, int K, const uint16_t* d_pairs, const float* d_cos,
+                                    const float* d_sin, const float* d_scale, const uint32_t* d_qweight,
+                                    const uint16_t* d_scales, const uint16_t* d_zeros, uint16_t* d_y, int M,
+                                    int d_in, int d_out, int group_size, void* d_workspace, size_t workspace_bytes,
+                                    paro_stream_t stream) {
+  paro_status st;
+  if ((st = check_linear_shape(M, d_in, d_out, group_size)) != PARO_OK) return st;
+  if ((st = check_width(d_in)) != PARO_OK) return st;
+  if ((st = check_tables(K, d_in, d_pairs, d_cos, d_sin, d_scale)) != PARO_OK) return st;
+  if (M == 0) return ok();
+  if ((st = check_weights(d_qweight, d_scales, d_zeros)) != PARO_OK) return st;
+  if (!d_x || !d_y) return fail(PARO_ERR_INVALID_ARG, "null activation pointer");
+  if (!aligned(d_x, 16) || !aligned(d_y, 16)) return fail(PARO_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
+  const size_t need = paro_w4a4_workspace_bytes(M, d_in, d_out, 1);
+  if (!d_workspace || workspace_bytes < need || !aligned(d_workspace, 256))
+    return fail(PARO_ERR_INVALID_ARG, "workspace must be 256-byte aligned and hold %zu bytes", need);
+  const size_t yb = (size_t)M * d_out * 2, xb = (size_t)M * d_in * 2;
+  if (overlap(d_y, yb, d_x, xb) || overlap(d_y, yb, d_workspace, need) || overlap(d_workspace, need, d_x, xb) ||
+      overlap(d_y, yb, d_qweight, (size_t)d_out * d_in / 2))
+    return fail(PARO_ERR_INVALID_ARG, "y, x and workspace must not overlap");
+  int* status = status_ptr();
+  if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
+  char* ws = static_cast<char*>(d_workspace);
+  uint16_t* xt = reinterpret_cast<uint16_t*>(ws);
+  int8_t* q = reinterpret_cast<int8_t*>(ws + r256(xb));
+  float* sx = reinterpret_cast<float*>(ws + r256(xb) + r256((size_t)M * d_in));
+  float* part = reinterpret_cast<float*>(ws + w4a4_front_bytes(M, d_in));
+  const int sms = paro::device_sm_count();
+  const int shares = paro::w4a4_shares(d_in, d_out, sms);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_transform(d_x, xt, false, M, d_in, K, d_pairs, d_cos, d_sin, d_scale, status, s, false);
+  if (e != cudaSuccess) return from_cuda(e, "rotate launch");
+  e = paro::launch_quantize_act(xt, q, sx, M, d_in, s);
+  if (e != cudaSuccess) return from_cuda(e, "quantize launch");
+  e = paro::launch_w4a4(q, sx, d_qweight, d_scales, d_zeros, d_y, M, d_in, d_out, shares > 1 ? part : nullptr,
+                        shares, s);
+  return from_cuda(e, "w4a4 linear launch");
+}
+
 paro_status paro_get_device_status(paro_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return from_cuda(e, "stream synchronize");

@@ -65,4 +65,16 @@ cudaError_t launch_fold_weights(const float* W, float* out, int rows, int d, int
 cudaError_t launch_quantize_pack(const float* Wt, int d_out, int d_in, uint32_t* qweight,
                                  __half* scales, __half* zeros, cudaStream_t stream);
 
+// The weight-activation variant (w4a4.cu): per-token INT4 codes of bf16
+// activations [M][d] (d % 8 == 0, 16-byte aligned rows), and the INT4 x INT4
+// linear.  The linear splits each 64-row tile's groups into w4a4_shares(...)
+// shares; with more than one it needs w4a4_partial_bytes(...) of fp32 partials
+// and a second, ordered reduction launch.
+int w4a4_shares(int d_in, int d_out, int sms);
+size_t w4a4_partial_bytes(int M, int d_in, int d_out, int sms);
+cudaError_t launch_quantize_act(const uint16_t* x, int8_t* q, float* sx, int M, int d, cudaStream_t stream);
+cudaError_t launch_w4a4(const int8_t* qx, const float* sx, const uint32_t* qw, const uint16_t* sw,
+                        const uint16_t* zw, uint16_t* y, int M, int d_in, int d_out, float* part, int shares,
+                        cudaStream_t stream);
+
 }  // namespace paro
