@@ -114,3 +114,32 @@ def test_fp16_overflow_of_bf16_inputs_on_the_tensor_cores_is_reported():
     assert paro.paro_get_device_status() == RANGE
     paro.paro_w4_linear(torch.from_numpy(p.x).to(DEV).to(torch.bfloat16), qw, sc, z)
     assert paro.paro_get_device_status() == 0
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_bad_pair_index_in_a_layer_is_reported_and_others_are_correct(M):
+    # a channel index >= d in one linear's tables: the transform clamps it into
+    # range (every access stays inside the rows) and reports
+    # PARO_ERR_INVALID_ARG (that linear's result is void), but still hands its
+    # x~ over, so the call ends at once (no bounded wait runs out) and every
+    # other linear of the call is correct
+    shapes = [(1536, 256), (8960, 1536), (1536, 512)]
+    probs, devs, layers = _layer(331 + M, shapes, M)
+    bad = probs[1].pairs.copy()
+    bad[4, 100, 0] = 9000  # >= d = 8960, in stage 4
+    devs[1]["tables"] = (torch.from_numpy(bad.view(np.int16)).to(DEV),) + devs[1]["tables"][1:]
+    layers = [paro.paro_linear(d["x"], *d["tables"], d["qw"], d["sc"], d["z"], d["y"]) for d in devs]
+    assert paro.paro_get_device_status() == 0
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    paro.paro_rotate_w4_linear_batched(layers)
+    end.record()
+    torch.cuda.synchronize()
+    assert start.elapsed_time(end) < 100.0  # milliseconds: no wait ran to its bound
+    assert paro.paro_get_device_status() == 1  # PARO_ERR_INVALID_ARG
+    for i in (0, 2):
+        p, d = probs[i], devs[i]
+        ref = oracle.rotate_w4_linear(p.x, p.pairs, p.cos_t, p.sin_t, p.scale,
+                                      d["qw"].cpu().numpy().view(np.uint32), d["sc"].cpu().numpy(),
+                                      d["z"].cpu().numpy())
+        assert_linear_close(d["y"].float().cpu().numpy(), ref)
