@@ -679,8 +679,9 @@ def sub_record(r, world, hbm, bf16, bf16_sus):
         rec.update(value=round(tf, 2), unit="TFLOP/s", frac_of_bf16=round(tf / bf16, 4))
         if "batched_plain" in t:
             tp = flops / (t["batched_plain"].ms * 1e-3) / 1e12
-            rec["roofline"] = {"bound": "tensor", "kernel": "w4_tc_kernel (tcgen05; one launch per step, plain "
-                                                            "weights, bf16 inputs rounded to fp16 in the kernel)",
+            rec["roofline"] = {"bound": "tensor", "kernel": "w4_tc_kernel (tcgen05) on plain weights: the step "
+                                                            "is one bf16->fp16 rounding launch into the workspace "
+                                                            "and one tensor-core launch; 2*M*d_in*d_out / step time",
                                "achieved": round(tp, 2), "peak": bf16, "unit": "TFLOP/s", "frac": round(tp / bf16, 4),
                                "peak_sustained": bf16_sus,
                                "frac_of_sustained": round(tp / bf16_sus, 4) if bf16_sus else None,

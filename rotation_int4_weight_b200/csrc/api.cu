@@ -576,14 +576,27 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
   if (!status) return fail(PARO_ERR_CUDA, "no CUDA device / status word unavailable");
   if (!any_transform) {
     // many tokens and no layer has a transform: when the tensor-core kernel takes
-    // every linear, one launch rounds the bf16 inputs to fp16 tiles itself
+    // every linear, one launch rounds every bf16 input to fp16 into the
+    // workspace and the tensor-core kernel reads them by TMA (converting each
+    // tile inside that kernel instead costs it a third more time: the
+    // conversion competes with the dequantisation for shared memory)
     bool all_tc = true;
     paro::TcLinear tl[PARO_MAX_BATCH];
+    const uint16_t* src[PARO_MAX_BATCH];
+    uint16_t* dst[PARO_MAX_BATCH];
+    size_t cnt[PARO_MAX_BATCH];
     for (int i = 0; i < n && all_tc; ++i) {
-      all_tc = rp[i].M >= kTensorCoreMinM && paro::tc_supported(rp[i].M, rp[i].d, gp[i].d_out, rp[i].x);
-      tl[i] = paro::TcLinear{rp[i].x, gp[i].qw, gp[i].sc, gp[i].z, gp[i].y, gp[i].M, gp[i].d_in, gp[i].d_out};
+      all_tc = rp[i].M >= kTensorCoreMinM && paro::tc_supported(rp[i].M, rp[i].d, gp[i].d_out, gp[i].x);
+      tl[i] = paro::TcLinear{gp[i].x, gp[i].qw, gp[i].sc, gp[i].z, gp[i].y, gp[i].M, gp[i].d_in, gp[i].d_out};
+      src[i] = rp[i].x;
+      dst[i] = static_cast<uint16_t*>(rp[i].out);
+      cnt[i] = (size_t)rp[i].M * rp[i].d;
     }
-    if (all_tc) return from_cuda(paro::launch_w4_tc_batch(tl, n, false, status, s), "batched w4 linear launch");
+    if (all_tc) {
+      e = paro::launch_to_f16(src, dst, cnt, n, status, s);
+      if (e == cudaSuccess) e = paro::launch_w4_tc_batch(tl, n, true, status, s);
+      return from_cuda(e, "batched w4 linear launch");
+    }
   }
   // the widest linear (the slowest transform) last, so that its units go to the
   // INT4 grid's last CTAs

@@ -540,6 +540,70 @@ bool tc_supported(int M, int d_in, int d_out, const void* x) {
          ((size_t)d_in * 2) % 16 == 0;
 }
 
+namespace {
+struct ConvBatch {
+  const uint4* src[kMaxBatch];
+  uint4* dst[kMaxBatch];
+  size_t begin[kMaxBatch + 1];  // prefix sums of the arrays' 8-value chunks
+  int count;
+};
+
+__global__ void __launch_bounds__(256) to_f16_kernel(const __grid_constant__ ConvBatch b, int* status) {
+  // every thread takes four chunks 'stride' apart per round, their loads issued
+  // before any is converted, so that enough bytes are in flight
+  const size_t total = b.begin[b.count], stride = (size_t)gridDim.x * blockDim.x;
+  bool ovf = false;
+  for (size_t i0 = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i0 < total; i0 += 4 * stride) {
+    uint4 v[4];
+    int a[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const size_t i = i0 + u * stride;
+      a[u] = 0;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (i < total) {
+        while (a[u] + 1 < b.count && i >= b.begin[a[u] + 1]) ++a[u];
+        v[u] = __ldcs(b.src[a[u]] + (i - b.begin[a[u]]));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const size_t i = i0 + u * stride;
+      if (i >= total) continue;
+      uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+        const __half2 h = __floats2half2_rn(f.x, f.y);
+        w[e] = *reinterpret_cast<const uint32_t*>(&h);
+        ovf |= half2_inf(w[e]);
+      }
+      b.dst[a[u]][i - b.begin[a[u]]] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  if (ovf) report_status(status, kStatusRange);
+}
+}  // namespace
+
+cudaError_t launch_to_f16(const uint16_t* const* src, uint16_t* const* dst, const size_t* n, int count, int* status,
+                          cudaStream_t stream) {
+  if (count < 1 || count > kMaxBatch) return cudaErrorInvalidValue;
+  ConvBatch b = {};
+  b.count = count;
+  for (int i = 0; i < count; ++i) {
+    if (n[i] % 8 || (reinterpret_cast<uintptr_t>(src[i]) | reinterpret_cast<uintptr_t>(dst[i])) & 15)
+      return cudaErrorInvalidValue;
+    b.src[i] = reinterpret_cast<const uint4*>(src[i]);
+    b.dst[i] = reinterpret_cast<uint4*>(dst[i]);
+    b.begin[i + 1] = b.begin[i] + n[i] / 8;
+  }
+  const size_t chunks = b.begin[count];
+  if (chunks == 0) return cudaSuccess;
+  const size_t want = (chunks + 1023) / 1024, cap = (size_t)device_sm_count() * 8;
+  to_f16_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, stream>>>(b, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_w4_tc_batch(const TcLinear* lins, int count, bool x_f16, int* status, cudaStream_t stream) {
   if (count < 1 || count > kTcMaxBatch) return cudaErrorInvalidValue;
   EncodeTiled enc = encode_fn();

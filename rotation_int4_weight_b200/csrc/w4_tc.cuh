@@ -47,6 +47,15 @@ bool tc_supported(int M, int d_in, int d_out, const void* x);
 // One persistent launch over up to kTcMaxBatch linears: a CTA per SM walks the
 // 256 x 256 output tiles of all of them, the linears with the longest K first.
 cudaError_t launch_w4_tc_batch(const TcLinear* lins, int count, bool x_f16, int* status, cudaStream_t stream);
+// bf16 -> fp16 (round to nearest) of up to kMaxBatch arrays in one launch,
+// n[i] values each (a multiple of 8, 16-byte aligned arrays); a value beyond
+// the fp16 range is reported as PARO_ERR_RANGE.  The plain (untransformed)
+// linears of a batched call with many tokens take this pass into the
+// workspace and the tensor-core kernel's fp16 path, rather than converting
+// each tile in the kernel, where the conversion competes with the
+// dequantisation for shared memory.
+cudaError_t launch_to_f16(const uint16_t* const* src, uint16_t* const* dst, const size_t* n, int count, int* status,
+                          cudaStream_t stream);
 
 // The dense-rotation contrast: y = x Q^T for bf16 x [M][d] and a bf16 d x d
 // matrix Q (row n = output channel n), on the same tensor-core pipeline with
