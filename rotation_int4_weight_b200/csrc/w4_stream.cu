@@ -313,8 +313,12 @@ __device__ __forceinline__ unsigned long long launch_tag(const unsigned long lon
   asm volatile("ld.acquire.gpu.global.u64 %0, [%1];\n" : "=l"(e) : "l"(ctl) : "memory");
   return 2ull * e + 1ull;
 }
-// Every CTA of a launch that has a workspace calls this once, last: the CTA
-// that completes the count advances the epoch (the count wraps back to zero).
+// Every CTA of a launch that has a workspace counts itself once, after it has
+// read the epoch: the CTA that completes the count advances the epoch (the
+// count wraps back to zero).  The INT4 CTAs count themselves after their units
+// (inline in the kernel, so that the count's round trip overlaps their
+// combine); a transform CTA of the fused form, or a CTA that gave up, calls
+// this at its end.
 __device__ __forceinline__ void finish_cta(unsigned long long* ctl) {
   if (!ctl) return;
   __syncthreads();
@@ -510,7 +514,10 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   // (the flag form orders everything after the transform's flags instead: the
   // transform waited for the previous launch before it published any)
   if (FU >= 0 && pdl_wait) asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  if (FU >= 0 && b.ctl) ltag = launch_tag(b.ctl);
+  // the fused form compares the transforms' flags with the launch tag from the
+  // start; the plain form needs it only for its partial tiles and reads it
+  // after the units (one round trip less before its first activations)
+  if (FU > 0 && b.ctl) ltag = launch_tag(b.ctl);
   // the activations of the unit in slot s (with the slot's arrival; its codes
   // were requested without one)
   auto issue_x = [&](const Cur& c, int s) {
@@ -768,6 +775,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
     finish_cta(b.ctl);
     return;
   }
+  if (FU == 0 && b.ctl) ltag = launch_tag(b.ctl);
 
   // ---- the last tile, and the partial tiles in shared memory -------------------------
   // slot 0: the warp's first tile when it began before the warp's units;
@@ -816,6 +824,13 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
         sts128f(ring + (uint32_t)(PF * 4) + off, make_float4(acc[rt][m][0], acc[rt][m][1], acc[rt][m][2], acc[rt][m][3]));
     }
   __syncthreads();
+  // every thread of this CTA has read the launch epoch (before the barrier
+  // above), so the CTA counts itself as finished now, for the last CTA of the
+  // launch to advance the epoch; the count's round trip overlaps the combine
+  // (nothing in this launch reads the epoch again, and the next launch reads
+  // it only once this one has completed)
+  unsigned checkin = 0u;
+  if (threadIdx.x == 0 && b.ctl) checkin = atomicInc(reinterpret_cast<unsigned*>(b.ctl + 1), gridDim.x - 1);
 
   // ---- combine: the warp holding a split tile's first unit in this CTA sums the
   // warps' partials in warp order.  A tile that crosses the CTA's bounds then
@@ -907,7 +922,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
         for (int e = 0; e < 4; ++e) tot[rt][m][e] += sum[rt][m][e];
     store_tile<NT>(P, tile, g, t, tot);
   }
-  finish_cta(b.ctl);
+  if (threadIdx.x == 0 && b.ctl && checkin == gridDim.x - 1) atomicAdd(b.ctl, 1ull);
 }
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
