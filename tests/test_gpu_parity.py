@@ -126,7 +126,9 @@ def test_pack_with_fold(cfg, only):
 
 # ---------------------------------------------------------------- rotation
 @pytest.mark.parametrize("M,d", [(1, 512), (3, 512), (4, 512), (5, 1536), (17, 1536), (9, 8960), (2, 14336),
-                                 (7, 130), (33, 4096)])
+                                 (7, 130), (33, 4096),
+                                 # many tokens (the channel-major kernel), ragged last row blocks
+                                 (130, 14336), (67, 8960), (129, 1536)])
 def test_rotate_parity(M, d):
     p = linear_problem(31, M * 1000 + d, d, 16, M)
     x = dev_x(p.x)
