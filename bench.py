@@ -54,16 +54,18 @@ METRIC = "rot+W4 linear: decode HBM GB/s (% peak), prefill TFLOP/s, rotation ove
 # one ncu capture (metrics dram__bytes_read.sum, dram__bytes_write.sum) of
 #   config 1: `bench.py --profile --variants batched --config 1 --steps 28 --warmup 3 --no-cpu`
 #             (the fused one-launch step; the 21st launch, --set full),
-#   config 3: `... --variants batched_plain --config 3 --steps 4` (the tensor-core launch),
+#   config 3: `... --variants batched,batched_plain --config 3 --steps 2` (the
+#             tensor-core launch on fp16 activations, the same kernel in both
+#             variants; the rounding pass of the plain step is not included),
 #   config 4: `... --variants batched_plain --config 4 --steps 8` (the INT4 launch alone;
 #             the first launch after four skipped),
 # with the sha256 prefix of the kernel's sources at capture time: once the
 # sources change, the figure no longer describes the kernel and the bench
 # reports null.  (Config 2's fused step was not captured.)
 TRAFFIC = {
-    1: {"bytes": 25986560 + 256, "src": ("w4_stream.cu", "w4_stream.cuh", "rotate_decode_cta.cuh"), "sha": "0733fd003a3a3e71"},
-    3: {"bytes": 346587136 + 137527040, "src": ("w4_tc.cu", "w4_tc.cuh"), "sha": "a093d18620409e5a"},
-    4: {"bytes": 25540608, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "69c1f87283208e9b"},
+    1: {"bytes": 25989888 + 1280, "src": ("w4_stream.cu", "w4_stream.cuh", "rotate_decode_cta.cuh"), "sha": "47b89a042eb2210a"},
+    3: {"bytes": 353620736 + 133817088, "src": ("w4_tc.cu", "w4_tc.cuh"), "sha": "58523abd4a64b532"},
+    4: {"bytes": 25540608, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "e3bb6081cd3d8b95"},
 }
 
 
@@ -685,7 +687,8 @@ def sub_record(r, world, hbm, bf16, bf16_sus):
                                "achieved": round(tp, 2), "peak": bf16, "unit": "TFLOP/s", "frac": round(tp / bf16, 4),
                                "peak_sustained": bf16_sus,
                                "frac_of_sustained": round(tp / bf16_sus, 4) if bf16_sus else None,
-                               "traffic": None}
+                               "traffic": measured_traffic(3, None),
+                               "traffic_what": "DRAM bytes of the tensor-core launch (the rounding pass apart)"}
         if "rotate" in t:
             gb = bytes_of(lins, M, "rotate") / (t["rotate"].ms * 1e-3) / 1e9
             rec["rotate_kernel"] = {"gbs": round(gb, 1), "frac_of_hbm": round(gb / hbm, 4),
