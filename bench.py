@@ -17,7 +17,7 @@ roofline  = the step's dominant kernel (at one token per linear the step is a
 sub_records = the rest of the metric: the Llama-3-8B-shaped layer at 2048
             tokens (TFLOP/s of the tensor-core INT4 linear, rotation overhead),
             the 196-linear Qwen2.5-1.5B-shaped stack at 16 tokens, and the
-            Llama-3-8B-shaped layer at one token
+            Llama-3-8B-shaped layer at 1, 4, 8 and 16 tokens
 cpu_baseline = the fp64 CPU oracle on a bounded sample of the same workload
 
 Timing: every timed region is exactly --steps steps, replayed as CUDA graphs
@@ -625,7 +625,7 @@ def bytes_of(step_lins, M, variant):
 
 
 def run_workload(torch, paro, args, config, M_arg, variants, dist, rank, dev, flush, clock_variant=None,
-                 isolated=False, e2e=False, min_seconds=0.25):
+                 isolated=False, e2e=False, min_seconds=0.25, per_linear=False):
     """Build one workload, time its variants; returns a dict of results."""
     name, shapes, M, n_layers, stack = workload(config, M_arg)
     layers = build_layers(config, M, n_layers, rank, dev, plan=not args.no_plan)
@@ -655,6 +655,22 @@ def run_workload(torch, paro, args, config, M_arg, variants, dist, rank, dev, fl
         out["e2e"] = time_plan(torch, plan, args.steps, args.warmup, dist, bytes_of(step_lins, M, "batched"),
                                min_seconds=min_seconds, flush=flush)
         del plan
+    if per_linear and not stack:
+        # each linear of the layer alone: a batched call of that one linear per
+        # step (fused, and plain), cycling over the same layers as above (last:
+        # the units made here take over the linears' x and y views)
+        out["per_linear"] = {}
+        for i, (lname, _, _) in enumerate(shapes):
+            lin_units = [Unit([u.lins[i]], paro) for u in units]
+            rec = {}
+            for v in ("batched", "batched_plain"):
+                plan = chained_plan(torch, paro, lin_units, v, args.steps)
+                sb = bytes_of([step_lins[i]], M, v)
+                tl = time_plan(torch, plan, args.steps, args.warmup, dist, sb, min_seconds=0.1, flush=flush)
+                rec["fused" if v == "batched" else "plain"] = tl
+                del plan
+            out["per_linear"][lname] = (step_lins[i], rec)
+            del lin_units
     return out
 
 
@@ -780,7 +796,7 @@ def main():
     if "batched" not in variants:
         variants.insert(0, "batched")
     head = run_workload(torch, paro, args, args.config, args.M, variants, dist, rank, dev, flush,
-                        clock_variant="batched", isolated=True, e2e=True)
+                        clock_variant="batched", isolated=True, e2e=True, per_linear=True)
     t, M, step_lins, units = head["timed"], head["M"], head["step_lins"], head["units"]
     ms = t["batched"].ms
     step_bytes = bytes_of(step_lins, M, "batched")
@@ -874,13 +890,29 @@ def main():
         "tokens_per_s": round(M * world / (ms * 1e-3), 1),
         "hbm_frac_of_measured": None if prefill else round(value / hbm, 4),
     }
+    if head.get("per_linear") and not prefill:
+        pl = {}
+        for lname, (lin, rec) in head["per_linear"].items():
+            e = {}
+            for k, tl in rec.items():
+                gb = bytes_of([lin], M, "batched" if k == "fused" else "batched_plain") / (tl.ms * 1e-3) / 1e9
+                e[k] = {"us": round(tl.ms * 1e3, 2), "gbs": round(gb, 1), "frac_of_hbm": round(gb / hbm, 4)}
+            if "fused" in e and "plain" in e:
+                e["rotation_overhead_pct"] = round(100 * (e["fused"]["us"] - e["plain"]["us"]) / e["plain"]["us"], 1)
+            pl[lname] = e
+        out["per_linear"] = pl
+        out["per_linear_what"] = ("each linear of the layer alone, one batched call of that linear per step, chained "
+                                  "over the same distinct layers; fused = with its transform, plain = plain weights")
     del head, units, step_lins, t
     torch.cuda.empty_cache()
     if not args.no_sub and args.config == 1 and args.M is None:
         subs = {}
         for key, cfg, m, vs in [("prefill_llama_m2048", 3, None, "batched,batched_plain,rotate,plain,fused,dense"),
                                 ("stack_qwen_196_linears_m16", 4, None, "batched,batched_plain"),
-                                ("decode_llama_m1", 2, 1, "batched,batched_plain")]:
+                                ("decode_llama_m1", 2, 1, "batched,batched_plain"),
+                                ("decode_llama_m4", 2, 4, "batched,batched_plain"),
+                                ("decode_llama_m8", 2, 8, "batched,batched_plain"),
+                                ("decode_llama_m16", 2, 16, "batched,batched_plain")]:
             r = run_workload(torch, paro, args, cfg, m, vs.split(","), dist, rank, dev, flush, min_seconds=0.5)
             subs[key] = sub_record(r, world, hbm, bf16, bf16_sus)
             if cfg == 4:
