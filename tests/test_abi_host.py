@@ -262,3 +262,35 @@ def test_planner_rejects_bad_tables():
     with pytest.raises(paro.ParoError) as e:
         paro.paro_plan_pair_order(pairs2, c2, s2)
     assert e.value.status == UNSUPPORTED
+
+
+@pytest.mark.parametrize("fn,args,expect", [
+    # paro_quantize_activations(x, q, sx, M, d, stream)
+    ("paro_quantize_activations", (A, B, C, 0, 512, None), OK),            # M == 0: nothing enqueued
+    ("paro_quantize_activations", (A, B, C, 2, 12, None), INVALID),        # d % 8
+    ("paro_quantize_activations", (MIS, B, C, 2, 512, None), INVALID),     # x not 16-byte aligned
+    ("paro_quantize_activations", (A, A, C, 2, 512, None), INVALID),       # q overlaps x
+    ("paro_quantize_activations", (None, B, C, 2, 512, None), INVALID),
+    # paro_w4a4_linear(q, sx, qweight, scales, zeros, y, M, d_in, d_out, group, ws, ws_bytes, stream)
+    ("paro_w4a4_linear", (A, B, W, C, D, E, 0, 512, 256, 128, None, 0, None), OK),
+    ("paro_w4a4_linear", (A, B, W, C, D, E, 2, 200, 256, 128, None, 0, None), INVALID),   # d_in % 128
+    ("paro_w4a4_linear", (A, B, W, C, D, E, 2, 512, 250, 128, None, 0, None), UNSUPPORTED),  # d_out % 16
+    ("paro_w4a4_linear", (A, B, W, C, D, E, 2, 512, 256, 64, None, 0, None), UNSUPPORTED),   # group 64
+    ("paro_w4a4_linear", (MIS, B, W, C, D, E, 2, 512, 256, 128, None, 0, None), INVALID),   # q misaligned
+    ("paro_w4a4_linear", (A, B, W, C, D, W, 2, 512, 256, 128, None, 0, None), INVALID),     # y overlaps weights
+])
+def test_w4a4_validation(fn, args, expect):
+    st = getattr(paro.lib, fn)(*args)
+    assert st == expect, (fn, args, paro.lib.paro_last_error())
+
+
+def test_w4a4_workspace_bytes():
+    # the fused call's workspace: bf16 x~, its codes and scales (each rounded up
+    # to 256 bytes), then the linear's fp32 partial sums (0 when it needs none)
+    r = lambda b: (b + 255) // 256 * 256
+    for M, d_in, d_out in [(1, 1536, 1536), (16, 8960, 1536), (3, 512, 96)]:
+        lin = paro.lib.paro_w4a4_workspace_bytes(M, d_in, d_out, 0)
+        fused = paro.lib.paro_w4a4_workspace_bytes(M, d_in, d_out, 1)
+        assert fused == r(2 * M * d_in) + r(M * d_in) + r(4 * M) + lin
+        assert lin % (4 * M * d_out) == 0   # shares x M x d_out fp32 values
+    assert paro.lib.paro_w4a4_workspace_bytes(0, 512, 512, 1) == 0
