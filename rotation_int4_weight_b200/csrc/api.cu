@@ -647,6 +647,15 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
     int R = 1, nt = 1;
     e = paro::plan_rot_batch(rt, n, &rb, &R);
     if (e == cudaSuccess) e = plan_stream(true, 0, &sb, &nt);
+    if (e == cudaSuccess && sb.total_units < 96LL * sb.ctas) {
+      // a short INT4 share per CTA (Qwen2.5-1.5B's layer: about 39 units): the
+      // INT4 launch leaves half as many SMs as the transform has CTAs to it,
+      // so that fewer INT4 CTAs start only when a transform ends (measured:
+      // the 16-token stack 1198 -> 1139 us, 4 tokens 34.1 -> 32.0 us; a long
+      // share, Llama-3-8B's, loses by it: 93 -> 102 us at 16 tokens)
+      const int half_sms = paro::device_sm_count() / 2, res = rb.total_ctas / 2;
+      e = plan_stream(true, res < half_sms ? res : half_sms, &sb, &nt);
+    }
     if (e != cudaSuccess) return from_cuda(e, "batched decode plan");
     // at most 16 rows of at most 8 linears, one row or more a CTA: the flag
     // area always suffices; checked so that no CTA could write past it
