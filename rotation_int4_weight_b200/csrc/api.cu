@@ -670,11 +670,13 @@ paro_status paro_rotate_w4_linear_batched(const paro_linear* h_layers, int count
       sb.p[i].xf_begin = t.cta_begin;
       sb.p[i].xf_count = (t.M + t.rows - 1) / t.rows;
     }
-    // With a long INT4 share per CTA (at least 96 units: Llama-3-8B's layer
-    // has about 180, Qwen2.5-1.5B's 39), the CTAs of the widest linear, whose
-    // transform ends last, take fewer units (measured at 8 and 16 tokens:
-    // Llama 54.3 -> 50.9 and 86.7 -> 79.5 us; Qwen's stack would lose 0.9 %).
-    if (sb.total_units >= 96LL * sb.ctas) paro::set_fused_split(sb, 0.9);
+    // The CTAs of the widest linear, whose transform ends last, take fewer
+    // units: with a long INT4 share per CTA (at least 96 units: Llama-3-8B's
+    // layer has about 180) 1 - 0.9 (w - o) / w of the others' (measured at 8
+    // and 16 tokens: Llama 54.3 -> 50.9 and 86.7 -> 79.5 us), with a short one
+    // (Qwen2.5-1.5B's 39, beside the reserved SMs above) 1 - 0.6 (w - o) / w
+    // (the 16-token stack 1114 -> 1007 us, the layer at 4 tokens 31.3 -> 29.5).
+    paro::set_fused_split(sb, sb.total_units >= 96LL * sb.ctas ? 0.9 : 0.6);
     e = paro::launch_rot_batch(rb, R, true, status, s, true, true);
     if (e == cudaSuccess) e = paro::launch_stream_flagged(sb, nt, status, s);
     return from_cuda(e, "batched decode launch");
