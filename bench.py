@@ -53,7 +53,7 @@ METRIC = "rot+W4 linear: decode HBM GB/s (% peak), prefill TFLOP/s, rotation ove
 # DRAM bytes (read + write) per launch of the kernel the roofline times, from
 # one ncu capture (metrics dram__bytes_read.sum, dram__bytes_write.sum) of
 #   config 1: `bench.py --profile --variants batched --config 1 --steps 28 --warmup 3 --no-cpu`
-#             (the fused one-launch step; the 21st launch, --set full),
+#             (the fused one-launch step; the 21st launch),
 #   config 3: `... --variants batched,batched_plain --config 3 --steps 2` (the
 #             tensor-core launch on fp16 activations, the same kernel in both
 #             variants; the rounding pass of the plain step is not included),
@@ -63,9 +63,9 @@ METRIC = "rot+W4 linear: decode HBM GB/s (% peak), prefill TFLOP/s, rotation ove
 # sources change, the figure no longer describes the kernel and the bench
 # reports null.  (Config 2's fused step was not captured.)
 TRAFFIC = {
-    1: {"bytes": 25989888 + 1280, "src": ("w4_stream.cu", "w4_stream.cuh", "rotate_decode_cta.cuh"), "sha": "47b89a042eb2210a"},
+    1: {"bytes": 25992192 + 0, "src": ("w4_stream.cu", "w4_stream.cuh", "rotate_decode_cta.cuh"), "sha": "3905aa9b1697c651"},
     3: {"bytes": 353620736 + 133817088, "src": ("w4_tc.cu", "w4_tc.cuh"), "sha": "58523abd4a64b532"},
-    4: {"bytes": 25540608, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "e3bb6081cd3d8b95"},
+    4: {"bytes": 25540864 + 0, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "15d03ac2594feb7a"},
 }
 
 
@@ -722,6 +722,63 @@ def sub_record(r, world, hbm, bf16, bf16_sus):
     return rec
 
 
+def run_timeline(torch, args):
+    """Phases of the fused one-token decode launch from the instrumented build
+    (global-timer stamps per CTA; see rotation_int4_weight_b200/_build.py).
+    The last launch of a chain of chained graphs is read back; times are in us
+    from the moment its CTAs' wait for the previous launch ended."""
+    import ctypes
+    import importlib.util
+    pkg = os.path.join(os.path.dirname(os.path.abspath(__file__)), "rotation_int4_weight_b200")
+    spec = importlib.util.spec_from_file_location("_paro_build", os.path.join(pkg, "_build.py"))
+    builder = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(builder)
+    builder.build(timeline=True)
+    os.environ["PARO_TIMELINE"] = "1"
+    import rotation_int4_weight_b200 as paro
+    if not paro.LIB_PATH.endswith("libparo_timeline.so"):
+        raise SystemExit("the package was loaded before --timeline could select the instrumented library")
+    read = paro.lib.paro_timeline_read
+    read.restype, read.argtypes = ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t]
+    dev = torch.device("cuda", 0)
+    name, shapes, M, n_layers, stack = workload(args.config, args.M)
+    if stack or M != 1:
+        raise SystemExit("--timeline covers the fused one-token form: a config at M = 1")
+    layers = build_layers(args.config, M, n_layers, 0, dev, plan=not args.no_plan)
+    units = [Unit(l, paro) for l in layers]
+    seq, distinct = chained_plan(torch, paro, units, "batched", args.steps)
+    for _ in range(args.warmup):
+        for g in seq:
+            g.replay()
+    torch.cuda.synchronize()
+    status = paro.paro_get_device_status()
+    buf = np.zeros(2 * 256 * 8, dtype=np.uint64)
+    rc = read(buf.ctypes.data, buf.nbytes)
+    if rc != 0 or status != 0:
+        raise SystemExit(f"timeline read {rc}, device status {status}")
+    t = buf.reshape(2, 256, 8).astype(np.int64)
+    last = t[0] if t[0, :, 0].max() > t[1, :, 0].max() else t[1]
+    rot = [i for i in range(256) if last[i, 5] == 1]
+    t0 = min(last[i, 1] for i in rot)
+    us = lambda v: round((float(v) - t0) / 1e3, 2)
+    out = {"workload": name, "steps_chained": args.steps, "time_origin": "end of the transform CTAs' wait for "
+           "the previous launch", "transform_ctas": [], "int4_ctas": []}
+    for i in rot:
+        r = last[i]
+        out["transform_ctas"].append({"cta": i, "entry": us(r[0]), "wait_done": us(r[1]), "staged": us(r[2]),
+                                      "stages_done": us(r[3]), "flag": us(r[4])})
+    int4 = np.array([i for i in range(256) if last[i, 5] == 2])
+    for pi in sorted(set(int(v) for v in last[int4, 7])):
+        g = int4[last[int4, 7] == pi]
+        rec = {"last_linear": pi, "ctas": int(len(g)),
+               "units_warp0": [int(last[g, 6].min()), int(last[g, 6].max())]}
+        for k, nm in enumerate(["entry", "wait_done", "first_unit", "units_done", "end"]):
+            col = [us(v) for v in last[g, k]]
+            rec[nm] = {"min": min(col), "median": round(float(np.median(col)), 2), "max": max(col)}
+        out["int4_ctas"].append(rec)
+    print(json.dumps({"timeline": out}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -739,6 +796,10 @@ def main():
     ap.add_argument("--profile", action="store_true",
                     help="run only the listed variants once each (no repetitions, no end-to-end leg, no "
                          "sub-records, no CPU baseline): a short launch sequence for ncu; not bench values")
+    ap.add_argument("--timeline", action="store_true",
+                    help="one-token configs: load the instrumented library (built on first use) and print the "
+                         "global-timer phases of the last fused launch of a chain of steps, per CTA group; "
+                         "not bench values")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -760,6 +821,10 @@ def main():
         dist = tdist
     else:
         torch.cuda.set_device(0)
+    if args.timeline:
+        if world > 1:
+            raise SystemExit("--timeline runs on one GPU")
+        return run_timeline(torch, args)
     import rotation_int4_weight_b200 as paro
     dev = torch.device("cuda", torch.cuda.current_device())
     hbm, bf16, bf16_sus, peak_kind = peaks()

@@ -23,7 +23,10 @@ __all__ = [
     "paro_quantize_activations", "paro_w4a4_linear", "paro_rotate_w4a4_linear",
 ]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libparo.so")
+# PARO_TIMELINE=1 loads the instrumented build (same kernels plus global-timer
+# stamps of the fused one-token decode launch; built by _build.py --timeline)
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libparo_timeline.so" if os.environ.get("PARO_TIMELINE") == "1" else "libparo.so")
 
 # name -> (restype, argtypes) of every entry point of include/paro.h
 _P, _I, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t

@@ -24,6 +24,23 @@
 namespace paro {
 namespace rotdec {
 
+#ifdef PARO_TIMELINE
+// Instrumented build only (rotation_int4_weight_b200/_build.py --timeline): the
+// global timer in ns, and the moments this CTA's transform passed its phases
+// (1 wait for the previous kernel done, 2 rows staged, 3 stages done), kept by
+// thread 0 for the caller to publish.
+__device__ __forceinline__ unsigned long long tl_now() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
+}
+__shared__ unsigned long long tl_rot[4];
+#define PARO_TL_ROT(k) \
+  if (threadIdx.x == 0) tl_rot[k] = tl_now()
+#else
+#define PARO_TL_ROT(k)
+#endif
+
 constexpr int kRotMaxRing = 8;
 constexpr int kRotBars = kRotMaxRing + 1;  // one mbarrier per ring slot, one for the channel scale
 
@@ -177,6 +194,7 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
   // output (which it may still read) wait for it to complete
   if (pdl_wait) asm volatile("griddepcontrol.wait;\n" ::: "memory");
   if (trigger_after_wait) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  PARO_TL_ROT(1);
   // rows -> xs as fp32: each thread two adjacent channels of every row, the
   // loads of LB channel pairs issued before their stores so that their
   // latencies overlap
@@ -210,6 +228,7 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
   // the current one is done, which costs a second barrier per stage.
   if (tid == kProd && K > 0 && ok) ok = mbar_wait_bounded(s_bar, 0u);
   int failed = __syncthreads_or(!ok);  // also: rows staged
+  PARO_TL_ROT(2);
   int issued = ring < K ? ring : K;    // stages requested so far (producer)
   bool scale_issued = P.sscale == 1;   // (producer)
 
@@ -294,6 +313,7 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
       failed = __syncthreads_or(!ok);
     }
   }
+  PARO_TL_ROT(3);
   if (bad) report_status(status, kStatusBadIndex);
   if (failed) {
     // a stage never arrived: report, let the latest copy of every slot land

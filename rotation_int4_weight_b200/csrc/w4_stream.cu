@@ -50,6 +50,24 @@
 #include "w4_stream.cuh"
 #include "rotate_decode_cta.cuh"
 
+#ifdef PARO_TIMELINE
+// Instrumented build only: per CTA of the fused one-token launch, global-timer
+// stamps in ns, in one of two slots chosen by the launch epoch's parity (so the
+// last two launches on a workspace are kept).  A transform CTA writes
+// {entry, wait done, rows staged, stages done, flag published, 1, 0, 0}; an
+// INT4 CTA {entry, wait done, warp 0's first unit landed, units done, end
+// (latest warp), 2, warp 0's units, linear of its last tile}.
+constexpr int kTimelineCtas = 256;
+__device__ unsigned long long g_paro_timeline[2][kTimelineCtas][8];
+extern "C" PARO_API int paro_timeline_read(void* host, size_t bytes) {
+  if (bytes < sizeof(g_paro_timeline)) return (int)PARO_ERR_INVALID_ARG;
+  return cudaMemcpyFromSymbol(host, g_paro_timeline, sizeof(g_paro_timeline)) == cudaSuccess ? 0 : (int)PARO_ERR_CUDA;
+}
+#define PARO_TL_NOW(v) v = rotdec::tl_now()
+#else
+#define PARO_TL_NOW(v)
+#endif
+
 namespace paro {
 namespace {
 
@@ -417,6 +435,10 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   __shared__ __align__(8) uint64_t bars[W * D];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#ifdef PARO_TIMELINE
+  unsigned long long tl_entry = 0, tl_wait = 0, tl_first = 0, tl_loop = 0;
+  PARO_TL_NOW(tl_entry);
+#endif
   // flag form: the preceding transform let this grid launch only after it had
   // waited for the previous launch, so the epoch is already this launch's
   unsigned long long ltag = 0;
@@ -448,6 +470,13 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
         __threadfence();
         __syncthreads();
         if (threadIdx.x == 0 && !rb.skip_flags) st_flag(b.xflags + blockIdx.x, launch_tag(b.ctl));
+#ifdef PARO_TIMELINE
+        if (threadIdx.x == 0 && b.ctl && blockIdx.x < kTimelineCtas) {
+          unsigned long long* o = g_paro_timeline[(launch_tag(b.ctl) >> 1) & 1][blockIdx.x];
+          o[0] = tl_entry; o[1] = rotdec::tl_rot[1]; o[2] = rotdec::tl_rot[2]; o[3] = rotdec::tl_rot[3];
+          o[4] = rotdec::tl_now(); o[5] = 1; o[6] = 0; o[7] = 0;
+        }
+#endif
       }
       finish_cta(b.ctl);
       return;
@@ -518,6 +547,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
   // start; the plain form needs it only for its partial tiles and reads it
   // after the units (one round trip less before its first activations)
   if (FU > 0 && b.ctl) ltag = launch_tag(b.ctl);
+  PARO_TL_NOW(tl_wait);
   // the activations of the unit in slot s (with the slot's arrival; its codes
   // were requested without one)
   auto issue_x = [&](const Cur& c, int s) {
@@ -645,6 +675,9 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
       break;
     }
     ++done;
+#ifdef PARO_TIMELINE
+    if (i == 0) PARO_TL_NOW(tl_first);
+#endif
     const uint32_t sw = ring + (uint32_t)slot * SLOT, sx = sw + kUnitBytes;
     const int mt = P.M;
 
@@ -776,6 +809,7 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
     return;
   }
   if (FU == 0 && b.ctl) ltag = launch_tag(b.ctl);
+  PARO_TL_NOW(tl_loop);
 
   // ---- the last tile, and the partial tiles in shared memory -------------------------
   // slot 0: the warp's first tile when it began before the warp's units;
@@ -923,6 +957,16 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
     store_tile<NT>(P, tile, g, t, tot);
   }
   if (threadIdx.x == 0 && b.ctl && checkin == gridDim.x - 1) atomicAdd(b.ctl, 1ull);
+#ifdef PARO_TIMELINE
+  if (FU > 0 && b.ctl && blockIdx.x < kTimelineCtas) {
+    unsigned long long* o = g_paro_timeline[(ltag >> 1) & 1][blockIdx.x];
+    if (threadIdx.x == 0) {
+      o[0] = tl_entry; o[1] = tl_wait; o[2] = tl_first; o[3] = tl_loop; o[5] = 2;
+      o[6] = (unsigned long long)n; o[7] = (unsigned long long)cur_pi;
+    }
+    if (lane == 0) atomicMax(o + 4, rotdec::tl_now());
+  }
+#endif
 }
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

@@ -44,6 +44,17 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(paro.lib, n)
 
 
+def test_default_library_carries_no_timeline_stamps():
+    # the global-timer stamps exist only in the instrumented build
+    # (_build.py --timeline, loaded with PARO_TIMELINE=1); the library the
+    # package loads by default exports nothing beyond the header
+    assert paro.LIB_PATH.endswith("libparo.so")
+    out = subprocess.run(["nm", "-D", "--defined-only", paro.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (paro_\w+)", out))
+    assert "paro_timeline_read" not in exported
+    assert exported == declared_symbols(), exported ^ declared_symbols()
+
+
 def test_status_strings_and_version():
     assert paro.paro_weight_layout_version() == 1
     for code, name in [(0, "PARO_OK"), (1, "PARO_ERR_INVALID_ARG"), (2, "PARO_ERR_UNSUPPORTED"),
