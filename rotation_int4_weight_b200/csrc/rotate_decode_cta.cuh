@@ -117,9 +117,13 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 // Returns true when the rows were written (uniform over the CTA).
 // trigger_after_wait: let the grid's dependents launch right after the wait
 // for the previous kernel (rather than earlier).
+// epoch, epoch_out: when given, thread 0 reads the launch epoch *epoch right
+// after that wait into *epoch_out, for the caller's flag.
 template <int R, bool F16OUT, int U, int NTHR>
 __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, unsigned char* smem, uint64_t* bars,
-                                               int* status, bool pdl_wait, bool trigger_after_wait = false) {
+                                               int* status, bool pdl_wait, bool trigger_after_wait = false,
+                                               const unsigned long long* epoch = nullptr,
+                                               unsigned long long* epoch_out = nullptr) {
   constexpr int kProd = NTHR - 32;  // the table-fetching thread (lane 0 of the last warp)
   constexpr int kComp = NTHR - 32;  // rotating threads
   const int d = P.d, K = P.K, half = d >> 1, ring = P.ring;
@@ -194,6 +198,12 @@ __device__ __forceinline__ bool rot_decode_cta(const RotProblem& P, int row0, un
   // output (which it may still read) wait for it to complete
   if (pdl_wait) asm volatile("griddepcontrol.wait;\n" ::: "memory");
   if (trigger_after_wait) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  // the epoch is final once the previous kernel has completed, so it is read
+  // now and used only when the flag is written, its latency hidden by the work
+  // between (relaxed: the wait made that kernel's writes visible, and an
+  // acquire would hold back this thread's row loads until it returned)
+  if (epoch && tid == 0)
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];\n" : "=l"(*epoch_out) : "l"(epoch) : "memory");
   PARO_TL_ROT(1);
   // rows -> xs as fp32: each thread two adjacent channels of every row, the
   // loads of LB channel pairs issued before their stores so that their

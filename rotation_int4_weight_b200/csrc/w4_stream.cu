@@ -455,24 +455,28 @@ w4_stream_kernel(const __grid_constant__ StreamBatch b, const __grid_constant__ 
       const RotProblem& Pt = rb.p[blockIdx.x];
       unsigned char* ts = smem_raw + (sbase - smem_u32(smem_raw));
       const int rounds = (Pt.d / 2 + W * 32 - 33) / (W * 32 - 32);
+      // the launch epoch for the flag, read by thread 0 right after the wait
+      // for the previous launch
+      const unsigned long long* ep = b.ctl && !rb.skip_flags ? b.ctl : nullptr;
+      unsigned long long e = 0;
       bool done;
       if (rounds <= 2)
-        done = rotdec::rot_decode_cta<1, true, 2, W * 32>(Pt, 0, ts, tbars, status, pdl_wait != 0);
+        done = rotdec::rot_decode_cta<1, true, 2, W * 32>(Pt, 0, ts, tbars, status, pdl_wait != 0, false, ep, &e);
       else if (rounds <= 5)
-        done = rotdec::rot_decode_cta<1, true, 5, W * 32>(Pt, 0, ts, tbars, status, pdl_wait != 0);
+        done = rotdec::rot_decode_cta<1, true, 5, W * 32>(Pt, 0, ts, tbars, status, pdl_wait != 0, false, ep, &e);
       else if (rounds <= 10)
-        done = rotdec::rot_decode_cta<1, true, 10, W * 32>(Pt, 0, ts, tbars, status, pdl_wait != 0);
+        done = rotdec::rot_decode_cta<1, true, 10, W * 32>(Pt, 0, ts, tbars, status, pdl_wait != 0, false, ep, &e);
       else
-        done = rotdec::rot_decode_cta<1, true, 8, W * 32>(Pt, 0, ts, tbars, status, pdl_wait != 0);
+        done = rotdec::rot_decode_cta<1, true, 8, W * 32>(Pt, 0, ts, tbars, status, pdl_wait != 0, false, ep, &e);
       if (done) {
         // every thread's x~ stores, then the flag (the INT4 CTAs read x~ through
         // the asynchronous proxy after seeing it)
         __threadfence();
         __syncthreads();
-        if (threadIdx.x == 0 && !rb.skip_flags) st_flag(b.xflags + blockIdx.x, launch_tag(b.ctl));
+        if (threadIdx.x == 0 && !rb.skip_flags) st_flag(b.xflags + blockIdx.x, 2ull * e + 1ull);
 #ifdef PARO_TIMELINE
         if (threadIdx.x == 0 && b.ctl && blockIdx.x < kTimelineCtas) {
-          unsigned long long* o = g_paro_timeline[(launch_tag(b.ctl) >> 1) & 1][blockIdx.x];
+          unsigned long long* o = g_paro_timeline[e & 1][blockIdx.x];
           o[0] = tl_entry; o[1] = rotdec::tl_rot[1]; o[2] = rotdec::tl_rot[2]; o[3] = rotdec::tl_rot[3];
           o[4] = rotdec::tl_now(); o[5] = 1; o[6] = 0; o[7] = 0;
         }
