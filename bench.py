@@ -63,9 +63,9 @@ METRIC = "rot+W4 linear: decode HBM GB/s (% peak), prefill TFLOP/s, rotation ove
 # sources change, the figure no longer describes the kernel and the bench
 # reports null.  (Config 2's fused step was not captured.)
 TRAFFIC = {
-    1: {"bytes": 25992192 + 0, "src": ("w4_stream.cu", "w4_stream.cuh", "rotate_decode_cta.cuh"), "sha": "3905aa9b1697c651"},
+    1: {"bytes": 25990656 + 0, "src": ("w4_stream.cu", "w4_stream.cuh", "rotate_decode_cta.cuh"), "sha": "f5a614ede539d503"},
     3: {"bytes": 353620736 + 133817088, "src": ("w4_tc.cu", "w4_tc.cuh"), "sha": "58523abd4a64b532"},
-    4: {"bytes": 25540864 + 0, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "15d03ac2594feb7a"},
+    4: {"bytes": 25540864 + 0, "src": ("w4_stream.cu", "w4_stream.cuh"), "sha": "8c2412e535f4abba"},
 }
 
 
